@@ -1,0 +1,456 @@
+/*
+ * qg_oracle.c -- plain CPU oracle for the quantized linear layer.
+ *
+ * TEST INFRASTRUCTURE.  Only the tests, the smoke check and the bench's
+ * cpu_baseline / reference leg may load this library.  The product path
+ * (the CUDA library and its Python binding) never calls it, and the two
+ * share no source: no headers, no helpers, no constants.
+ *
+ * Every function below is the plain definition of one step, written from the
+ * pages, in this order:
+ *
+ *   affine quantization   x_int = round(x/s) + z ;  x_hat = (x_int - z) * s
+ *       "AI Infra guide, ch.4 Quantization", sec. 1.1 (the quantization math)
+ *   symmetric scale       s = max|x| / 127, z = 0            (same page, sec. 1.2 table)
+ *   asymmetric scale      s = (max - min) / 255, z adjusted  (same page, sec. 1.2 table)
+ *   granularity           per-channel / per-group / per-token (same page, sec. 1.3)
+ *   group-wise INT4, g=128, independent scale + zero per group
+ *       "LLM inference cost: W8A8/W4A8 ...", sec. 2.2 (first technique)
+ *   SmoothQuant           Y = (X diag(s)^-1)(diag(s) W),
+ *                         s_j = max|X_j|^a / max|W_j|^(1-a), a = 0.5
+ *       "AI Infra guide, ch.4 Quantization", sec. 2.2
+ *   weight-only INT4      Y = X * dequant(W)     (same page, sec. 3.1)
+ *   W4A8                  4-bit weights, 8-bit activations, group-wise
+ *       "LLM inference cost: W8A8/W4A8 ...", sec. 2.2
+ *
+ * Readings where the pages are silent (each one is listed in the design notes):
+ *   A  the asymmetric range is widened to include 0: mn' = min(min V, 0),
+ *      mx' = max(max V, 0), so that z lies in [0,15] and 0 is exact;
+ *   B  the 4-bit asymmetric scale divides by 15 = 2^4 - 1 (the page's 255 is 2^8 - 1);
+ *   C  the fp16 scale is rounded toward +infinity, so that s >= r/15 and every
+ *      element keeps the |x - x_hat| <= s/2 bound;
+ *   D  the code is round(x/s) + z in that literal order, ties to even;
+ *   E  8 codes per uint32 along K, low nibble first: packed[kb][n] holds
+ *      k = 8kb .. 8kb+7 of column n;
+ *   F  the W4A16 output dtype equals the activation dtype;
+ *   G  the smoothing statistics come from a separate calibration batch;
+ *   H  X~ = X * inv_s with inv_s = 1/s formed first (one fp32 rounding each);
+ *      W~ = W * s (one fp32 rounding);
+ *   I  symmetric INT4 clamps to [-7, 7] (s = max|w|/7), INT8 to [-127, 127];
+ *   J  a zero range gives scale 0 and all codes 0 (also when the fp32 scale
+ *      underflows to 0).
+ *
+ * Precision: every step that produces a stored integer or a stored scale runs in
+ * IEEE binary32 with round-to-nearest-even (built with -fno-fast-math
+ * -ffp-contract=off; nearbyintf under the default FE_TONEAREST mode).  GEMM
+ * references run in binary64.
+ *
+ * Layouts: row-major everywhere.  X[M][K], W[K][N], Y[M][N]; groups run along K.
+ *
+ * Status codes returned here are the oracle's own: 0 ok, 1 non-finite input,
+ * 2 a scale that does not fit fp16.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define OR_OK 0
+#define OR_NONFINITE 1
+#define OR_RANGE 2
+
+/* ------------------------------------------------------------------------- */
+/* binary16 and bfloat16, decoded and encoded from the IEEE 754 definitions. */
+/* ------------------------------------------------------------------------- */
+
+/* Value of a binary16 bit pattern: 1 sign, 5 exponent (bias 15), 10 fraction. */
+float qgo_f16_to_f32(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int e = (h >> 10) & 0x1F;
+    int f = h & 0x3FF;
+    float v;
+    if (e == 0x1F)
+        v = f ? NAN : INFINITY;
+    else if (e == 0)
+        v = ldexpf((float)f, -24);              /* subnormal: f * 2^-24 */
+    else
+        v = ldexpf((float)(f + 1024), e - 25);  /* (1 + f/2^10) * 2^(e-15) */
+    return sign ? -v : v;
+}
+
+/* Largest binary16 pattern whose magnitude does not exceed a (a >= 0, finite):
+ * rounding toward zero.  Magnitudes at or above 65536 clamp to 65504 (0x7BFF). */
+static uint16_t f16_trunc_mag(float a)
+{
+    if (a >= 65536.0f) return 0x7BFF;
+    if (a >= 0x1p-14f) {
+        int e;
+        float m = frexpf(a, &e);        /* a = m * 2^e, m in [0.5, 1) */
+        /* a = (1 + frac) * 2^(e-1); unbiased exponent e-1, biased e-1+15 */
+        int be = e - 1 + 15;
+        if (be >= 31) return 0x7BFF;
+        /* fraction bits: (2m - 1) * 2^10, truncated */
+        uint32_t frac = (uint32_t)((2.0f * m - 1.0f) * 1024.0f);
+        return (uint16_t)((be << 10) | frac);
+    }
+    /* subnormal range: multiples of 2^-24 */
+    return (uint16_t)(uint32_t)(a * 16777216.0f);
+}
+
+/* binary32 -> binary16, rounding toward +infinity. */
+uint16_t qgo_f32_to_f16_ru(float x)
+{
+    if (isnan(x)) return 0x7E00;
+    if (isinf(x)) return x > 0 ? 0x7C00 : 0xFC00;
+    if (x == 0.0f) return signbit(x) ? 0x8000 : 0x0000;
+    if (x > 0.0f) {
+        uint16_t h = f16_trunc_mag(x);
+        if (qgo_f16_to_f32(h) < x) h = (uint16_t)(h + 1); /* next pattern up; 0x7BFF+1 = +inf */
+        return h;
+    }
+    /* negative: toward +infinity is toward zero in magnitude */
+    return (uint16_t)(0x8000 | f16_trunc_mag(-x));
+}
+
+/* binary32 -> bfloat16 (the upper 16 bits of binary32), round to nearest, ties to even. */
+uint16_t qgo_f32_to_bf16_rn(float x)
+{
+    uint32_t u;
+    memcpy(&u, &x, 4);
+    if (isnan(x)) return (uint16_t)((u >> 16) | 0x0040);
+    uint32_t hi = u >> 16;
+    uint32_t lo = u & 0xFFFF;
+    if (lo > 0x8000 || (lo == 0x8000 && (hi & 1))) hi += 1; /* carries into the exponent */
+    return (uint16_t)hi;
+}
+
+float qgo_bf16_to_f32(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+static int clampi(int v, int lo, int hi) { return v < lo ? lo : (v > hi ? hi : v); }
+
+/* W~[k][n] = W[k][n] * s[k] (reading H), or W itself when s is NULL. */
+static float smoothed(const float* W, const float* s, int64_t N, int64_t k, int64_t n)
+{
+    float w = W[k * N + n];
+    return s ? w * s[k] : w;
+}
+
+/* ------------------------------------------------------------------------- */
+/* O1: group-wise asymmetric INT4 (affine quantization, per-group granularity) */
+/* ------------------------------------------------------------------------- */
+int qgo_quantize_w4_asym(const float* W, const float* s_smooth, int64_t K, int64_t N, int group,
+                         uint8_t* codes, uint16_t* scales_f16, uint8_t* zeros)
+{
+    int64_t G = K / group;
+    int status = OR_OK;
+#pragma omp parallel for schedule(static) reduction(max : status)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t g = 0; g < G; ++g) {
+            float mn = 0.0f, mx = 0.0f; /* reading A: the range always contains 0 */
+            int bad = 0;
+            for (int i = 0; i < group; ++i) {
+                float v = smoothed(W, s_smooth, N, g * group + i, n);
+                if (!isfinite(v)) bad = 1;
+                if (v < mn) mn = v;
+                if (v > mx) mx = v;
+            }
+            if (bad) { status = status > OR_NONFINITE ? status : OR_NONFINITE; continue; }
+            float r = mx - mn;
+            float s32 = r / 15.0f;                    /* reading B */
+            uint16_t s16 = qgo_f32_to_f16_ru(s32);    /* reading C */
+            if (s32 > 65504.0f) { status = OR_RANGE; continue; }
+            float s = qgo_f16_to_f32(s16);
+            int z = 0;
+            if (r == 0.0f) { s16 = 0; s = 0.0f; }
+            else z = clampi((int)nearbyintf(-mn / s), 0, 15);
+            scales_f16[g * N + n] = s16;
+            zeros[g * N + n] = (uint8_t)z;
+            for (int i = 0; i < group; ++i) {
+                int64_t k = g * group + i;
+                int q = 0;
+                if (s != 0.0f) {
+                    float v = smoothed(W, s_smooth, N, k, n);
+                    q = clampi((int)nearbyintf(v / s) + z, 0, 15); /* reading D */
+                }
+                codes[k * N + n] = (uint8_t)q;
+            }
+        }
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------------- */
+/* O1s: group-wise symmetric INT4 (z = 0, s = max|w|/7), codes in [-7, 7]      */
+/* ------------------------------------------------------------------------- */
+int qgo_quantize_w4_sym(const float* W, const float* s_smooth, int64_t K, int64_t N, int group,
+                        int8_t* codes, float* scales)
+{
+    int64_t G = K / group;
+    int status = OR_OK;
+#pragma omp parallel for schedule(static) reduction(max : status)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t g = 0; g < G; ++g) {
+            float amax = 0.0f;
+            int bad = 0;
+            for (int i = 0; i < group; ++i) {
+                float v = smoothed(W, s_smooth, N, g * group + i, n);
+                if (!isfinite(v)) bad = 1;
+                float a = fabsf(v);
+                if (a > amax) amax = a;
+            }
+            if (bad) { status = status > OR_NONFINITE ? status : OR_NONFINITE; continue; }
+            float s = amax / 7.0f;
+            scales[g * N + n] = s;
+            for (int i = 0; i < group; ++i) {
+                int64_t k = g * group + i;
+                int q = 0;
+                if (s != 0.0f) q = clampi((int)nearbyintf(smoothed(W, s_smooth, N, k, n) / s), -7, 7);
+                codes[k * N + n] = (int8_t)q;
+            }
+        }
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------------- */
+/* O2: 8 nibbles per uint32 along K, low nibble first (reading E)              */
+/* ------------------------------------------------------------------------- */
+void qgo_pack_nibbles(const uint8_t* codes, int64_t K, int64_t N, uint32_t* packed)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t kb = 0; kb < K / 8; ++kb)
+        for (int64_t n = 0; n < N; ++n) {
+            uint32_t w = 0;
+            for (int i = 0; i < 8; ++i)
+                w |= (uint32_t)(codes[(8 * kb + i) * N + n] & 0xF) << (4 * i);
+            packed[kb * N + n] = w;
+        }
+}
+
+void qgo_unpack_nibbles(const uint32_t* packed, int64_t K, int64_t N, uint8_t* codes)
+{
+    for (int64_t k = 0; k < K; ++k)
+        for (int64_t n = 0; n < N; ++n)
+            codes[k * N + n] = (uint8_t)((packed[(k / 8) * N + n] >> (4 * (k % 8))) & 0xF);
+}
+
+/* Nibble of packed weight (k, n). */
+static int nib(const uint32_t* packed, int64_t N, int64_t k, int64_t n)
+{
+    return (int)((packed[(k / 8) * N + n] >> (4 * (k % 8))) & 0xF);
+}
+
+/* ------------------------------------------------------------------------- */
+/* O3: W4A16 GEMM reference.  W_deq[k][n] = (q - z) * s (exact in binary64).   */
+/* y[r][n] = sum_k X[m_r][k] * W_deq[k][n] and bound[r][n] = sum_k |X||W_deq|.  */
+/* rows == NULL means every row; otherwise only rows[0..nrows) are computed.   */
+/* ------------------------------------------------------------------------- */
+static double w4_asym_deq(const uint32_t* packed, const uint16_t* scales, const uint8_t* zeros,
+                          int64_t N, int group, int64_t k, int64_t n)
+{
+    int64_t g = k / group;
+    int q = nib(packed, N, k, n);
+    return (double)(q - (int)zeros[g * N + n]) * (double)qgo_f16_to_f32(scales[g * N + n]);
+}
+
+void qgo_gemm_w4a16_ref(const float* X, int64_t M, int64_t K, int64_t N, const uint32_t* packed,
+                        const uint16_t* scales, const uint8_t* zeros, int group,
+                        const int64_t* rows, int64_t nrows, double* y, double* bound)
+{
+    if (!rows) nrows = M;
+    memset(y, 0, sizeof(double) * nrows * N);
+    memset(bound, 0, sizeof(double) * nrows * N);
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            double w = w4_asym_deq(packed, scales, zeros, N, group, k, n);
+            for (int64_t r = 0; r < nrows; ++r) {
+                double x = (double)X[(rows ? rows[r] : r) * K + k];
+                y[r * N + n] += x * w;
+                bound[r * N + n] += fabs(x) * fabs(w);
+            }
+        }
+}
+
+/* ------------------------------------------------------------------------- */
+/* O4: SmoothQuant smoothing factors (reading G: from a calibration batch).    */
+/* s_j = max_m|Xcal[m][j]|^alpha / max_n|W[j][n]|^(1-alpha); inv_s_j = 1/s_j.  */
+/* alpha == 0.5 uses fp32 sqrt and division (both correctly rounded).          */
+/* A zero statistic on either side gives s_j = 1.                              */
+/* ------------------------------------------------------------------------- */
+int qgo_smooth_scales(const float* Xcal, int64_t Mc, const float* W, int64_t K, int64_t N,
+                      float alpha, float* s, float* inv_s)
+{
+    int status = OR_OK;
+#pragma omp parallel for schedule(static) reduction(max : status)
+    for (int64_t j = 0; j < K; ++j) {
+        float ax = 0.0f, aw = 0.0f;
+        for (int64_t m = 0; m < Mc; ++m) {
+            float v = Xcal[m * K + j];
+            if (!isfinite(v)) status = OR_NONFINITE;
+            if (fabsf(v) > ax) ax = fabsf(v);
+        }
+        for (int64_t n = 0; n < N; ++n) {
+            float v = W[j * N + n];
+            if (!isfinite(v)) status = OR_NONFINITE;
+            if (fabsf(v) > aw) aw = fabsf(v);
+        }
+        float sj;
+        if (ax == 0.0f || aw == 0.0f)
+            sj = 1.0f;
+        else if (alpha == 0.5f)
+            sj = sqrtf(ax) / sqrtf(aw);
+        else
+            sj = (float)(pow((double)ax, (double)alpha) / pow((double)aw, 1.0 - (double)alpha));
+        s[j] = sj;
+        inv_s[j] = 1.0f / sj;
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------------- */
+/* O5: per-token dynamic symmetric INT8 activations after smoothing.           */
+/* X~ = X * inv_s; t_m = max_j|X~[m][j]| / 127; q = clamp(round(X~/t_m), +-127) */
+/* ------------------------------------------------------------------------- */
+int qgo_smooth_quant_act_i8(const float* X, int64_t M, int64_t K, const float* inv_s,
+                            int8_t* Xq, float* t)
+{
+    int status = OR_OK;
+#pragma omp parallel for schedule(static) reduction(max : status)
+    for (int64_t m = 0; m < M; ++m) {
+        float a = 0.0f;
+        for (int64_t j = 0; j < K; ++j) {
+            float v = inv_s ? X[m * K + j] * inv_s[j] : X[m * K + j];
+            if (!isfinite(v)) status = OR_NONFINITE;
+            if (fabsf(v) > a) a = fabsf(v);
+        }
+        float tm = a / 127.0f;
+        t[m] = tm;
+        for (int64_t j = 0; j < K; ++j) {
+            float v = inv_s ? X[m * K + j] * inv_s[j] : X[m * K + j];
+            int q = 0;
+            if (tm != 0.0f && isfinite(v)) q = clampi((int)nearbyintf(v / tm), -127, 127);
+            Xq[m * K + j] = (int8_t)q;
+        }
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------------- */
+/* O6: per-output-channel symmetric INT8 weights on W~ = diag(s) W.            */
+/* sw_n = max_k|W~[k][n]| / 127; q = clamp(round(W~/sw_n), +-127)             */
+/* ------------------------------------------------------------------------- */
+int qgo_quantize_w8_channel(const float* W, const float* s_smooth, int64_t K, int64_t N,
+                            int8_t* Wq, float* sw)
+{
+    int status = OR_OK;
+#pragma omp parallel for schedule(static) reduction(max : status)
+    for (int64_t n = 0; n < N; ++n) {
+        float a = 0.0f;
+        for (int64_t k = 0; k < K; ++k) {
+            float v = smoothed(W, s_smooth, N, k, n);
+            if (!isfinite(v)) status = OR_NONFINITE;
+            if (fabsf(v) > a) a = fabsf(v);
+        }
+        float s = a / 127.0f;
+        sw[n] = s;
+        for (int64_t k = 0; k < K; ++k) {
+            int q = 0;
+            float v = smoothed(W, s_smooth, N, k, n);
+            if (s != 0.0f && isfinite(v)) q = clampi((int)nearbyintf(v / s), -127, 127);
+            Wq[k * N + n] = (int8_t)q;
+        }
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------------- */
+/* O7: W8A8 GEMM.  acc = sum_k qx*qw (exact integer);                          */
+/* Y = bf16_rn(((float)acc * t_m) * sw_n); reference = fp64 dot of the        */
+/* dequantized operands (qx*t_m)(qw*sw_n) and its absolute-value bound.         */
+/* acc, y_bf16, yref, bound are [nrows][N]; any of acc / y_bf16 may be NULL.   */
+/* ------------------------------------------------------------------------- */
+void qgo_gemm_w8a8(const int8_t* Xq, const float* t, int64_t M, int64_t K, const int8_t* Wq,
+                   const float* sw, int64_t N, const int64_t* rows, int64_t nrows,
+                   int32_t* acc, uint16_t* y_bf16, double* yref, double* bound)
+{
+    if (!rows) nrows = M;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t r = 0; r < nrows; ++r) {
+            int64_t m = rows ? rows[r] : r;
+            int64_t a = 0;
+            double y = 0.0, b = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                int qx = Xq[m * K + k], qw = Wq[k * N + n];
+                a += (int64_t)qx * qw;
+                double xd = (double)qx * (double)t[m], wd = (double)qw * (double)sw[n];
+                y += xd * wd;
+                b += fabs(xd) * fabs(wd);
+            }
+            if (acc) acc[r * N + n] = (int32_t)a;
+            if (y_bf16) y_bf16[r * N + n] = qgo_f32_to_bf16_rn(((float)a * t[m]) * sw[n]);
+            yref[r * N + n] = y;
+            bound[r * N + n] = b;
+        }
+}
+
+/* ------------------------------------------------------------------------- */
+/* O8: W4A8 GEMM with per-group partial sums.                                  */
+/* P[m][g][n] = sum_{k in g} qx*qw4 (exact integer, qw4 in [-7,7] stored as    */
+/* two's-complement nibbles); Y = t_m * sum_g P * s_gn.  The reference is the  */
+/* fp64 dot of (qx*t_m)(qw4*s_gn) and its absolute-value bound.                */
+/* part is [nrows][K/group][N] or NULL.                                        */
+/* ------------------------------------------------------------------------- */
+void qgo_gemm_w4a8(const int8_t* Xq, const float* t, int64_t M, int64_t K, const uint32_t* packed,
+                   const float* sg, int64_t N, int group, const int64_t* rows, int64_t nrows,
+                   int32_t* part, double* yref, double* bound)
+{
+    if (!rows) nrows = M;
+    int64_t G = K / group;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t r = 0; r < nrows; ++r) {
+            int64_t m = rows ? rows[r] : r;
+            double y = 0.0, b = 0.0;
+            for (int64_t g = 0; g < G; ++g) {
+                int64_t p = 0;
+                for (int i = 0; i < group; ++i) {
+                    int64_t k = g * group + i;
+                    int v = nib(packed, N, k, n);
+                    int qw = v >= 8 ? v - 16 : v; /* two's-complement nibble */
+                    int qx = Xq[m * K + k];
+                    p += (int64_t)qx * qw;
+                    double xd = (double)qx * (double)t[m], wd = (double)qw * (double)sg[g * N + n];
+                    y += xd * wd;
+                    b += fabs(xd) * fabs(wd);
+                }
+                if (part) part[(r * G + g) * N + n] = (int32_t)p;
+            }
+            yref[r * N + n] = y;
+            bound[r * N + n] = b;
+        }
+}
+
+/* Plain fp64 product of unquantized operands (the "no quantization" sanity figure):
+ * y[r][n] = sum_k X[m_r][k] * W[k][n]. */
+void qgo_gemm_f64(const float* X, int64_t M, int64_t K, const float* W, int64_t N,
+                  const int64_t* rows, int64_t nrows, double* y)
+{
+    if (!rows) nrows = M;
+    memset(y, 0, sizeof(double) * nrows * N);
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            double w = (double)W[k * N + n];
+            for (int64_t r = 0; r < nrows; ++r)
+                y[r * N + n] += (double)X[(rows ? rows[r] : r) * K + k] * w;
+        }
+}

@@ -1,0 +1,41 @@
+"""Plant a plausible mistake in a copy of the oracle (on the CPU) and check that the pins
+catch it.  Each mutation edits one expression of qg_oracle.c; the pin named beside it must
+then fail.  This shows the pins constrain the oracle's arithmetic, not just its shape."""
+import pytest
+
+import oracle
+import test_oracle_pins as pins
+
+MUTATIONS = [
+    # (original text, mutated text, pins that must fail)
+    ("nearbyintf(v / s) + z, 0, 15)", "nearbyintf(v / s), 0, 15)",
+     [pins.test_w4_asym_round_trip_bound_and_ranges]),
+    ("float s32 = r / 15.0f;", "float s32 = r / 16.0f;",
+     [lambda: pins.test_w4_asym_hand_examples(0)]),
+    ("uint16_t s16 = qgo_f32_to_f16_ru(s32);", "uint16_t s16 = (uint16_t)(qgo_f32_to_f16_ru(s32) - (qgo_f32_to_f16_ru(s32) > 0 && qgo_f16_to_f32(qgo_f32_to_f16_ru(s32)) != s32));",
+     [lambda: pins.test_w4_asym_hand_examples(0)]),
+    ("<< (4 * i);", "<< (4 * (7 - i));", [lambda: pins.test_pack_hand_words(0)]),
+    ("return (double)(q - (int)zeros[g * N + n])", "return (double)((int)zeros[g * N + n] - q)",
+     [pins.test_w4a16_ref_reduces_to_integer_matmul]),
+    ("int64_t g = k / group;\n    int q = nib(packed, N, k, n);", "int64_t g = n % (K_UNUSED + 1);\n    int q = nib(packed, N, k, n);",
+     [pins.test_w4a16_ref_reduces_to_integer_matmul]),
+    ("sj = sqrtf(ax) / sqrtf(aw);", "sj = sqrtf(aw) / sqrtf(ax);", [pins.test_smooth_half_alpha_equalises_ranges]),
+    ("int qw = v >= 8 ? v - 16 : v;", "int qw = v;", [pins.test_w4a8_partials_and_reference]),
+    ("float tm = a / 127.0f;", "float tm = a / 128.0f;", [pins.test_act_i8_closed_form_and_brute_force]),
+    ("float s = amax / 7.0f;", "float s = amax / 8.0f;", [pins.test_w4_sym_absmax_bound_brute_force]),
+]
+
+
+@pytest.mark.parametrize("idx", range(len(MUTATIONS)))
+def test_planted_mistake_is_caught(idx, tmp_path):
+    orig, mutated, must_fail = MUTATIONS[idx]
+    src = oracle.source_text()
+    assert orig in src, f"mutation anchor not found: {orig!r}"
+    text = src.replace(orig, mutated)
+    if "K_UNUSED" in mutated:
+        text = "#define K_UNUSED 0\n" + text
+    L = oracle.build_variant(text, str(tmp_path / f"mut{idx}.so"))
+    with oracle.use_library(L):
+        for pin in must_fail:
+            with pytest.raises(AssertionError):
+                pin()
