@@ -1,0 +1,398 @@
+#!/usr/bin/env python
+"""Benchmark of the quantized linear layer hot path on B200.
+
+Default workload (the one the headline metric is quoted on): the W4A16 decode sweep,
+Llama-2-7B-shaped layers, M in {1,4,16,32} x (K,N) in {(4096,12288), (4096,4096),
+(4096,22016), (11008,4096)}, bf16 activations, group-128 asymmetric INT4 weights.
+One step = the 16 fused dequant-GEMM calls of the sweep on one batch of synthetic
+input (weights quantized once, resident in HBM).  The value is algorithmic HBM
+bytes per second over the timed steps: packed weights + fp16 scales + u8 zeros +
+bf16 X + bf16 Y per call.  Weight buffers rotate over enough copies that every
+call reads its weights from HBM, not L2.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--workload w4a16_decode|w8a8|w4a16_prefill|w4a8|w4a16_tiny]
+
+Under torchrun every rank runs the same workload on its own GPU (replicas, weak
+scaling); timing is the max over ranks of CUDA-event time; rank 0 prints one JSON line.
+`--impl reference` times the CPU oracle (the deliberately plain reference) on a
+bounded sample of the same workload instead.
+"""
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "quantized GEMM TFLOPS/TOPS and HBM GB/s (% of roofline) at M=1..8192"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        d["source"] = "measured"
+        return d
+    return dict(FALLBACK_PEAKS)
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        self.proc.wait()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 10:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[2]) for r in rows if num(r[2]) is not None]
+        mx = [num(r[3]) for r in rows if num(r[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[6 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------
+def dist_setup(n_gpus):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# W4A16 decode sweep on the GPU
+# ---------------------------------------------------------------------------
+def l2_bytes():
+    return torch.cuda.get_device_properties(torch.cuda.current_device()).L2_cache_size
+
+
+def w4_bytes(K, N):
+    return K * N // 2 + (K // 128) * N * 3
+
+
+class DecodeSweep:
+    """All (K, N) x M calls of the decode sweep with weights resident and rotating."""
+
+    def __init__(self, q, seed=0):
+        cfg = synth.CONFIGS["w4a16_decode"]
+        self.q = q
+        self.shapes = []
+        L2 = l2_bytes()
+        for (K, N) in cfg["KN"]:
+            W = torch.from_numpy(synth.workload_weights("w4a16_decode", K, N, seed)).cuda()
+            codes = torch.empty(K, N, dtype=torch.uint8, device="cuda")
+            scales = torch.empty(K // 128, N, dtype=torch.int16, device="cuda")
+            zeros = torch.empty(K // 128, N, dtype=torch.uint8, device="cuda")
+            packed = torch.empty(K // 8, N, dtype=torch.int32, device="cuda")
+            q.qg_quantize_w4_group(W, None, 128, False, codes, scales, zeros)
+            q.qg_pack_nibbles(codes, packed)
+            del W, codes
+            copies = max(2, min(48, math.ceil(2 * L2 / w4_bytes(K, N))))
+            ws = [(packed.clone(), scales.clone(), zeros.clone()) for _ in range(copies)]
+            calls = []
+            for M in cfg["M"]:
+                _, xb = synth.activations(M, K, "bf16", seed=M)
+                X = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+                Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+                calls.append(dict(M=M, X=X, Y=Y))
+            self.shapes.append(dict(K=K, N=N, copies=ws, calls=calls))
+        torch.cuda.synchronize()
+        assert q.qg_device_status() == q.QG_OK
+
+    def calls(self):
+        for sh in self.shapes:
+            for c in sh["calls"]:
+                yield sh, c
+
+    def bytes_per_step(self):
+        return sum(w4_bytes(sh["K"], sh["N"]) + 2 * c["M"] * sh["K"] + 2 * c["M"] * sh["N"] for sh, c in self.calls())
+
+    def flops_per_step(self):
+        return sum(2 * c["M"] * sh["K"] * sh["N"] for sh, c in self.calls())
+
+    def launches_per_step(self):
+        return sum(1 for _ in self.calls())
+
+    def step(self, s):
+        q = self.q
+        for sh in self.shapes:
+            p, sc, z = sh["copies"][s % len(sh["copies"])]
+            for c in sh["calls"]:
+                q.qg_gemm_w4a16(c["X"], p, sc, z, c["Y"])
+
+    def n_variants(self):
+        return max(len(sh["copies"]) for sh in self.shapes)
+
+
+def capture_graphs(fn, n):
+    """One CUDA graph per rotation index (each replays one step)."""
+    graphs = []
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for i in range(n):
+            fn(i)                      # warm (sets kernel attributes, caches)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    for i in range(n):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn(i)
+        graphs.append(g)
+    torch.cuda.synchronize()
+    return graphs
+
+
+def time_graphs(graphs, steps, warmup, world):
+    for i in range(warmup):
+        graphs[i % len(graphs)].replay()
+    barrier(world)
+    torch.cuda.synchronize()
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    start.record()
+    for i in range(steps):
+        graphs[(warmup + i) % len(graphs)].replay()
+    end.record()
+    torch.cuda.synchronize()
+    barrier(world)
+    return start.elapsed_time(end)
+
+
+def per_call_times(sweep, reps=64):
+    """Average device time per launch of each (K, N, M) call, rotating weights,
+    each call captured alone in a graph of `reps` launches."""
+    q = sweep.q
+    out = []
+    for sh in sweep.shapes:
+        for c in sh["calls"]:
+            def fn(i, sh=sh, c=c):
+                for r in range(reps):
+                    p, sc, z = sh["copies"][(i * reps + r) % len(sh["copies"])]
+                    q.qg_gemm_w4a16(c["X"], p, sc, z, c["Y"])
+            gs = capture_graphs(fn, 1)
+            ms = time_graphs(gs, 5, 2, 1) / 5 / reps
+            by = w4_bytes(sh["K"], sh["N"]) + 2 * c["M"] * (sh["K"] + sh["N"])
+            out.append(dict(K=sh["K"], N=sh["N"], M=c["M"], us=ms * 1e3, gbs=by / (ms * 1e-3) / 1e9,
+                            tflops=2 * c["M"] * sh["K"] * sh["N"] / (ms * 1e-3) / 1e12))
+    return out
+
+
+def e2e_decode(sweep, steps, warmup, world):
+    """Same sweep through the C ABI with host buffers: every call copies its X from
+    pinned host memory to the device and its Y back, inside the timed region."""
+    q = sweep.q
+    host = []
+    h2d = d2h = 0
+    for sh, c in sweep.calls():
+        xh = c["X"].cpu().pin_memory()
+        yh = torch.empty(c["Y"].shape, dtype=c["Y"].dtype).pin_memory()
+        host.append((sh, c, xh, yh))
+        h2d += xh.numel() * 2
+        d2h += yh.numel() * 2
+
+    def fn(i):
+        for sh, c, xh, yh in host:
+            p, sc, z = sh["copies"][i % len(sh["copies"])]
+            c["X"].copy_(xh, non_blocking=True)
+            q.qg_gemm_w4a16(c["X"], p, sc, z, c["Y"])
+            yh.copy_(c["Y"], non_blocking=True)
+    graphs = capture_graphs(fn, sweep.n_variants())
+    ms = max_over_ranks(time_graphs(graphs, steps, warmup, world), world)
+    return ms, h2d, d2h
+
+
+def cpu_baseline_decode(seconds_hint=15.0, col_frac=16):
+    """The oracle, as it stands, on a bounded sample of the sweep: every (K, N, M)
+    call restricted to the first N/col_frac output columns."""
+    import oracle
+    cfg = synth.CONFIGS["w4a16_decode"]
+    prepared = []
+    for (K, N) in cfg["KN"]:
+        Ns = max(8, N // col_frac)
+        W = synth.workload_weights("w4a16_decode", K, N)[:, :Ns].copy()
+        codes, scales, zeros, _ = oracle.quantize_w4_asym(W)
+        packed = oracle.pack_nibbles(codes)
+        for M in cfg["M"]:
+            X, _ = synth.activations(M, K, "bf16", seed=M)
+            prepared.append((K, Ns, M, X, packed, scales, zeros))
+    t0 = time.perf_counter()
+    by = 0
+    for K, Ns, M, X, packed, scales, zeros in prepared:
+        oracle.gemm_w4a16_ref(X, packed, scales, zeros)
+        by += w4_bytes(K, Ns) + 2 * M * (K + Ns)
+    dt = time.perf_counter() - t0
+    cores = len(os.sched_getaffinity(0))
+    return dict(value=by / dt / 1e9, unit="GB/s", cores=cores, kind="oracle",
+                sample=f"all 16 decode-sweep calls on the first 1/{col_frac} of the output columns "
+                       f"({by / 1e6:.1f} MB algorithmic), fp64 reference GEMM, {dt:.2f} s"), dt
+
+
+def run_reference(args, world, rank):
+    """--impl reference: the CPU oracle timed on a bounded sample of the workload."""
+    if rank != 0:
+        return
+    col_frac = 64
+    _, dt = cpu_baseline_decode(col_frac=col_frac)  # warm-up + size estimate
+    times = []
+    by = None
+    for i in range(args.warmup + args.steps):
+        cb, dt = cpu_baseline_decode(col_frac=col_frac)
+        if i >= args.warmup:
+            times.append(dt)
+            by = cb["value"] * dt * 1e9
+    total = sum(times)
+    value = by * len(times) / total / 1e9
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / len(times) * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "w4a16_decode sample: 16 calls on 1/64 of the columns"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "kind": "oracle", "cores": cb["cores"],
+                             "sample": cb["sample"]},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="w4a16_decode")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, int(os.environ.get("WORLD_SIZE", "1")), rank)
+        return
+
+    world, rank, local = dist_setup(args.gpus)
+    import bit_quantized_gemm_group_b200 as q
+    pk = peaks()
+    sweep = DecodeSweep(q)
+    graphs = capture_graphs(sweep.step, sweep.n_variants())
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    ms = time_graphs(graphs, args.steps, args.warmup, world)
+    ck = clocks.stop()
+    ms = max_over_ranks(ms, world)
+    ms_step = ms / args.steps
+    by = sweep.bytes_per_step()
+    value = by * world * args.steps / (ms * 1e-3) / 1e9
+    achieved = by / (ms_step * 1e-3) / 1e9
+
+    e2e_ms, h2d, d2h = e2e_decode(sweep, args.steps, args.warmup, world)
+    e2e_val = by * world * args.steps / (e2e_ms * 1e-3) / 1e9
+    calls = per_call_times(sweep) if rank == 0 else []
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu, _ = cpu_baseline_decode()
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "w4a16_decode: M in {1,4,16,32} x (K,N) in {(4096,12288),(4096,4096),"
+                                   "(4096,22016),(11008,4096)}, group-128 asym INT4, bf16 X/Y",
+                       "l2": "weights rotate over copies totalling >= 2x L2 per shape (no L2 reuse across calls)",
+                       "launch": "one CUDA graph per step (16 launches)"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm_gbs"], "traffic": None, "peak_source": pk["source"],
+                         "kernel": "w4a16_skinny_kernel (whole step)"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": sweep.launches_per_step() * args.steps,
+            "clocks": ck,
+            "tflops": sweep.flops_per_step() / (ms_step * 1e-3) / 1e12,
+            "per_call": [{k: (round(v, 3) if isinstance(v, float) else v) for k, v in c.items()} for c in calls],
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        del graphs
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,158 @@
+"""Python binding of libqgemm.so, the B200 (sm_100a) quantized linear layer.
+
+Argument marshalling only: every function here passes device pointers, sizes and
+the current CUDA stream of its tensors to the C function of the same name in
+include/qgemm.h and raises QgError on a non-OK status.  All compute runs in the
+library's CUDA kernels; there is no CPU path.  The library must have been built
+(``python -m bit_quantized_gemm_group_b200.build``); importing without it raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libqgemm.so")
+
+STATUS = {0: "QG_OK", 1: "QG_ERR_NULL", 2: "QG_ERR_SHAPE", 3: "QG_ERR_ALIGN", 4: "QG_ERR_DTYPE",
+          5: "QG_ERR_NONFINITE", 6: "QG_ERR_RANGE", 7: "QG_ERR_TIMEOUT", 8: "QG_ERR_CUDA", 9: "QG_ERR_UNSUPPORTED"}
+QG_OK, QG_ERR_NULL, QG_ERR_SHAPE, QG_ERR_ALIGN, QG_ERR_DTYPE = 0, 1, 2, 3, 4
+QG_ERR_NONFINITE, QG_ERR_RANGE, QG_ERR_TIMEOUT, QG_ERR_CUDA, QG_ERR_UNSUPPORTED = 5, 6, 7, 8, 9
+QG_F16, QG_BF16 = 0, 1
+
+EXPORTS = ["qg_quantize_w4_group", "qg_pack_nibbles", "qg_gemm_w4a16", "qg_smooth_quant_act_i8", "qg_gemm_w8a8",
+           "qg_gemm_w4a8", "qg_smooth_scales", "qg_quantize_w8_channel", "qg_device_status", "qg_status_string",
+           "qg_last_error", "qg_selftest_bounded_wait"]
+
+
+class QgError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        msg = f"{where}: {STATUS.get(status, status)}"
+        if status == QG_ERR_CUDA and _lib is not None:
+            msg += " (" + _lib.qg_last_error().decode() + ")"
+        super().__init__(msg)
+
+
+_P, _I, _SZ = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+_SIGS = {
+    "qg_quantize_w4_group": [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P],
+    "qg_pack_nibbles": [_P, _I, _I, _P, _P],
+    "qg_gemm_w4a16": [_P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _P, _SZ, _P],
+    "qg_smooth_quant_act_i8": [_P, _I, _I, _P, _P, _P, _P],
+    "qg_gemm_w8a8": [_P, _P, _I, _I, _P, _P, _I, _P, _P, _P, _SZ, _P],
+    "qg_gemm_w4a8": [_P, _P, _I, _I, _P, _P, _I, _I, _P, _P, _P, _SZ, _P],
+    "qg_smooth_scales": [_P, _I, _P, _I, _I, ctypes.c_float, _P, _P, _P],
+    "qg_quantize_w8_channel": [_P, _P, _I, _I, _P, _P, _P],
+    "qg_device_status": [_P],
+    "qg_selftest_bounded_wait": [ctypes.c_uint64, _P],
+}
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    if not os.path.exists(path):
+        raise ImportError(f"libqgemm.so not built at {path}; run python -m bit_quantized_gemm_group_b200.build")
+    L = ctypes.CDLL(path)
+    for name, argtypes in _SIGS.items():
+        f = getattr(L, name)
+        f.argtypes = argtypes
+        f.restype = ctypes.c_int
+    L.qg_status_string.argtypes = [ctypes.c_int]
+    L.qg_status_string.restype = ctypes.c_char_p
+    L.qg_last_error.argtypes = []
+    L.qg_last_error.restype = ctypes.c_char_p
+    return L
+
+
+_lib = load_library()
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libqgemm takes device tensors only")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous (row-major)")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(st: int, where: str):
+    if st != QG_OK:
+        raise QgError(st, where)
+
+
+def qg_quantize_w4_group(W, s_smooth, group, symmetric, codes, scales, zeros, stream=None):
+    K, N = W.shape
+    _check(_lib.qg_quantize_w4_group(_ptr(W), _ptr(s_smooth), K, N, group, int(bool(symmetric)), _ptr(codes),
+                                     _ptr(scales), _ptr(zeros), _stream(stream)), "qg_quantize_w4_group")
+
+
+def qg_pack_nibbles(codes, packed, stream=None):
+    K, N = codes.shape
+    _check(_lib.qg_pack_nibbles(_ptr(codes), K, N, _ptr(packed), _stream(stream)), "qg_pack_nibbles")
+
+
+def qg_gemm_w4a16(X, packed, scales, zeros, Y, group=128, stream=None):
+    M, K = X.shape
+    N = packed.shape[1]
+    xdt = QG_BF16 if X.dtype == torch.bfloat16 else QG_F16 if X.dtype == torch.float16 else -1
+    _check(_lib.qg_gemm_w4a16(_ptr(X), xdt, M, K, N, _ptr(packed), _ptr(scales), _ptr(zeros), group, _ptr(Y), None, 0,
+                              _stream(stream)), "qg_gemm_w4a16")
+
+
+def qg_smooth_quant_act_i8(X, inv_s, Xq, t, stream=None):
+    M, K = X.shape
+    _check(_lib.qg_smooth_quant_act_i8(_ptr(X), M, K, _ptr(inv_s), _ptr(Xq), _ptr(t), _stream(stream)),
+           "qg_smooth_quant_act_i8")
+
+
+def qg_gemm_w8a8(Xq, t, Wq, sw, Y, acc_dbg=None, stream=None):
+    M, K = Xq.shape
+    N = Wq.shape[1]
+    _check(_lib.qg_gemm_w8a8(_ptr(Xq), _ptr(t), M, K, _ptr(Wq), _ptr(sw), N, _ptr(Y), _ptr(acc_dbg), None, 0,
+                             _stream(stream)), "qg_gemm_w8a8")
+
+
+def qg_gemm_w4a8(Xq, t, packed, sg, Y, part_dbg=None, group=128, stream=None):
+    M, K = Xq.shape
+    N = packed.shape[1]
+    _check(_lib.qg_gemm_w4a8(_ptr(Xq), _ptr(t), M, K, _ptr(packed), _ptr(sg), N, group, _ptr(Y), _ptr(part_dbg), None,
+                             0, _stream(stream)), "qg_gemm_w4a8")
+
+
+def qg_smooth_scales(Xcal, W, alpha, s, inv_s, stream=None):
+    Mc, K = Xcal.shape
+    N = W.shape[1]
+    _check(_lib.qg_smooth_scales(_ptr(Xcal), Mc, _ptr(W), K, N, ctypes.c_float(alpha), _ptr(s), _ptr(inv_s),
+                                 _stream(stream)), "qg_smooth_scales")
+
+
+def qg_quantize_w8_channel(W, s, Wq, sw, stream=None):
+    K, N = W.shape
+    _check(_lib.qg_quantize_w8_channel(_ptr(W), _ptr(s), K, N, _ptr(Wq), _ptr(sw), _stream(stream)),
+           "qg_quantize_w8_channel")
+
+
+def qg_device_status(stream=None) -> int:
+    return _lib.qg_device_status(_stream(stream))
+
+
+def qg_selftest_bounded_wait(limit_ns: int = 0, stream=None):
+    _check(_lib.qg_selftest_bounded_wait(limit_ns, _stream(stream)), "qg_selftest_bounded_wait")
+
+
+def qg_status_string(status: int) -> str:
+    return _lib.qg_status_string(status).decode()

@@ -1,0 +1,382 @@
+// qgemm.cu -- C ABI of libqgemm.so: argument validation, launch configuration and
+// dispatch to the sm_100a kernels.  Declarations and full contracts: include/qgemm.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "../../include/qgemm.h"
+#include "act_quant.cuh"
+#include "common.cuh"
+#include "int8_skinny.cuh"
+#include "quantize.cuh"
+#include "tc_gemm.cuh"
+#include "w4a16_skinny.cuh"
+
+namespace {
+
+thread_local char g_last_error[256] = "";
+
+qg_status cuda_fail(cudaError_t e, const char* where)
+{
+    snprintf(g_last_error, sizeof(g_last_error), "%s: %s", where, cudaGetErrorString(e));
+    return QG_ERR_CUDA;
+}
+
+#define QG_CUDA(call)                                      \
+    do {                                                   \
+        cudaError_t e_ = (call);                           \
+        if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
+    } while (0)
+
+bool misaligned(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u); }
+
+constexpr int kMaxDevices = 64;
+
+int current_device()
+{
+    int dev = 0;
+    cudaGetDevice(&dev);
+    return dev >= 0 && dev < kMaxDevices ? dev : 0;
+}
+
+int num_sms()
+{
+    static int cache[kMaxDevices] = {0};
+    const int dev = current_device();
+    if (cache[dev] == 0) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cache[dev] = n > 0 ? n : 148;
+    }
+    return cache[dev];
+}
+
+// Launch `kern` with a thread-block cluster of (1, cy, 1).
+template <typename Kern, typename Arg>
+qg_status launch_cluster(Kern kern, dim3 grid, dim3 block, size_t smem, int cy, qg_stream_t stream, const Arg& arg)
+{
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = cy;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    QG_CUDA(cudaLaunchKernelEx(&cfg, kern, arg));
+    return QG_OK;
+}
+
+// Choose the split-K cluster size S in {1,2,4,8} (S <= groups) that best fills the
+// GPU: the fraction of CTA slots used over all waves, ties going to more CTAs.
+int choose_split(int nslabs, int groups, int ctas_per_sm)
+{
+    const int slots = num_sms() * std::max(ctas_per_sm, 1);
+    int best = 1;
+    double best_eff = -1.0;
+    for (int S = 1; S <= 8; S *= 2) {
+        if (S > groups) break;
+        const long total = (long)nslabs * S;
+        const long waves = (total + slots - 1) / slots;
+        const double eff = (double)total / (double)(waves * slots);
+        if (eff > best_eff + 1e-9) {
+            best_eff = eff;
+            best = S;
+        }
+    }
+    return best;
+}
+
+// Per kernel instance and device: raise the dynamic shared memory limit once and
+// remember the occupancy, so that a launch makes no query calls after the first.
+struct KernelInfo {
+    int occ[kMaxDevices] = {0};
+};
+
+template <typename Kern>
+qg_status prepare_kernel(KernelInfo& info, Kern k, int threads, size_t smem, int* occ)
+{
+    const int dev = current_device();
+    if (info.occ[dev] == 0) {
+        if (smem > 48 * 1024)
+            QG_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+        int n = 0;
+        QG_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, smem));
+        info.occ[dev] = n > 0 ? n : 1;
+    }
+    *occ = info.occ[dev];
+    return QG_OK;
+}
+
+// ---------------------------------------------------------------------------
+// W4A16 skinny path (M <= 32 per launch)
+// ---------------------------------------------------------------------------
+template <int MT, bool BF16>
+qg_status launch_w4a16_skinny(const qg::SkinnyParams& p, qg_stream_t stream)
+{
+    constexpr int WN = 2, WK = 4, DEPTH = 4;
+    constexpr int BN = 64 * WN, MP = 8 * MT;
+    auto kern = qg::w4a16_skinny_kernel<MT, BF16, WN, WK, DEPTH>;
+    const size_t smem = (size_t)WK * BN * MP * 4;
+    static KernelInfo info;
+    int occ = 1;
+    qg_status st = prepare_kernel(info, kern, WN * WK * 32, smem, &occ);
+    if (st != QG_OK) return st;
+    const int nslabs = (p.N + BN - 1) / BN;
+    const int S = choose_split(nslabs, p.K / 128, occ);
+    return launch_cluster(kern, dim3(nslabs, S, 1), dim3(WN * WK * 32), smem, S, stream, p);
+}
+
+template <bool BF16>
+qg_status w4a16_skinny_dispatch(qg::SkinnyParams p, qg_stream_t stream)
+{
+    for (int m0 = 0; m0 < p.M; m0 += 32) {
+        qg::SkinnyParams q = p;
+        q.M = std::min(32, p.M - m0);
+        q.X = p.X + (int64_t)m0 * p.K;
+        q.Y = p.Y + (int64_t)m0 * p.N;
+        qg_status st;
+        if (q.M <= 8) st = launch_w4a16_skinny<1, BF16>(q, stream);
+        else if (q.M <= 16) st = launch_w4a16_skinny<2, BF16>(q, stream);
+        else st = launch_w4a16_skinny<4, BF16>(q, stream);
+        if (st != QG_OK) return st;
+    }
+    return QG_OK;
+}
+
+// ---------------------------------------------------------------------------
+// int8 skinny paths
+// ---------------------------------------------------------------------------
+template <int MT>
+qg_status launch_w8a8_skinny(const qg::Int8SkinnyParams& p, qg_stream_t stream)
+{
+    constexpr int WN = 1, WK = 8;
+    constexpr int BN = 128 * WN, MP = 8 * MT;
+    auto kern = qg::w8a8_skinny_kernel<MT, WN, WK>;
+    const size_t smem = (size_t)WK * BN * MP * 4;
+    static KernelInfo info;
+    int occ = 1;
+    qg_status st = prepare_kernel(info, kern, WN * WK * 32, smem, &occ);
+    if (st != QG_OK) return st;
+    const int nslabs = (p.N + BN - 1) / BN;
+    const int S = choose_split(nslabs, p.K / 128, occ);
+    return launch_cluster(kern, dim3(nslabs, S, 1), dim3(WN * WK * 32), smem, S, stream, p);
+}
+
+template <int MT>
+qg_status launch_w4a8_skinny(const qg::Int8SkinnyParams& p, qg_stream_t stream)
+{
+    constexpr int WN = 2, WK = 4;
+    constexpr int BN = 64 * WN, MP = 8 * MT;
+    auto kern = qg::w4a8_skinny_kernel<MT, WN, WK>;
+    const size_t smem = (size_t)WK * BN * MP * 4;
+    static KernelInfo info;
+    int occ = 1;
+    qg_status st = prepare_kernel(info, kern, WN * WK * 32, smem, &occ);
+    if (st != QG_OK) return st;
+    const int nslabs = (p.N + BN - 1) / BN;
+    const int S = choose_split(nslabs, p.K / 128, occ);
+    return launch_cluster(kern, dim3(nslabs, S, 1), dim3(WN * WK * 32), smem, S, stream, p);
+}
+
+}  // namespace
+
+// ===========================================================================
+// C ABI
+// ===========================================================================
+extern "C" {
+
+const char* qg_status_string(qg_status s)
+{
+    switch (s) {
+        case QG_OK: return "QG_OK";
+        case QG_ERR_NULL: return "QG_ERR_NULL";
+        case QG_ERR_SHAPE: return "QG_ERR_SHAPE";
+        case QG_ERR_ALIGN: return "QG_ERR_ALIGN";
+        case QG_ERR_DTYPE: return "QG_ERR_DTYPE";
+        case QG_ERR_NONFINITE: return "QG_ERR_NONFINITE";
+        case QG_ERR_RANGE: return "QG_ERR_RANGE";
+        case QG_ERR_TIMEOUT: return "QG_ERR_TIMEOUT";
+        case QG_ERR_CUDA: return "QG_ERR_CUDA";
+        case QG_ERR_UNSUPPORTED: return "QG_ERR_UNSUPPORTED";
+    }
+    return "QG_ERR_UNKNOWN";
+}
+
+const char* qg_last_error(void) { return g_last_error; }
+
+qg_status qg_device_status(qg_stream_t stream)
+{
+    QG_CUDA(cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)));
+    unsigned int v = 0, zero = 0;
+    QG_CUDA(cudaMemcpyFromSymbol(&v, qg::g_status, sizeof(v)));
+    QG_CUDA(cudaMemcpyToSymbol(qg::g_status, &zero, sizeof(zero)));
+    return (qg_status)v;
+}
+
+qg_status qg_quantize_w4_group(const float* W, const float* s_smooth, int K, int N, int group, int symmetric,
+                               uint8_t* codes, void* scales, uint8_t* zeros, qg_stream_t stream)
+{
+    if (!W || !codes || !scales || (!symmetric && !zeros)) return QG_ERR_NULL;
+    if (symmetric && zeros) return QG_ERR_NULL;
+    if (K < 1 || N < 1 || group < 8 || group > 1024 || group % 8 || K % group) return QG_ERR_SHAPE;
+    if (misaligned(W) || misaligned(s_smooth) || misaligned(codes) || misaligned(scales) || misaligned(zeros))
+        return QG_ERR_ALIGN;
+    const dim3 grid((N + 255) / 256, K / group), block(256);
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (symmetric)
+        qg::quantize_w4_sym_kernel<<<grid, block, 0, s>>>(W, s_smooth, K, N, group, reinterpret_cast<int8_t*>(codes),
+                                                           static_cast<float*>(scales));
+    else
+        qg::quantize_w4_asym_kernel<<<grid, block, 0, s>>>(W, s_smooth, K, N, group, codes,
+                                                            static_cast<uint16_t*>(scales), zeros);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+
+qg_status qg_pack_nibbles(const uint8_t* codes, int K, int N, uint32_t* packed, qg_stream_t stream)
+{
+    if (!codes || !packed) return QG_ERR_NULL;
+    if (K < 8 || N < 1 || K % 8) return QG_ERR_SHAPE;
+    if (misaligned(codes) || misaligned(packed)) return QG_ERR_ALIGN;
+    const dim3 grid(((N + 3) / 4 + 255) / 256, K / 8), block(256);
+    qg::pack_nibbles_kernel<<<grid, block, 0, reinterpret_cast<cudaStream_t>(stream)>>>(codes, K, N, packed);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+
+qg_status qg_gemm_w4a16(const void* X, qg_dtype xdt, int M, int K, int N, const uint32_t* packed,
+                        const uint16_t* scales, const uint8_t* zeros, int group, void* Y, void* workspace,
+                        size_t ws_bytes, qg_stream_t stream)
+{
+    (void)workspace;
+    (void)ws_bytes;
+    if (xdt != QG_F16 && xdt != QG_BF16) return QG_ERR_DTYPE;
+    if (M < 0 || K < 128 || N < 8 || K % 128 || N % 8 || group != 128) return QG_ERR_SHAPE;
+    if (M == 0) return QG_OK;
+    if (!X || !packed || !scales || !zeros || !Y) return QG_ERR_NULL;
+    if (misaligned(X) || misaligned(packed) || misaligned(scales) || misaligned(zeros) || misaligned(Y))
+        return QG_ERR_ALIGN;
+    if (xdt == QG_BF16 && M >= qg::kTcMinM) {
+        qg::TcW4A16Args a{static_cast<const uint16_t*>(X), packed, scales, zeros, static_cast<uint16_t*>(Y), M, K, N};
+        return qg::tc_w4a16_launch(a, stream);
+    }
+    qg::SkinnyParams p{static_cast<const uint16_t*>(X), packed, scales, zeros, static_cast<uint16_t*>(Y), M, K, N};
+    return xdt == QG_BF16 ? w4a16_skinny_dispatch<true>(p, stream) : w4a16_skinny_dispatch<false>(p, stream);
+}
+
+qg_status qg_smooth_quant_act_i8(const uint16_t* X, int M, int K, const float* inv_s, int8_t* Xq, float* t,
+                                 qg_stream_t stream)
+{
+    if (M < 0 || K < 8 || K % 8) return QG_ERR_SHAPE;
+    if (M == 0) return QG_OK;
+    if (!X || !Xq || !t) return QG_ERR_NULL;
+    if (misaligned(X) || misaligned(inv_s) || misaligned(Xq) || misaligned(t)) return QG_ERR_ALIGN;
+    qg::smooth_quant_act_i8_kernel<<<M, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(X, K, inv_s, Xq, t);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+
+qg_status qg_gemm_w8a8(const int8_t* Xq, const float* t, int M, int K, const int8_t* Wq, const float* sw, int N,
+                       uint16_t* Y, int32_t* acc_dbg, void* workspace, size_t ws_bytes, qg_stream_t stream)
+{
+    (void)workspace;
+    (void)ws_bytes;
+    if (M < 0 || K < 128 || N < 16 || K % 128 || N % 16) return QG_ERR_SHAPE;
+    if (M == 0) return QG_OK;
+    if (!Xq || !t || !Wq || !sw || !Y) return QG_ERR_NULL;
+    if (misaligned(Xq) || misaligned(t) || misaligned(Wq) || misaligned(sw) || misaligned(Y) || misaligned(acc_dbg))
+        return QG_ERR_ALIGN;
+    if (M >= qg::kTcMinM) {
+        qg::TcInt8Args a{Xq, t, Wq, sw, nullptr, nullptr, Y, acc_dbg, M, K, N};
+        return qg::tc_w8a8_launch(a, stream);
+    }
+    for (int m0 = 0; m0 < M; m0 += 16) {
+        qg::Int8SkinnyParams p{Xq + (int64_t)m0 * K, t + m0, Wq, sw, nullptr, nullptr, Y + (int64_t)m0 * N,
+                               acc_dbg ? acc_dbg + (int64_t)m0 * N : nullptr, std::min(16, M - m0), K, N};
+        qg_status st = p.M <= 8 ? launch_w8a8_skinny<1>(p, stream) : launch_w8a8_skinny<2>(p, stream);
+        if (st != QG_OK) return st;
+    }
+    return QG_OK;
+}
+
+qg_status qg_gemm_w4a8(const int8_t* Xq, const float* t, int M, int K, const uint32_t* packed, const float* sg,
+                       int N, int group, uint16_t* Y, int32_t* part_dbg, void* workspace, size_t ws_bytes,
+                       qg_stream_t stream)
+{
+    (void)workspace;
+    (void)ws_bytes;
+    if (M < 0 || K < 128 || N < 16 || K % 128 || N % 16 || group != 128) return QG_ERR_SHAPE;
+    if (M == 0) return QG_OK;
+    if (!Xq || !t || !packed || !sg || !Y) return QG_ERR_NULL;
+    if (misaligned(Xq) || misaligned(t) || misaligned(packed) || misaligned(sg) || misaligned(Y) ||
+        misaligned(part_dbg))
+        return QG_ERR_ALIGN;
+    if (M >= qg::kTcMinM) {
+        qg::TcInt8Args a{Xq, t, nullptr, nullptr, packed, sg, Y, part_dbg, M, K, N};
+        return qg::tc_w4a8_launch(a, stream);
+    }
+    const int G = K / 128;
+    for (int m0 = 0; m0 < M; m0 += 32) {
+        qg::Int8SkinnyParams p{Xq + (int64_t)m0 * K, t + m0, nullptr, nullptr, packed, sg, Y + (int64_t)m0 * N,
+                               part_dbg ? part_dbg + (int64_t)m0 * G * N : nullptr, std::min(32, M - m0), K, N};
+        qg_status st = p.M <= 8 ? launch_w4a8_skinny<1>(p, stream)
+                       : p.M <= 16 ? launch_w4a8_skinny<2>(p, stream)
+                                   : launch_w4a8_skinny<4>(p, stream);
+        if (st != QG_OK) return st;
+    }
+    return QG_OK;
+}
+
+qg_status qg_smooth_scales(const uint16_t* Xcal, int Mc, const float* W, int K, int N, float alpha, float* s,
+                           float* inv_s, qg_stream_t stream)
+{
+    if (!Xcal || !W || !s || !inv_s) return QG_ERR_NULL;
+    if (Mc < 1 || K < 1 || N < 1) return QG_ERR_SHAPE;
+    if (!(alpha >= 0.0f && alpha <= 1.0f)) return QG_ERR_SHAPE;
+    if (misaligned(Xcal) || misaligned(W) || misaligned(s) || misaligned(inv_s)) return QG_ERR_ALIGN;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    qg::col_absmax_bf16_kernel<<<(K + 255) / 256, 256, 0, st>>>(Xcal, Mc, K, s);
+    QG_CUDA(cudaGetLastError());
+    qg::row_absmax_f32_kernel<<<K, 256, 0, st>>>(W, K, N, inv_s);
+    QG_CUDA(cudaGetLastError());
+    qg::smooth_finalize_kernel<<<(K + 255) / 256, 256, 0, st>>>(s, inv_s, K, alpha);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+
+qg_status qg_quantize_w8_channel(const float* W, const float* s, int K, int N, int8_t* Wq, float* sw,
+                                 qg_stream_t stream)
+{
+    if (!W || !Wq || !sw) return QG_ERR_NULL;
+    if (K < 1 || N < 1) return QG_ERR_SHAPE;
+    if (misaligned(W) || misaligned(s) || misaligned(Wq) || misaligned(sw)) return QG_ERR_ALIGN;
+    qg::quantize_w8_channel_kernel<<<(N + 127) / 128, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(W, s, K, N,
+                                                                                                          Wq, sw);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+
+qg_status qg_selftest_bounded_wait(uint64_t limit_ns, qg_stream_t stream)
+{
+    unsigned long long lim = limit_ns ? (unsigned long long)limit_ns : 2000000000ull;
+    unsigned long long saved = 0;
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    QG_CUDA(cudaMemcpyFromSymbol(&saved, qg::g_wait_limit_ns, sizeof(saved)));
+    QG_CUDA(cudaMemcpyToSymbolAsync(qg::g_wait_limit_ns, &lim, sizeof(lim), 0, cudaMemcpyHostToDevice, st));
+    qg::selftest_wait_kernel<<<1, 32, 0, st>>>();
+    QG_CUDA(cudaGetLastError());
+    QG_CUDA(cudaMemcpyToSymbolAsync(qg::g_wait_limit_ns, &saved, sizeof(saved), 0, cudaMemcpyHostToDevice, st));
+    QG_CUDA(cudaStreamSynchronize(st));
+    return QG_OK;
+}
+
+}  // extern "C"

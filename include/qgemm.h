@@ -1,0 +1,210 @@
+/*
+ * qgemm.h -- C ABI of libqgemm.so, the B200 (sm_100a) quantized linear layer.
+ *
+ * What the library computes (the pages' definitions; page titles abbreviated):
+ *   [Q]  "AI Infra guide, ch.4 Quantization" (aiinfra.vidrealm.tech), sec. 1.1-1.3:
+ *        affine quantization x_int = round(x/s) + z, x_hat = (x_int - z) s;
+ *        symmetric s = max|x|/127; asymmetric s = (max-min)/255 with z adjusted;
+ *        per-channel / per-group / per-token granularity.
+ *   [S]  same page, sec. 2.2 (SmoothQuant): Y = (X diag(s)^-1)(diag(s) W),
+ *        s_j = max|X_j|^alpha / max|W_j|^(1-alpha), alpha = 0.5 typical.
+ *   [W4] same page, sec. 3.1 and 3.5: weight-only INT4, dequantize and multiply,
+ *        fused (Marlin-style) so that no dequantized copy of W is written.
+ *   [G]  "LLM inference cost: W8A8/W4A8 ..." (0539edu.com), sec. 2.2: group-wise
+ *        quantization with an independent scale and zero per group of 128; W4A8.
+ *
+ * Readings taken where the pages are silent (the same ones the test oracle takes):
+ *   asymmetric INT4 uses s = (max' - min')/15 over a range widened to contain 0,
+ *   stored as fp16 rounded toward +infinity; z = clamp(round(-min'/s), 0, 15);
+ *   code = clamp(round(x/s) + z, 0, 15) in that order; round = half to even in
+ *   binary32; symmetric INT4 uses s = max|x|/7 (fp32) and codes in [-7, 7];
+ *   INT8 codes lie in [-127, 127]; a zero range gives scale 0 and codes 0.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     keeps none of them after the call returns and allocates no device memory.
+ *   - Tensors are dense and row-major: X[M][K] activations, W[K][N] weights,
+ *     Y[M][N] = X W.  Groups run along K.
+ *   - fp16 / bf16 tensors are passed as uint16_t bit patterns.
+ *   - Every call is asynchronous on `stream` (NULL = the legacy default stream).
+ *     The return value reports argument validation and launch errors only; a
+ *     call that returns anything but QG_OK launched nothing.
+ *   - Conditions found on the device (a non-finite input, a scale that does not
+ *     fit fp16, a bounded wait that ran out) set a sticky per-device status word
+ *     instead; qg_device_status() synchronizes the stream, returns that word and
+ *     clears it.
+ *   - Shape rules common to all calls: M >= 0, K >= 1, N >= 1; M == 0 returns
+ *     QG_OK and launches nothing.  Each call lists its own extra rules.
+ *   - Base pointers must be 16-byte aligned (QG_ERR_ALIGN otherwise).
+ */
+#ifndef QGEMM_H
+#define QGEMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st* qg_stream_t;
+
+typedef enum {
+    QG_OK = 0,
+    QG_ERR_NULL = 1,        /* a required pointer is NULL */
+    QG_ERR_SHAPE = 2,       /* a size breaks the call's shape rules */
+    QG_ERR_ALIGN = 3,       /* a base pointer is not 16-byte aligned */
+    QG_ERR_DTYPE = 4,       /* unknown dtype enumerator */
+    QG_ERR_NONFINITE = 5,   /* (device) an input that must be finite was NaN or Inf */
+    QG_ERR_RANGE = 6,       /* (device) an fp16 scale would overflow */
+    QG_ERR_TIMEOUT = 7,     /* (device) a bounded wait inside a kernel gave up */
+    QG_ERR_CUDA = 8,        /* the CUDA runtime reported an error; see qg_last_error() */
+    QG_ERR_UNSUPPORTED = 9  /* the device is not sm_100 or a feature is missing */
+} qg_status;
+
+typedef enum { QG_F16 = 0, QG_BF16 = 1 } qg_dtype;
+
+/* --------------------------------------------------------------------------
+ * Group-wise INT4 weight quantization.   [Q] sec. 1.1-1.3, [G] sec. 2.2
+ *
+ * W        fp32 [K][N].
+ * s_smooth fp32 [K] or NULL.  When given, the quantized matrix is diag(s) W,
+ *          i.e. W[k][n] * s_smooth[k] rounded once to fp32 ([S] sec. 2.2).
+ * group    group size along K; K % group == 0, group % 8 == 0, 8 <= group <= 1024
+ *          (128 everywhere in the workloads).
+ * symmetric
+ *   0: asymmetric.  codes u8 [K][N] in [0,15]; scales = fp16 bits [K/group][N]
+ *      (uint16_t*), rounded toward +infinity; zeros u8 [K/group][N] in [0,15].
+ *   1: symmetric.   codes = int8 [K][N] in [-7,7] (stored through the uint8_t*
+ *      pointer as two's complement bytes); scales = fp32 [K/group][N]
+ *      (float*); zeros must be NULL.
+ * Device errors: QG_ERR_NONFINITE (a non-finite element; that group's outputs
+ * are left unspecified), QG_ERR_RANGE (asymmetric scale above 65504).
+ * ------------------------------------------------------------------------ */
+qg_status qg_quantize_w4_group(const float* W, const float* s_smooth, int K, int N, int group,
+                               int symmetric, uint8_t* codes, void* scales, uint8_t* zeros,
+                               qg_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * Pack 4-bit codes 8 per uint32 along K, low nibble first:
+ *   packed[kb][n] = sum_{i<8} (codes[8kb+i][n] & 0xF) << 4i
+ * codes u8 [K][N] (symmetric codes as two's complement bytes), packed u32 [K/8][N].
+ * K % 8 == 0.   (Storage of 8 nibbles per uint32, low first: [G] workload definition.)
+ * ------------------------------------------------------------------------ */
+qg_status qg_pack_nibbles(const uint8_t* codes, int K, int N, uint32_t* packed, qg_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * W4A16 fused dequant-GEMM.   [W4] sec. 3.1, 3.5; [G] sec. 2.2 (pseudo-code of
+ * the quantized matmul with per-group scale and zero)
+ *
+ *   Y[m][n] = sum_k X[m][k] * (q[k][n] - z[k/g][n]) * s[k/g][n]
+ *
+ * X        fp16 or bf16 [M][K] (xdt); Y has the same dtype, [M][N].
+ * packed   u32 [K/8][N] from qg_pack_nibbles of asymmetric codes.
+ * scales   fp16 bits [K/group][N]; zeros u8 [K/group][N].
+ * group    128 (the only group size the GEMM kernels take).
+ * Rules: K % 128 == 0, N % 8 == 0.  Accumulation is fp32; the dequantized weight
+ * is rounded once to the activation dtype before the tensor-core product.
+ * workspace / ws_bytes are unused (pass NULL, 0); the split-K reduction runs in
+ * on-chip distributed shared memory.
+ * ------------------------------------------------------------------------ */
+qg_status qg_gemm_w4a16(const void* X, qg_dtype xdt, int M, int K, int N, const uint32_t* packed,
+                        const uint16_t* scales, const uint8_t* zeros, int group, void* Y,
+                        void* workspace, size_t ws_bytes, qg_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * Fused smoothing + per-token dynamic symmetric INT8 quantization of
+ * activations.   [S] sec. 2.2; [Q] sec. 1.2 (s = max|x|/127), sec. 1.3 (per token)
+ *
+ *   X~[m][j] = X[m][j] * inv_s[j]           (one fp32 rounding; inv_s NULL -> X~ = X)
+ *   t[m]     = max_j |X~[m][j]| / 127        (fp32)
+ *   Xq[m][j] = clamp(round(X~[m][j] / t[m]), -127, 127);  t[m] == 0 -> all zero
+ *
+ * X bf16 [M][K]; inv_s fp32 [K] or NULL; Xq int8 [M][K]; t fp32 [M].
+ * Rules: K % 8 == 0.   Device error: QG_ERR_NONFINITE.
+ * ------------------------------------------------------------------------ */
+qg_status qg_smooth_quant_act_i8(const uint16_t* X, int M, int K, const float* inv_s, int8_t* Xq,
+                                 float* t, qg_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * W8A8 GEMM (SmoothQuant).   [S] sec. 2.2-2.3; [Q] sec. 1.3
+ *
+ *   acc[m][n] = sum_k Xq[m][k] * Wq[k][n]          (int32, exact)
+ *   Y[m][n]   = bf16_rn( ((float)acc * t[m]) * sw[n] )
+ *
+ * Xq int8 [M][K], t fp32 [M] (from qg_smooth_quant_act_i8); Wq int8 [K][N],
+ * sw fp32 [N] (from qg_quantize_w8_channel); Y bf16 [M][N].
+ * acc_dbg: NULL, or int32 [M][N] that also receives the exact accumulators.
+ * Rules: K % 128 == 0, N % 16 == 0.  workspace / ws_bytes unused (NULL, 0).
+ * ------------------------------------------------------------------------ */
+qg_status qg_gemm_w8a8(const int8_t* Xq, const float* t, int M, int K, const int8_t* Wq,
+                       const float* sw, int N, uint16_t* Y, int32_t* acc_dbg, void* workspace,
+                       size_t ws_bytes, qg_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * W4A8 GEMM with per-group fp32 rescaling.   [G] sec. 2.2 (W4A8, group-wise)
+ *
+ *   P[m][g][n] = sum_{k in group g} Xq[m][k] * q[k][n]     (int32, exact)
+ *   Y[m][n]    = bf16_rn( t[m] * sum_g P[m][g][n] * sg[g][n] )   (fp32)
+ *
+ * Xq int8 [M][K], t fp32 [M]; packed u32 [K/8][N] of symmetric codes (two's
+ * complement nibbles in [-7,7]); sg fp32 [K/group][N]; Y bf16 [M][N].
+ * part_dbg: NULL, or int32 [M][K/group][N] that also receives every P.
+ * Rules: group == 128, K % 128 == 0, N % 16 == 0.  workspace unused (NULL, 0).
+ * ------------------------------------------------------------------------ */
+qg_status qg_gemm_w4a8(const int8_t* Xq, const float* t, int M, int K, const uint32_t* packed,
+                       const float* sg, int N, int group, uint16_t* Y, int32_t* part_dbg,
+                       void* workspace, size_t ws_bytes, qg_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * SmoothQuant factors from a calibration batch.   [S] sec. 2.2
+ *
+ *   ax[j] = max_m |Xcal[m][j]|,  aw[j] = max_n |W[j][n]|
+ *   s[j]  = ax^alpha / aw^(1-alpha)  (alpha == 0.5: sqrt(ax)/sqrt(aw) in fp32,
+ *           correctly rounded; otherwise fp64 pow, rounded to fp32)
+ *   s[j]  = 1 when ax or aw is 0;   inv_s[j] = 1 / s[j] (fp32)
+ *
+ * Xcal bf16 [Mc][K]; W fp32 [K][N]; s, inv_s fp32 [K].  0 <= alpha <= 1.
+ * Device error: QG_ERR_NONFINITE.
+ * ------------------------------------------------------------------------ */
+qg_status qg_smooth_scales(const uint16_t* Xcal, int Mc, const float* W, int K, int N, float alpha,
+                           float* s, float* inv_s, qg_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * Per-output-channel symmetric INT8 weights.   [Q] sec. 1.2-1.3; [S] sec. 2.2
+ *
+ *   W~ = diag(s) W (s NULL -> W~ = W);  sw[n] = max_k |W~[k][n]| / 127
+ *   Wq[k][n] = clamp(round(W~[k][n] / sw[n]), -127, 127);  sw[n] == 0 -> zeros
+ *
+ * W fp32 [K][N]; s fp32 [K] or NULL; Wq int8 [K][N]; sw fp32 [N].
+ * Device error: QG_ERR_NONFINITE.
+ * ------------------------------------------------------------------------ */
+qg_status qg_quantize_w8_channel(const float* W, const float* s, int K, int N, int8_t* Wq, float* sw,
+                                 qg_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * Status and diagnostics
+ * ------------------------------------------------------------------------ */
+
+/* Synchronizes `stream`, returns the current device's sticky status word
+ * (QG_OK if nothing was recorded) and clears it. */
+qg_status qg_device_status(qg_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char* qg_status_string(qg_status s);
+
+/* Text of the last CUDA error seen by this thread inside the library ("" if none). */
+const char* qg_last_error(void);
+
+/* Test hook for the bounded-wait machinery: launches one block that waits on a
+ * shared-memory barrier nothing will ever complete, giving up after `limit_ns`
+ * nanoseconds (0 = the library default of 2 s).  The wait ends by itself; the
+ * device status then reads QG_ERR_TIMEOUT.  No fault, trap or hang is involved. */
+qg_status qg_selftest_bounded_wait(uint64_t limit_ns, qg_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QGEMM_H */

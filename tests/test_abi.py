@@ -1,0 +1,102 @@
+"""The C-ABI library loads, exports every entry point include/qgemm.h declares, and
+rejects bad arguments before launching anything.  CPU only: every call here fails
+validation, so no CUDA call is reached."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qgemm.h")
+
+
+def declared_symbols():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qg_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    syms = declared_symbols()
+    for name in ["qg_quantize_w4_group", "qg_pack_nibbles", "qg_gemm_w4a16", "qg_smooth_quant_act_i8",
+                 "qg_gemm_w8a8", "qg_gemm_w4a8", "qg_smooth_scales", "qg_quantize_w8_channel", "qg_device_status",
+                 "qg_status_string"]:
+        assert name in syms
+
+
+def test_library_exports_every_declared_symbol():
+    import bit_quantized_gemm_group_b200 as q
+    L = q.lib()
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+    assert set(q.EXPORTS) >= set(declared_symbols())
+
+
+def test_status_strings():
+    import bit_quantized_gemm_group_b200 as q
+    for code, name in q.STATUS.items():
+        assert q.qg_status_string(code) == name
+
+
+P = ctypes.c_void_p
+A = P(0x10000)        # aligned fake device address (never dereferenced: validation fails first)
+B = P(0x10008)        # 8-byte but not 16-byte aligned
+
+
+@pytest.mark.parametrize("args,want", [
+    # quantize_w4_group(W, s, K, N, group, sym, codes, scales, zeros, stream)
+    ((None, None, 256, 64, 128, 0, A, A, A, None), 1),
+    ((A, None, 256, 64, 128, 0, A, A, None, None), 1),       # asym needs zeros
+    ((A, None, 256, 64, 128, 1, A, A, A, None), 1),          # sym takes no zeros
+    ((A, None, 200, 64, 128, 0, A, A, A, None), 2),          # K % group
+    ((A, None, 256, 64, 12, 0, A, A, A, None), 2),           # group % 8
+    ((A, None, 256, 0, 128, 0, A, A, A, None), 2),
+    ((B, None, 256, 64, 128, 0, A, A, A, None), 3),
+])
+def test_quantize_rejects(args, want):
+    import bit_quantized_gemm_group_b200 as q
+    assert q.lib().qg_quantize_w4_group(*args) == want
+
+
+@pytest.mark.parametrize("args,want", [
+    # gemm_w4a16(X, xdt, M, K, N, packed, scales, zeros, group, Y, ws, ws_bytes, stream)
+    ((A, 7, 1, 256, 64, A, A, A, 128, A, None, 0, None), 4),
+    ((A, 1, 1, 200, 64, A, A, A, 128, A, None, 0, None), 2),
+    ((A, 1, 1, 256, 60, A, A, A, 128, A, None, 0, None), 2),
+    ((A, 1, 1, 256, 64, A, A, A, 64, A, None, 0, None), 2),
+    ((A, 1, -1, 256, 64, A, A, A, 128, A, None, 0, None), 2),
+    ((A, 1, 0, 256, 64, A, A, A, 128, A, None, 0, None), 0),     # M == 0: OK, nothing launched
+    ((None, 1, 0, 256, 64, None, None, None, 128, None, None, 0, None), 0),
+    ((None, 1, 1, 256, 64, A, A, A, 128, A, None, 0, None), 1),
+    ((A, 1, 1, 256, 64, A, A, A, 128, B, None, 0, None), 3),
+])
+def test_gemm_w4a16_rejects(args, want):
+    import bit_quantized_gemm_group_b200 as q
+    assert q.lib().qg_gemm_w4a16(*args) == want
+
+
+@pytest.mark.parametrize("fn,args,want", [
+    ("qg_gemm_w8a8", (A, A, 4, 256, A, A, 72, A, None, None, 0, None), 2),     # N % 16
+    ("qg_gemm_w8a8", (A, A, 4, 256, A, A, 64, A, B, None, 0, None), 3),        # misaligned debug output
+    ("qg_gemm_w8a8", (A, None, 4, 256, A, A, 64, A, None, None, 0, None), 1),
+    ("qg_gemm_w8a8", (None, None, 0, 256, None, None, 64, None, None, None, 0, None), 0),
+    ("qg_gemm_w4a8", (A, A, 4, 256, A, A, 64, 64, A, None, None, 0, None), 2),  # group != 128
+    ("qg_gemm_w4a8", (A, A, 4, 256, A, None, 64, 128, A, None, None, 0, None), 1),
+    ("qg_smooth_quant_act_i8", (A, 4, 12, None, A, A, None), 2),                # K % 8
+    ("qg_smooth_quant_act_i8", (A, 4, 16, B, A, A, None), 3),
+    ("qg_smooth_quant_act_i8", (None, 0, 16, None, None, None, None), 0),
+    ("qg_pack_nibbles", (A, 12, 16, A, None), 2),
+    ("qg_pack_nibbles", (None, 16, 16, A, None), 1),
+    ("qg_quantize_w8_channel", (A, None, 0, 16, A, A, None), 2),
+])
+def test_other_calls_reject(fn, args, want):
+    import bit_quantized_gemm_group_b200 as q
+    assert getattr(q.lib(), fn)(*args) == want
+
+
+def test_smooth_scales_rejects_alpha():
+    import bit_quantized_gemm_group_b200 as q
+    f = q.lib().qg_smooth_scales
+    assert f(A, 4, A, 16, 16, ctypes.c_float(1.5), A, A, None) == 2
+    assert f(A, 4, A, 16, 16, ctypes.c_float(float("nan")), A, A, None) == 2
