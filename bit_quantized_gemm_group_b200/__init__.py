@@ -17,14 +17,17 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libqgemm.so")
 
 STATUS = {0: "QG_OK", 1: "QG_ERR_NULL", 2: "QG_ERR_SHAPE", 3: "QG_ERR_ALIGN", 4: "QG_ERR_DTYPE",
-          5: "QG_ERR_NONFINITE", 6: "QG_ERR_RANGE", 7: "QG_ERR_TIMEOUT", 8: "QG_ERR_CUDA", 9: "QG_ERR_UNSUPPORTED"}
+          5: "QG_ERR_NONFINITE", 6: "QG_ERR_RANGE", 7: "QG_ERR_TIMEOUT", 8: "QG_ERR_CUDA", 9: "QG_ERR_UNSUPPORTED",
+          10: "QG_ERR_WORKSPACE"}
 QG_OK, QG_ERR_NULL, QG_ERR_SHAPE, QG_ERR_ALIGN, QG_ERR_DTYPE = 0, 1, 2, 3, 4
 QG_ERR_NONFINITE, QG_ERR_RANGE, QG_ERR_TIMEOUT, QG_ERR_CUDA, QG_ERR_UNSUPPORTED = 5, 6, 7, 8, 9
+QG_ERR_WORKSPACE = 10
 QG_F16, QG_BF16 = 0, 1
+QG_OP_GEMM_W4A16, QG_OP_GEMM_W8A8, QG_OP_GEMM_W4A8 = 0, 1, 2
 
 EXPORTS = ["qg_quantize_w4_group", "qg_pack_nibbles", "qg_gemm_w4a16", "qg_smooth_quant_act_i8", "qg_gemm_w8a8",
            "qg_gemm_w4a8", "qg_smooth_scales", "qg_quantize_w8_channel", "qg_device_status", "qg_status_string",
-           "qg_last_error", "qg_selftest_bounded_wait"]
+           "qg_last_error", "qg_selftest_bounded_wait", "qg_workspace_size"]
 
 
 class QgError(RuntimeError):
@@ -63,6 +66,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     L.qg_status_string.restype = ctypes.c_char_p
     L.qg_last_error.argtypes = []
     L.qg_last_error.restype = ctypes.c_char_p
+    L.qg_workspace_size.argtypes = [_I, _I, _I, _I]
+    L.qg_workspace_size.restype = ctypes.c_size_t
     return L
 
 
@@ -105,11 +110,42 @@ def qg_pack_nibbles(codes, packed, stream=None):
     _check(_lib.qg_pack_nibbles(_ptr(codes), K, N, _ptr(packed), _stream(stream)), "qg_pack_nibbles")
 
 
-def qg_gemm_w4a16(X, packed, scales, zeros, Y, group=128, stream=None):
+_WS = {}
+
+
+def qg_workspace_size(op: int, M: int, K: int, N: int) -> int:
+    return _lib.qg_workspace_size(op, M, K, N)
+
+
+def default_workspace(op, M, K, N, device):
+    """A zero-filled workspace for (op, M, K, N), cached per device and grown on demand.
+    Calls that may run concurrently (different streams) need workspaces of their own."""
+    need = _lib.qg_workspace_size(op, M, K, N)
+    if need == 0:
+        return None
+    key = torch.device(device).index if torch.device(device).index is not None else torch.cuda.current_device()
+    buf = _WS.get(key)
+    if buf is None or buf.numel() < need:
+        buf = torch.zeros(max(need, 1 << 20), dtype=torch.uint8, device=device)
+        _WS[key] = buf
+    return buf
+
+
+def _ws(workspace, op, M, K, N, device):
+    """workspace='auto' -> cached zero-filled buffer; None / False -> no workspace."""
+    if isinstance(workspace, str) and workspace == "auto":
+        workspace = default_workspace(op, M, K, N, device)
+    if workspace is None or workspace is False:
+        return None, 0
+    return _ptr(workspace), workspace.numel() * workspace.element_size()
+
+
+def qg_gemm_w4a16(X, packed, scales, zeros, Y, group=128, workspace="auto", stream=None):
     M, K = X.shape
     N = packed.shape[1]
     xdt = QG_BF16 if X.dtype == torch.bfloat16 else QG_F16 if X.dtype == torch.float16 else -1
-    _check(_lib.qg_gemm_w4a16(_ptr(X), xdt, M, K, N, _ptr(packed), _ptr(scales), _ptr(zeros), group, _ptr(Y), None, 0,
+    wp, wb = _ws(workspace, QG_OP_GEMM_W4A16, M, K, N, X.device)
+    _check(_lib.qg_gemm_w4a16(_ptr(X), xdt, M, K, N, _ptr(packed), _ptr(scales), _ptr(zeros), group, _ptr(Y), wp, wb,
                               _stream(stream)), "qg_gemm_w4a16")
 
 

@@ -83,7 +83,7 @@ QG_DEV_INLINE uint4 ldg_stream_v4(const void* p)
 {
     // read-once data: do not keep it in L1
     uint4 v;
-    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+    asm("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p));
     return v;
@@ -92,7 +92,7 @@ QG_DEV_INLINE uint4 ldg_stream_v4(const void* p)
 QG_DEV_INLINE uint4 ldg_v4(const void* p)
 {
     uint4 v;
-    asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+    asm("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                  : "l"(p));
     return v;
@@ -149,6 +149,26 @@ QG_DEV_INLINE bool mbar_wait(uint64_t* bar, uint32_t parity)
             return false;
         }
     }
+}
+
+// Named barrier `id` over `count` threads that also ANDs a predicate across them.
+QG_DEV_INLINE int named_bar_and(uint32_t id, uint32_t count, bool v)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 q, %1, 0;\n\t"
+        "bar.red.and.pred p, %2, %3, q;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(r)
+        : "r"((uint32_t)v), "r"(id), "r"(count)
+        : "memory");
+    return (int)r;
+}
+
+QG_DEV_INLINE void named_bar_sync(uint32_t id, uint32_t count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
 QG_DEV_INLINE void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }

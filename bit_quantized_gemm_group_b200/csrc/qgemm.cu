@@ -1,6 +1,7 @@
 // qgemm.cu -- C ABI of libqgemm.so: argument validation, launch configuration and
 // dispatch to the sm_100a kernels.  Declarations and full contracts: include/qgemm.h.
 #include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stdio.h>
@@ -14,6 +15,7 @@
 #include "int8_skinny.cuh"
 #include "quantize.cuh"
 #include "tc_gemm.cuh"
+#include "w4a16_decode.cuh"
 #include "w4a16_skinny.cuh"
 
 namespace {
@@ -153,6 +155,125 @@ qg_status w4a16_skinny_dispatch(qg::SkinnyParams p, qg_stream_t stream)
 }
 
 // ---------------------------------------------------------------------------
+// TMA descriptors (driver entry point fetched through the runtime; no libcuda link)
+// ---------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (!fn) {
+        void* ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+// 2-D tiled map over a row-major [outer][inner] array.
+qg_status make_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, size_t elem_bytes, const void* base, uint64_t inner,
+                       uint64_t outer, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle sw)
+{
+    auto enc = tmap_encoder();
+    if (!enc) {
+        snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled unavailable");
+        return QG_ERR_UNSUPPORTED;
+    }
+    cuuint64_t dims[2] = {inner, outer};
+    cuuint64_t strides[1] = {inner * elem_bytes};
+    cuuint32_t box[2] = {box_inner, box_outer};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled failed (%d)", (int)r);
+        return QG_ERR_CUDA;
+    }
+    return QG_OK;
+}
+
+// ---------------------------------------------------------------------------
+// W4A16 decode (stream-K, TMA-fed, workspace)
+// ---------------------------------------------------------------------------
+struct DecodePlan {
+    int MP, G, nslabs, units, grid;
+    size_t partial_bytes, counter_bytes;
+};
+
+DecodePlan decode_plan(int M, int K, int N)
+{
+    DecodePlan d;
+    const int mc = std::min(M, 32);
+    d.MP = mc <= 8 ? 8 : mc <= 16 ? 16 : 32;
+    d.G = K / 128;
+    d.nslabs = (N + qg::kDecBN - 1) / qg::kDecBN;
+    d.units = d.G * d.nslabs;
+    d.grid = std::min(num_sms(), d.units);
+    d.partial_bytes = (size_t)d.grid * 2 * qg::kDecBN * d.MP * sizeof(float);
+    d.counter_bytes = ((size_t)d.nslabs * sizeof(int) + 255) & ~size_t(255);
+    return d;
+}
+
+bool decode_eligible(int M, int N) { return M >= 1 && N % 16 == 0; }
+
+template <int MT, bool BF16>
+qg_status launch_w4a16_decode(const qg::SkinnyParams& sp, const uint32_t* packed, const uint16_t* scales,
+                              const uint8_t* zeros, void* ws, qg_stream_t stream)
+{
+    constexpr int ST = MT <= 2 ? 4 : 3;
+    auto kern = qg::w4a16_decode_kernel<MT, BF16, ST>;
+    const size_t smem = qg::DecodeSmem<MT, ST>::TOTAL;
+    static KernelInfo info;
+    int occ = 1;
+    qg_status st = prepare_kernel(info, kern, 384, smem, &occ);
+    if (st != QG_OK) return st;
+    const DecodePlan d = decode_plan(sp.M, sp.K, sp.N);
+    CUtensorMap tw, ts, tz;
+    if ((st = make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, sp.N, sp.K / 8, 32, 16,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
+        return st;
+    if ((st = make_tmap_2d(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, scales, sp.N, d.G, 128, 1,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK)
+        return st;
+    if ((st = make_tmap_2d(&tz, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, zeros, sp.N, d.G, 128, 1,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK)
+        return st;
+    qg::DecodeParams p;
+    p.X = sp.X;
+    p.Y = sp.Y;
+    p.counters = static_cast<int*>(ws);
+    p.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + d.counter_bytes);
+    p.M = sp.M;
+    p.K = sp.K;
+    p.N = sp.N;
+    p.G = d.G;
+    p.nslabs = d.nslabs;
+    p.units = d.units;
+    p.grid = d.grid;
+    kern<<<d.grid, 384, smem, reinterpret_cast<cudaStream_t>(stream)>>>(p, tw, ts, tz);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+
+template <bool BF16>
+qg_status w4a16_decode_dispatch(qg::SkinnyParams p, const uint32_t* packed, const uint16_t* scales,
+                                const uint8_t* zeros, void* ws, qg_stream_t stream)
+{
+    for (int m0 = 0; m0 < p.M; m0 += 32) {
+        qg::SkinnyParams q = p;
+        q.M = std::min(32, p.M - m0);
+        q.X = p.X + (int64_t)m0 * p.K;
+        q.Y = p.Y + (int64_t)m0 * p.N;
+        qg_status st;
+        if (q.M <= 8) st = launch_w4a16_decode<1, BF16>(q, packed, scales, zeros, ws, stream);
+        else if (q.M <= 16) st = launch_w4a16_decode<2, BF16>(q, packed, scales, zeros, ws, stream);
+        else st = launch_w4a16_decode<4, BF16>(q, packed, scales, zeros, ws, stream);
+        if (st != QG_OK) return st;
+    }
+    return QG_OK;
+}
+
+// ---------------------------------------------------------------------------
 // int8 skinny paths
 // ---------------------------------------------------------------------------
 template <int MT>
@@ -207,11 +328,25 @@ const char* qg_status_string(qg_status s)
         case QG_ERR_TIMEOUT: return "QG_ERR_TIMEOUT";
         case QG_ERR_CUDA: return "QG_ERR_CUDA";
         case QG_ERR_UNSUPPORTED: return "QG_ERR_UNSUPPORTED";
+        case QG_ERR_WORKSPACE: return "QG_ERR_WORKSPACE";
     }
     return "QG_ERR_UNKNOWN";
 }
 
 const char* qg_last_error(void) { return g_last_error; }
+
+size_t qg_workspace_size(qg_op op, int M, int K, int N)
+{
+    if (M < 1 || K < 128 || N < 8 || K % 128) return 0;
+    switch (op) {
+        case QG_OP_GEMM_W4A16: {
+            if (!decode_eligible(M, N)) return 0;
+            const DecodePlan d = decode_plan(M, K, N);
+            return d.counter_bytes + d.partial_bytes;
+        }
+        default: return 0;
+    }
+}
 
 qg_status qg_device_status(qg_stream_t stream)
 {
@@ -257,8 +392,6 @@ qg_status qg_gemm_w4a16(const void* X, qg_dtype xdt, int M, int K, int N, const 
                         const uint16_t* scales, const uint8_t* zeros, int group, void* Y, void* workspace,
                         size_t ws_bytes, qg_stream_t stream)
 {
-    (void)workspace;
-    (void)ws_bytes;
     if (xdt != QG_F16 && xdt != QG_BF16) return QG_ERR_DTYPE;
     if (M < 0 || K < 128 || N < 8 || K % 128 || N % 8 || group != 128) return QG_ERR_SHAPE;
     if (M == 0) return QG_OK;
@@ -270,6 +403,12 @@ qg_status qg_gemm_w4a16(const void* X, qg_dtype xdt, int M, int K, int N, const 
         return qg::tc_w4a16_launch(a, stream);
     }
     qg::SkinnyParams p{static_cast<const uint16_t*>(X), packed, scales, zeros, static_cast<uint16_t*>(Y), M, K, N};
+    if (workspace && decode_eligible(M, N)) {
+        if (ws_bytes < qg_workspace_size(QG_OP_GEMM_W4A16, M, K, N)) return QG_ERR_WORKSPACE;
+        if (misaligned(workspace)) return QG_ERR_ALIGN;
+        return xdt == QG_BF16 ? w4a16_decode_dispatch<true>(p, packed, scales, zeros, workspace, stream)
+                              : w4a16_decode_dispatch<false>(p, packed, scales, zeros, workspace, stream);
+    }
     return xdt == QG_BF16 ? w4a16_skinny_dispatch<true>(p, stream) : w4a16_skinny_dispatch<false>(p, stream);
 }
 

@@ -1,0 +1,330 @@
+// w4a16_decode.cuh -- decode-shape W4A16 fused dequant-GEMM (M <= 32 per launch).
+//
+//   Y[m][n] = sum_k X[m][k] (q[k][n] - z[g][n]) s[g][n],   g = k / 128
+// ("AI Infra guide, ch.4 Quantization" sec. 3.1 weight-only INT4, sec. 3.5 fused
+// INT4 x FP16 kernel; group-wise scale and zero: "LLM inference cost: W8A8/W4A8 ..."
+// sec. 2.2).  Decode is a weight stream: the design keeps HBM busy and the ALU cost
+// per weight small.
+//
+// Work split (stream-K).  The N columns form slabs of 128; one unit is one group
+// (128 k) of one slab.  The persistent grid (one CTA per SM) divides the
+// nslabs x G units into equal contiguous ranges, so every SM streams the same
+// number of bytes.  A CTA's range is a list of slab pieces; a piece that covers a
+// whole slab writes Y directly, a partial piece writes its fp32 tile to the
+// workspace and bumps the slab's counter; the CTA that brings the counter to the
+// number of pieces sums all pieces in CTA order (deterministic) and writes Y, then
+// resets the counter to zero.
+//
+// Data movement.  One producer warp streams each group's packed words (16 rows of
+// the [K/8][N] matrix x 128 columns, as four 128-byte-wide boxes with 128-byte
+// swizzle), fp16 scales and u8 zeros into a ring of shared-memory stages with TMA;
+// a stage holds up to four groups of one slab.  Eight consumer warps: warp (wn, wg)
+// takes columns 64wn..64wn+63 of group wg of each stage.
+//
+// Math.  Swap-AB mma.sync (weights are the m16 operand, up to 32 tokens are n8
+// tiles).  A lane's 128-bit read gives 4 columns x 8 k; OR-ing a nibble pair into
+// the exponent field of a bf16 (fp16) pair yields exactly 128 + q (1024 + q) with
+// one LOP3, so the MMA accumulates D = sum (128 + q) x per group.  The zero point and
+// scale are applied once per group and output element:
+//     acc += s * (D - (128 + z) * sum_{k in g} x)
+// where sum x comes from one extra MMA tile whose A operand is all ones, already in
+// the accumulator layout.  Inside a 32-k step the k order is permuted so that a
+// lane's own word feeds its fragment slots; the activation pairs get the same
+// permutation with two byte permutes per register.  Shared-memory rows are visited
+// in the order 0,2,4,6 | 1,3,5,7 | 8,... so the eight lanes of each 128-bit access
+// phase hit eight different 16-byte bank groups under the 128-byte swizzle.
+#pragma once
+#include "common.cuh"
+#include "w4a16_skinny.cuh"
+
+namespace qg {
+
+struct DecodeParams {
+    const uint16_t* X;
+    uint16_t* Y;
+    float* partials;  // [grid][2][128][MP]
+    int* counters;    // [nslabs], zero between calls
+    int M, K, N;
+    int G, nslabs, units, grid;
+};
+
+constexpr int kDecBN = 128;             // columns per slab
+constexpr int kDecGroupsPerStage = 4;
+constexpr int kDecGroupW = 16 * 128 * 4;  // packed words of one group: 16 rows x 128 columns x 4 B
+constexpr int kDecStageBytes = 35840;   // 4 x 8 KB words + 4 x 256 B scales + 4 x 128 B zeros, 1 KB aligned
+constexpr int kDecScaleOff = 4 * kDecGroupW;
+constexpr int kDecZeroOff = kDecScaleOff + 4 * 256;
+
+QG_DEV_INLINE int dec_first_unit(int c, int units, int grid) { return (int)((int64_t)c * units / grid); }
+
+template <int MT, int ST>
+struct DecodeSmem {
+    static constexpr int MP = 8 * MT;
+    static constexpr int RED = 4 * kDecBN * MP * 4;
+    static constexpr int TOTAL = ST * kDecStageBytes + RED + 2 * ST * 8 + 64 + 1024;
+};
+
+template <int MT, bool BF16, int ST>
+__global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams p,
+                                                               const __grid_constant__ CUtensorMap tm_w,
+                                                               const __grid_constant__ CUtensorMap tm_s,
+                                                               const __grid_constant__ CUtensorMap tm_z)
+{
+    using H = HalfOps<BF16>;
+    constexpr int MP = 8 * MT;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* ring = smem;
+    float* red = reinterpret_cast<float*>(smem + ST * kDecStageBytes);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * kDecStageBytes + DecodeSmem<MT, ST>::RED);
+    uint64_t* empty = full + ST;
+    int* flag = reinterpret_cast<int*>(empty + ST);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = p.G;
+    const int u0 = dec_first_unit(blockIdx.x, p.units, p.grid), u1 = dec_first_unit(blockIdx.x + 1, p.units, p.grid);
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < ST; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 8);
+        }
+        fence_mbar_init();
+    }
+    __syncthreads();
+
+    if (warp >= 8) {
+        // ---------------- producer warpgroup (one thread issues TMA) ----------------
+        // Registers: launched with 384 x 168; this warpgroup gives up 128 x 128 and the
+        // two consumer warpgroups take 256 x 64 (168 -> 232).
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
+        if (warp == 8 && lane == 0) {
+            tma_prefetch_desc(&tm_w);
+            tma_prefetch_desc(&tm_s);
+            tma_prefetch_desc(&tm_z);
+            int stage = 0;
+            uint32_t phase = 0;
+            for (int u = u0; u < u1;) {
+                const int slab = u / G, ga = u % G;
+                const int gb = min(G, ga + (u1 - u));
+                for (int g0 = ga; g0 < gb; g0 += kDecGroupsPerStage) {
+                    const int ng = min(kDecGroupsPerStage, gb - g0);
+                    if (!mbar_wait(&empty[stage], phase ^ 1)) return;
+                    mbar_arrive_expect_tx(&full[stage], (uint32_t)ng * (kDecGroupW + 256 + 128));
+                    uint8_t* st = ring + stage * kDecStageBytes;
+                    for (int i = 0; i < ng; ++i) {
+                        const int g = g0 + i;
+#pragma unroll
+                        for (int b = 0; b < 4; ++b)
+                            tma_load_2d(&tm_w, &full[stage], st + i * kDecGroupW + b * 2048, slab * kDecBN + 32 * b,
+                                        16 * g);
+                        tma_load_2d(&tm_s, &full[stage], st + kDecScaleOff + i * 256, slab * kDecBN, g);
+                        tma_load_2d(&tm_z, &full[stage], st + kDecZeroOff + i * 128, slab * kDecBN, g);
+                    }
+                    if (++stage == ST) { stage = 0; phase ^= 1; }
+                }
+                u += gb - ga;
+            }
+        }
+        return;
+    }
+
+    // ---------------- consumers ----------------
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 232;");
+    const int wn = warp & 1, wg = warp >> 1;
+    const int g8 = lane >> 2, t4 = lane & 3;
+    const uint32_t ONE = BF16 ? 0x3F803F80u : 0x3C003C00u;
+    float acc[2][2][MT][4];
+#pragma unroll
+    for (int h = 0; h < 2; ++h)
+#pragma unroll
+        for (int c = 0; c < 2; ++c)
+#pragma unroll
+            for (int j = 0; j < MT; ++j)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) acc[h][c][j][e] = 0.0f;
+
+    int stage = 0;
+    uint32_t phase = 0;
+    bool ok = true;
+    bool first_piece = true;
+    // After a wait gives up (status already recorded) the warp keeps walking the same
+    // schedule without waiting or computing, so that every named barrier still sees
+    // all 256 consumer threads; nothing is written to global memory after that.
+    for (int u = u0; u < u1;) {
+        const int slab = u / G, ga = u % G;
+        const int gb = min(G, ga + (u1 - u));
+        const int n0 = slab * kDecBN;
+        for (int g0 = ga; g0 < gb; g0 += kDecGroupsPerStage) {
+            const int ng = min(kDecGroupsPerStage, gb - g0);
+            if (ok && !mbar_wait(&full[stage], phase)) ok = false;
+            const uint8_t* st = ring + stage * kDecStageBytes;
+            if (ok && wg < ng) {
+                const int g = g0 + wg;
+                // per-column scale and (128 + z) of the lane's 8 columns
+                float sc[2][4], zc[2][4];
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                    const int col = 64 * wn + 32 * h + 4 * g8;
+                    const uint2 s4 = *reinterpret_cast<const uint2*>(st + kDecScaleOff + wg * 256 + col * 2);
+                    const uint32_t z4 = *reinterpret_cast<const uint32_t*>(st + kDecZeroOff + wg * 128 + col);
+                    const uint32_t sw[2] = {s4.x, s4.y};
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        sc[h][c] = __half2float(__ushort_as_half((unsigned short)(sw[c >> 1] >> (16 * (c & 1)))));
+                        zc[h][c] = H::BIAS + (float)((z4 >> (8 * c)) & 0xFFu);
+                    }
+                }
+                float D[2][2][MT][4], Dx[MT][4];
+#pragma unroll
+                for (int j = 0; j < MT; ++j) {
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) Dx[j][e] = 0.0f;
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+#pragma unroll
+                        for (int c = 0; c < 2; ++c)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) D[h][c][j][e] = 0.0f;
+                }
+                const uint8_t* wbase = st + wg * kDecGroupW;
+#pragma unroll
+                for (int s = 0; s < 4; ++s) {
+                    const int row = 8 * (s >> 1) + 2 * t4 + (s & 1);  // kb row within the group
+                    uint4 wv[2];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h)
+                        wv[h] = *reinterpret_cast<const uint4*>(wbase + (2 * wn + h) * 2048 + row * 128 +
+                                                                ((g8 ^ (row & 7)) << 4));
+                    uint32_t xb[MT][4];
+#pragma unroll
+                    for (int j = 0; j < MT; ++j) {
+                        const int tok = 8 * j + g8;
+                        uint4 xv = make_uint4(0u, 0u, 0u, 0u);
+                        if (tok < p.M) xv = ldg_v4(p.X + (int64_t)tok * p.K + 128 * g + 8 * row);
+                        xb[j][0] = prmt(xv.x, xv.z, 0x5410);
+                        xb[j][1] = prmt(xv.x, xv.z, 0x7632);
+                        xb[j][2] = prmt(xv.y, xv.w, 0x5410);
+                        xb[j][3] = prmt(xv.y, xv.w, 0x7632);
+                    }
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint32_t w[4] = {wv[h].x, wv[h].y, wv[h].z, wv[h].w};
+                        uint32_t R[4][4];
+#pragma unroll
+                        for (int c = 0; c < 4; ++c)
+#pragma unroll
+                            for (int r = 0; r < 4; ++r) R[c][r] = lop3_and_or(w[c] >> (4 * r), 0x000F000Fu, H::MAGIC);
+#pragma unroll
+                        for (int cp = 0; cp < 2; ++cp)
+#pragma unroll
+                            for (int j = 0; j < MT; ++j) {
+                                mma_16816<BF16>(D[h][cp][j], R[2 * cp][0], R[2 * cp + 1][0], R[2 * cp][1],
+                                                R[2 * cp + 1][1], xb[j][0], xb[j][1]);
+                                mma_16816<BF16>(D[h][cp][j], R[2 * cp][2], R[2 * cp + 1][2], R[2 * cp][3],
+                                                R[2 * cp + 1][3], xb[j][2], xb[j][3]);
+                            }
+                    }
+#pragma unroll
+                    for (int j = 0; j < MT; ++j) {
+                        mma_16816<BF16>(Dx[j], ONE, ONE, ONE, ONE, xb[j][0], xb[j][1]);
+                        mma_16816<BF16>(Dx[j], ONE, ONE, ONE, ONE, xb[j][2], xb[j][3]);
+                    }
+                }
+                // group epilogue: acc += s * (D - (128 + z) * sum x)
+#pragma unroll
+                for (int h = 0; h < 2; ++h)
+#pragma unroll
+                    for (int cp = 0; cp < 2; ++cp)
+#pragma unroll
+                        for (int j = 0; j < MT; ++j)
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const int c = 2 * cp + (e >> 1);
+                                const float xs = Dx[j][e & 1];
+                                acc[h][cp][j][e] = fmaf(sc[h][c], fmaf(-zc[h][c], xs, D[h][cp][j][e]), acc[h][cp][j][e]);
+                            }
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[stage]);
+            if (++stage == ST) { stage = 0; phase ^= 1; }
+        }
+        // ---------------- piece end: reduce the four group-warps, then write ----------------
+        float* myred = red + (size_t)wg * kDecBN * MP;
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+#pragma unroll
+            for (int cp = 0; cp < 2; ++cp)
+#pragma unroll
+                for (int j = 0; j < MT; ++j) {
+                    const int nl = 64 * wn + 32 * h + 4 * g8 + 2 * cp;
+                    const int tk = 8 * j + 2 * t4;
+                    *reinterpret_cast<float2*>(myred + (size_t)nl * MP + tk) = make_float2(acc[h][cp][j][0], acc[h][cp][j][1]);
+                    *reinterpret_cast<float2*>(myred + (size_t)(nl + 1) * MP + tk) =
+                        make_float2(acc[h][cp][j][2], acc[h][cp][j][3]);
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) acc[h][cp][j][e] = 0.0f;
+                }
+        named_bar_sync(1, 256);
+        for (int e = threadIdx.x; e < kDecBN * MP; e += 256) {
+            float v = red[e];
+#pragma unroll
+            for (int q = 1; q < 4; ++q) v += red[(size_t)q * kDecBN * MP + e];
+            red[e] = v;
+        }
+        named_bar_sync(1, 256);
+        const int nvalid = min(kDecBN, p.N - n0);
+        // any warp that gave up makes the whole CTA skip its global writes
+        const int all_ok = named_bar_and(1, 256, ok);
+        if (!all_ok) {
+            ok = false;
+        } else if (ga == 0 && gb == G) {
+            for (int e = threadIdx.x; e < p.M * kDecBN; e += 256) {
+                const int tok = e / kDecBN, nn = e % kDecBN;
+                if (nn < nvalid) p.Y[(int64_t)tok * p.N + n0 + nn] = H::to_bits(red[nn * MP + tok]);
+            }
+        } else {
+            const int slot = first_piece ? 0 : 1;
+            float* mine = p.partials + ((size_t)blockIdx.x * 2 + slot) * kDecBN * MP;
+            for (int e = threadIdx.x; e < kDecBN * MP; e += 256) mine[e] = red[e];
+            __threadfence();
+            named_bar_sync(1, 256);
+            if (threadIdx.x == 0) {
+                // CTAs that hold a piece of this slab: the ones containing its first and last unit
+                const int ufirst = slab * G, ulast = slab * G + G - 1;
+                int cf = (int)((int64_t)ufirst * p.grid / p.units);
+                while (cf > 0 && dec_first_unit(cf, p.units, p.grid) > ufirst) --cf;
+                while (dec_first_unit(cf + 1, p.units, p.grid) <= ufirst) ++cf;
+                int cl = (int)((int64_t)ulast * p.grid / p.units);
+                while (cl > 0 && dec_first_unit(cl, p.units, p.grid) > ulast) --cl;
+                while (dec_first_unit(cl + 1, p.units, p.grid) <= ulast) ++cl;
+                const int old = atomicAdd(&p.counters[slab], 1);
+                const bool last = old == cl - cf;
+                flag[0] = last ? 1 : 0;
+                flag[1] = cf;
+                flag[2] = cl;
+                if (last) p.counters[slab] = 0;
+            }
+            named_bar_sync(1, 256);
+            if (flag[0]) {
+                __threadfence();
+                const int cf = flag[1], cl = flag[2];
+                for (int e = threadIdx.x; e < p.M * kDecBN; e += 256) {
+                    const int tok = e / kDecBN, nn = e % kDecBN;
+                    if (nn >= nvalid) continue;
+                    float v = 0.0f;
+                    for (int c = cf; c <= cl; ++c) {
+                        const int sl = dec_first_unit(c, p.units, p.grid) >= slab * G ? 0 : 1;
+                        v += __ldcg(p.partials + ((size_t)c * 2 + sl) * kDecBN * MP + nn * MP + tok);
+                    }
+                    p.Y[(int64_t)tok * p.N + n0 + nn] = H::to_bits(v);
+                }
+            }
+        }
+        named_bar_sync(1, 256);
+        first_piece = false;
+        u += gb - ga;
+    }
+}
+
+}  // namespace qg

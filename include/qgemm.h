@@ -60,8 +60,12 @@ typedef enum {
     QG_ERR_RANGE = 6,       /* (device) an fp16 scale would overflow */
     QG_ERR_TIMEOUT = 7,     /* (device) a bounded wait inside a kernel gave up */
     QG_ERR_CUDA = 8,        /* the CUDA runtime reported an error; see qg_last_error() */
-    QG_ERR_UNSUPPORTED = 9  /* the device is not sm_100 or a feature is missing */
+    QG_ERR_UNSUPPORTED = 9, /* the device is not sm_100 or a feature is missing */
+    QG_ERR_WORKSPACE = 10   /* workspace given but smaller than qg_workspace_size() */
 } qg_status;
+
+/* Operations that may use a caller-provided workspace (qg_workspace_size). */
+typedef enum { QG_OP_GEMM_W4A16 = 0, QG_OP_GEMM_W8A8 = 1, QG_OP_GEMM_W4A8 = 2 } qg_op;
 
 typedef enum { QG_F16 = 0, QG_BF16 = 1 } qg_dtype;
 
@@ -104,10 +108,15 @@ qg_status qg_pack_nibbles(const uint8_t* codes, int K, int N, uint32_t* packed, 
  * packed   u32 [K/8][N] from qg_pack_nibbles of asymmetric codes.
  * scales   fp16 bits [K/group][N]; zeros u8 [K/group][N].
  * group    128 (the only group size the GEMM kernels take).
- * Rules: K % 128 == 0, N % 8 == 0.  Accumulation is fp32; the dequantized weight
- * is rounded once to the activation dtype before the tensor-core product.
- * workspace / ws_bytes are unused (pass NULL, 0); the split-K reduction runs in
- * on-chip distributed shared memory.
+ * Rules: K % 128 == 0, N % 8 == 0.  Accumulation is fp32.
+ * workspace: NULL, or a device buffer of at least
+ *   qg_workspace_size(QG_OP_GEMM_W4A16, M, K, N) bytes that was zero-filled before
+ *   its first use.  With a workspace, decode shapes (M <= 32 per launch, N % 16 == 0)
+ *   use the stream-K kernel, which keeps per-slab partial tiles and arrival
+ *   counters there; every call that completes leaves the counters at zero again.
+ *   After a device error (qg_device_status() != QG_OK) zero-fill it again.
+ *   The workspace must not be shared by calls that may run concurrently.
+ *   Without one, the split-K reduction runs in distributed shared memory (slower).
  * ------------------------------------------------------------------------ */
 qg_status qg_gemm_w4a16(const void* X, qg_dtype xdt, int M, int K, int N, const uint32_t* packed,
                         const uint16_t* scales, const uint8_t* zeros, int group, void* Y,
@@ -182,6 +191,10 @@ qg_status qg_smooth_scales(const uint16_t* Xcal, int Mc, const float* W, int K, 
  * ------------------------------------------------------------------------ */
 qg_status qg_quantize_w8_channel(const float* W, const float* s, int K, int N, int8_t* Wq, float* sw,
                                  qg_stream_t stream);
+
+/* Bytes of workspace the given operation and shape can use (0 = none).  The
+ * value depends only on (op, M, K, N) and on the current device. */
+size_t qg_workspace_size(qg_op op, int M, int K, int N);
 
 /* --------------------------------------------------------------------------
  * Status and diagnostics

@@ -100,3 +100,16 @@ def test_smooth_scales_rejects_alpha():
     f = q.lib().qg_smooth_scales
     assert f(A, 4, A, 16, 16, ctypes.c_float(1.5), A, A, None) == 2
     assert f(A, 4, A, 16, 16, ctypes.c_float(float("nan")), A, A, None) == 2
+
+
+def test_workspace_size_and_too_small_workspace():
+    import bit_quantized_gemm_group_b200 as q
+    L = q.lib()
+    need = L.qg_workspace_size(0, 32, 4096, 4096)
+    assert need > 0
+    assert L.qg_workspace_size(0, 1, 4096, 136) == 0       # N % 16 != 0: no workspace path
+    assert L.qg_workspace_size(1, 16, 4096, 11008) == 0    # W8A8 takes none
+    assert L.qg_workspace_size(0, 0, 4096, 4096) == 0
+    # a workspace smaller than required is refused before any launch
+    assert L.qg_gemm_w4a16(A, 1, 32, 4096, 4096, A, A, A, 128, A, A, need - 1, None) == 10
+    assert L.qg_gemm_w4a16(A, 1, 32, 4096, 4096, A, A, A, 128, A, B, need, None) == 3

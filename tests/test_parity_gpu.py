@@ -131,7 +131,7 @@ def test_smooth_quant_act_i8_bitexact(M, K, chan, mult):
 # ---------------------------------------------------------------------------
 # W4A16
 # ---------------------------------------------------------------------------
-def _w4a16_case(K, N, cfg, Ms, xdtype, rows=None):
+def _w4a16_case(K, N, cfg, Ms, xdtype, rows=None, workspace="auto", repeat=1):
     W = synth.workload_weights(cfg, K, N)
     codes, scales, zeros, packed = quant_w4_asym(W)
     c_o, s_o, z_o, _ = oracle.quantize_w4_asym(W)
@@ -141,8 +141,14 @@ def _w4a16_case(K, N, cfg, Ms, xdtype, rows=None):
     for M in Ms:
         X, Xb = synth.activations(M, K, xdtype, seed=M)
         Y = torch.full((M, N), float("nan"), dtype=tdt, device="cuda")   # poisoned: every element must be written
-        q.qg_gemm_w4a16(x_device(Xb, tdt), packed, scales, zeros, Y)
+        Xd = x_device(Xb, tdt)
+        q.qg_gemm_w4a16(Xd, packed, scales, zeros, Y, workspace=workspace)
         _status_ok()
+        for _ in range(repeat - 1):   # the workspace counters are back at zero: same bits again
+            Y2 = torch.full_like(Y, float("nan"))
+            q.qg_gemm_w4a16(Xd, packed, scales, zeros, Y2, workspace=workspace)
+            _status_ok()
+            assert torch.equal(Y2.view(torch.int16), Y.view(torch.int16))
         r = rows(M) if rows else None
         yref, b = oracle.gemm_w4a16_ref(X, p_o, s_o, z_o, rows=r)
         y = u16(Y)
@@ -161,11 +167,26 @@ def test_gemm_w4a16_decode_sweep(K, N):
     _w4a16_case(K, N, "w4a16_decode", synth.CONFIGS["w4a16_decode"]["M"], "bf16")
 
 
+@pytest.mark.parametrize("K,N", [(4096, 4096), (11008, 4096)])
+def test_gemm_w4a16_decode_without_workspace(K, N):
+    """The cluster/DSMEM split-K kernel (no workspace) on the same inputs."""
+    _w4a16_case(K, N, "w4a16_decode", [1, 16, 32], "bf16", workspace=None)
+
+
+def test_gemm_w4a16_decode_repeatable():
+    """Stream-K fixup: calls in a row give identical bits (deterministic reduction order,
+    arrival counters reset by the last arriver)."""
+    _w4a16_case(4096, 12288, "w4a16_decode", [1, 4, 32], "bf16", repeat=3)
+
+
 @pytest.mark.parametrize("xdtype", ["bf16", "f16"])
 def test_gemm_w4a16_edge_shapes(xdtype):
     # K = 3 groups, N not a multiple of any tile width, M across every token-tile boundary
     _w4a16_case(384, 136, "w4a16_decode", [1, 2, 3, 5, 7, 8, 9, 17, 31, 33, 63, 65, 127, 129], xdtype)
+    _w4a16_case(384, 144, "w4a16_decode", [1, 2, 3, 5, 7, 8, 9, 17, 31, 33, 63, 65, 127, 129], xdtype)  # ragged slab
     _w4a16_case(128, 8, "w4a16_decode", [1, 4], xdtype)
+    _w4a16_case(128, 16, "w4a16_decode", [1, 4, 32], xdtype)     # one group, one partial slab
+    _w4a16_case(2048, 4096, "w4a16_decode", [3, 12, 27], xdtype)  # fewer units per CTA than a stage
 
 
 # ---------------------------------------------------------------------------
