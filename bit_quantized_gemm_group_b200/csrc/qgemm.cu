@@ -210,11 +210,13 @@ DecodePlan decode_plan(int M, int K, int N)
     d.units = d.G * d.nslabs;
     d.grid = std::min(num_sms(), d.units);
     d.partial_bytes = (size_t)d.grid * 2 * qg::kDecBN * d.MP * sizeof(float);
-    d.counter_bytes = ((size_t)d.nslabs * sizeof(int) + 255) & ~size_t(255);
+    // The counter region has one fixed size for every shape, so that the counters of
+    // one call never overlap the partial tiles another shape wrote into the same buffer.
+    d.counter_bytes = (size_t)qg::kDecMaxSlabs * sizeof(int);
     return d;
 }
 
-bool decode_eligible(int M, int N) { return M >= 1 && N % 16 == 0; }
+bool decode_eligible(int M, int N) { return M >= 1 && N % 16 == 0 && (N + qg::kDecBN - 1) / qg::kDecBN <= qg::kDecMaxSlabs; }
 
 template <int MT, bool BF16>
 qg_status launch_w4a16_decode(const qg::SkinnyParams& sp, const uint32_t* packed, const uint16_t* scales,

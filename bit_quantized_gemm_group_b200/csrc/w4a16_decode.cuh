@@ -43,12 +43,13 @@ struct DecodeParams {
     const uint16_t* X;
     uint16_t* Y;
     float* partials;  // [grid][2][128][MP]
-    int* counters;    // [nslabs], zero between calls
+    int* counters;    // [kDecMaxSlabs], zero between calls
     int M, K, N;
     int G, nslabs, units, grid;
 };
 
 constexpr int kDecBN = 128;             // columns per slab
+constexpr int kDecMaxSlabs = 8192;      // counters at the start of the workspace: N <= 8192 * 128
 constexpr int kDecGroupsPerStage = 4;
 constexpr int kDecGroupW = 16 * 128 * 4;  // packed words of one group: 16 rows x 128 columns x 4 B
 constexpr int kDecStageBytes = 35840;   // 4 x 8 KB words + 4 x 256 B scales + 4 x 128 B zeros, 1 KB aligned

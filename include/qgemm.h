@@ -111,7 +111,7 @@ qg_status qg_pack_nibbles(const uint8_t* codes, int K, int N, uint32_t* packed, 
  * Rules: K % 128 == 0, N % 8 == 0.  Accumulation is fp32.
  * workspace: NULL, or a device buffer of at least
  *   qg_workspace_size(QG_OP_GEMM_W4A16, M, K, N) bytes that was zero-filled before
- *   its first use.  With a workspace, decode shapes (M <= 32 per launch, N % 16 == 0)
+ *   its first use.  With a workspace, decode shapes (N % 16 == 0, N <= 2^20)
  *   use the stream-K kernel, which keeps per-slab partial tiles and arrival
  *   counters there; every call that completes leaves the counters at zero again.
  *   After a device error (qg_device_status() != QG_OK) zero-fill it again.

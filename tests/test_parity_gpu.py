@@ -179,6 +179,15 @@ def test_gemm_w4a16_decode_repeatable():
     _w4a16_case(4096, 12288, "w4a16_decode", [1, 4, 32], "bf16", repeat=3)
 
 
+def test_gemm_w4a16_workspace_shared_across_shapes():
+    """One workspace serves calls of different shapes in turn: a call with many slabs after
+    one with few must find every arrival counter at zero (they sit at a fixed offset)."""
+    q = qlib()
+    ws = torch.zeros(q.qg_workspace_size(q.QG_OP_GEMM_W4A16, 32, 4096, 22016), dtype=torch.uint8, device="cuda")
+    for (K, N, M) in [(4096, 12288, 32), (4096, 22016, 1), (4096, 4096, 16), (4096, 22016, 32)]:
+        _w4a16_case(K, N, "w4a16_decode", [M], "bf16", workspace=ws)
+
+
 @pytest.mark.parametrize("xdtype", ["bf16", "f16"])
 def test_gemm_w4a16_edge_shapes(xdtype):
     # K = 3 groups, N not a multiple of any tile width, M across every token-tile boundary
