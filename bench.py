@@ -328,6 +328,40 @@ def run_reference(args, world, rank):
     print(json.dumps(line), flush=True)
 
 
+def run_single(spec, reps, workspace="auto"):
+    """--single K,N,M: one decode-sweep call shape, `reps` timed launches (no graph),
+    for profiling a kernel in isolation.  Prints per-launch device time."""
+    import bit_quantized_gemm_group_b200 as q
+    K, N, M = (int(x) for x in spec.split(","))
+    W = torch.from_numpy(synth.workload_weights("w4a16_decode", K, N)).cuda()
+    codes = torch.empty(K, N, dtype=torch.uint8, device="cuda")
+    scales = torch.empty(K // 128, N, dtype=torch.int16, device="cuda")
+    zeros = torch.empty(K // 128, N, dtype=torch.uint8, device="cuda")
+    packed = torch.empty(K // 8, N, dtype=torch.int32, device="cuda")
+    q.qg_quantize_w4_group(W, None, 128, False, codes, scales, zeros)
+    q.qg_pack_nibbles(codes, packed)
+    _, xb = synth.activations(M, K, "bf16", seed=M)
+    X = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    flush = torch.empty(2 * l2_bytes(), dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        q.qg_gemm_w4a16(X, packed, scales, zeros, Y, workspace=workspace)
+    torch.cuda.synchronize()
+    ts = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        q.qg_gemm_w4a16(X, packed, scales, zeros, Y, workspace=workspace)
+        b.record()
+        torch.cuda.synchronize()
+        ts.append(a.elapsed_time(b) * 1e3)
+    assert q.qg_device_status() == q.QG_OK
+    by = w4_bytes(K, N) + 2 * M * (K + N)
+    med = float(np.median(ts))
+    print(json.dumps({"single": [K, N, M], "us_median": med, "us_min": min(ts), "gbs": by / (med * 1e-6) / 1e9}))
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -336,8 +370,15 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="w4a16_decode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--single", default=None, help="K,N,M: time one decode call shape alone (profiling aid)")
+    ap.add_argument("--reps", type=int, default=5)
+    ap.add_argument("--no-workspace", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.single:
+        torch.cuda.set_device(0)
+        run_single(args.single, args.reps, None if args.no_workspace else "auto")
+        return
 
     if args.impl == "reference":
         rank = int(os.environ.get("RANK", "0"))

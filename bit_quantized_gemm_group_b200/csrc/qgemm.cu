@@ -222,7 +222,8 @@ template <int MT, bool BF16>
 qg_status launch_w4a16_decode(const qg::SkinnyParams& sp, const uint32_t* packed, const uint16_t* scales,
                               const uint8_t* zeros, void* ws, qg_stream_t stream)
 {
-    constexpr int ST = MT <= 2 ? 4 : 3;
+    constexpr int ST = MT == 1 ? 4 : MT == 2 ? 3 : 2;  // ring depth that fits next to the reduction buffer
+    static_assert(qg::DecodeSmem<MT, ST>::TOTAL <= 227 * 1024, "decode kernel shared memory");
     auto kern = qg::w4a16_decode_kernel<MT, BF16, ST>;
     const size_t smem = qg::DecodeSmem<MT, ST>::TOTAL;
     static KernelInfo info;
@@ -240,6 +241,10 @@ qg_status launch_w4a16_decode(const qg::SkinnyParams& sp, const uint32_t* packed
     if ((st = make_tmap_2d(&tz, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, zeros, sp.N, d.G, 128, 1,
                            CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK)
         return st;
+    CUtensorMap tx;
+    if ((st = make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, sp.X, sp.K, sp.M, 64, 8 * MT,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
+        return st;
     qg::DecodeParams p;
     p.X = sp.X;
     p.Y = sp.Y;
@@ -252,8 +257,19 @@ qg_status launch_w4a16_decode(const qg::SkinnyParams& sp, const uint32_t* packed
     p.nslabs = d.nslabs;
     p.units = d.units;
     p.grid = d.grid;
-    kern<<<d.grid, 384, smem, reinterpret_cast<cudaStream_t>(stream)>>>(p, tw, ts, tz);
-    QG_CUDA(cudaGetLastError());
+    // programmatic dependent launch: this grid may start while the previous kernel in
+    // the stream drains; the kernel orders itself with griddepcontrol.wait.
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(d.grid);
+    cfg.blockDim = dim3(384);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    QG_CUDA(cudaLaunchKernelEx(&cfg, kern, p, tw, ts, tz, tx));
     return QG_OK;
 }
 

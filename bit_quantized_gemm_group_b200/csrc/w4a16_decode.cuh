@@ -52,32 +52,39 @@ constexpr int kDecBN = 128;             // columns per slab
 constexpr int kDecMaxSlabs = 8192;      // counters at the start of the workspace: N <= 8192 * 128
 constexpr int kDecGroupsPerStage = 4;
 constexpr int kDecGroupW = 16 * 128 * 4;  // packed words of one group: 16 rows x 128 columns x 4 B
-constexpr int kDecStageBytes = 35840;   // 4 x 8 KB words + 4 x 256 B scales + 4 x 128 B zeros, 1 KB aligned
 constexpr int kDecScaleOff = 4 * kDecGroupW;
 constexpr int kDecZeroOff = kDecScaleOff + 4 * 256;
+constexpr int kDecXOff = kDecZeroOff + 4 * 128 + 512;  // 1 KB aligned
 
 QG_DEV_INLINE int dec_first_unit(int c, int units, int grid) { return (int)((int64_t)c * units / grid); }
 
+// Stage: 4 groups x {packed words 8 KB, fp16 scales 256 B, u8 zeros 128 B, X tile
+// MP tokens x 128 k bf16 as two 128-byte-swizzled boxes of 64 k}.
 template <int MT, int ST>
 struct DecodeSmem {
     static constexpr int MP = 8 * MT;
+    static constexpr int XG = MP * 256;  // X bytes per group
+    static constexpr int STAGE = kDecXOff + 4 * XG;
     static constexpr int RED = 4 * kDecBN * MP * 4;
-    static constexpr int TOTAL = ST * kDecStageBytes + RED + 2 * ST * 8 + 64 + 1024;
+    static constexpr int TOTAL = ST * STAGE + RED + 2 * ST * 8 + 64 + 1024;
+    static constexpr uint32_t GROUP_TX = kDecGroupW + 256 + 128 + XG;
 };
 
 template <int MT, bool BF16, int ST>
 __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams p,
                                                                const __grid_constant__ CUtensorMap tm_w,
                                                                const __grid_constant__ CUtensorMap tm_s,
-                                                               const __grid_constant__ CUtensorMap tm_z)
+                                                               const __grid_constant__ CUtensorMap tm_z,
+                                                               const __grid_constant__ CUtensorMap tm_x)
 {
     using H = HalfOps<BF16>;
     constexpr int MP = 8 * MT;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    using L = DecodeSmem<MT, ST>;
     uint8_t* ring = smem;
-    float* red = reinterpret_cast<float*>(smem + ST * kDecStageBytes);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * kDecStageBytes + DecodeSmem<MT, ST>::RED);
+    float* red = reinterpret_cast<float*>(smem + ST * L::STAGE);
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * L::STAGE + L::RED);
     uint64_t* empty = full + ST;
     int* flag = reinterpret_cast<int*>(empty + ST);
 
@@ -85,6 +92,9 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
     const int G = p.G;
     const int u0 = dec_first_unit(blockIdx.x, p.units, p.grid), u1 = dec_first_unit(blockIdx.x + 1, p.units, p.grid);
 
+    // The next grid in the stream may start launching now; it waits for this one to
+    // finish (griddepcontrol.wait) before it touches X, Y or the workspace.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0) {
         for (int i = 0; i < ST; ++i) {
             mbar_init(&full[i], 1);
@@ -103,16 +113,21 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
             tma_prefetch_desc(&tm_w);
             tma_prefetch_desc(&tm_s);
             tma_prefetch_desc(&tm_z);
-            int stage = 0;
+            tma_prefetch_desc(&tm_x);
+            // Weights, scales and zeros do not depend on the previous grid: the first
+            // ring-full of them is requested before waiting for it; X after.
+            int stage = 0, issued = 0;
             uint32_t phase = 0;
+            bool waited = false;
+            int pend_g0[ST], pend_ng[ST];
             for (int u = u0; u < u1;) {
                 const int slab = u / G, ga = u % G;
                 const int gb = min(G, ga + (u1 - u));
                 for (int g0 = ga; g0 < gb; g0 += kDecGroupsPerStage) {
                     const int ng = min(kDecGroupsPerStage, gb - g0);
                     if (!mbar_wait(&empty[stage], phase ^ 1)) return;
-                    mbar_arrive_expect_tx(&full[stage], (uint32_t)ng * (kDecGroupW + 256 + 128));
-                    uint8_t* st = ring + stage * kDecStageBytes;
+                    mbar_arrive_expect_tx(&full[stage], (uint32_t)ng * L::GROUP_TX);
+                    uint8_t* st = ring + stage * L::STAGE;
                     for (int i = 0; i < ng; ++i) {
                         const int g = g0 + i;
 #pragma unroll
@@ -122,6 +137,30 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
                         tma_load_2d(&tm_s, &full[stage], st + kDecScaleOff + i * 256, slab * kDecBN, g);
                         tma_load_2d(&tm_z, &full[stage], st + kDecZeroOff + i * 128, slab * kDecBN, g);
                     }
+                    if (!waited && issued < ST) {
+                        pend_g0[issued] = g0;
+                        pend_ng[issued] = ng;
+                    }
+                    if (!waited && (issued + 1 == ST || (g0 + kDecGroupsPerStage >= gb && u + (gb - ga) >= u1))) {
+                        // ring full (or schedule done): now wait for the previous grid, then load X
+                        asm volatile("griddepcontrol.wait;" ::: "memory");
+                        waited = true;
+                        for (int j = 0; j <= issued; ++j) {
+                            uint8_t* sj = ring + j * L::STAGE;
+                            for (int i = 0; i < pend_ng[j]; ++i)
+#pragma unroll
+                                for (int b = 0; b < 2; ++b)
+                                    tma_load_2d(&tm_x, &full[j], sj + kDecXOff + i * L::XG + b * (L::XG / 2),
+                                                128 * (pend_g0[j] + i) + 64 * b, 0);
+                        }
+                    } else if (waited) {
+                        for (int i = 0; i < ng; ++i)
+#pragma unroll
+                            for (int b = 0; b < 2; ++b)
+                                tma_load_2d(&tm_x, &full[stage], st + kDecXOff + i * L::XG + b * (L::XG / 2),
+                                            128 * (g0 + i) + 64 * b, 0);
+                    }
+                    ++issued;
                     if (++stage == ST) { stage = 0; phase ^= 1; }
                 }
                 u += gb - ga;
@@ -132,6 +171,7 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
 
     // ---------------- consumers ----------------
     asm volatile("setmaxnreg.inc.sync.aligned.u32 232;");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     const int wn = warp & 1, wg = warp >> 1;
     const int g8 = lane >> 2, t4 = lane & 3;
     const uint32_t ONE = BF16 ? 0x3F803F80u : 0x3C003C00u;
@@ -159,7 +199,7 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
         for (int g0 = ga; g0 < gb; g0 += kDecGroupsPerStage) {
             const int ng = min(kDecGroupsPerStage, gb - g0);
             if (ok && !mbar_wait(&full[stage], phase)) ok = false;
-            const uint8_t* st = ring + stage * kDecStageBytes;
+            const uint8_t* st = ring + stage * L::STAGE;
             if (ok && wg < ng) {
                 const int g = g0 + wg;
                 // per-column scale and (128 + z) of the lane's 8 columns
@@ -198,11 +238,11 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
                         wv[h] = *reinterpret_cast<const uint4*>(wbase + (2 * wn + h) * 2048 + row * 128 +
                                                                 ((g8 ^ (row & 7)) << 4));
                     uint32_t xb[MT][4];
+                    const uint8_t* xs = st + kDecXOff + wg * L::XG + (row >> 3) * (L::XG / 2);
 #pragma unroll
                     for (int j = 0; j < MT; ++j) {
-                        const int tok = 8 * j + g8;
-                        uint4 xv = make_uint4(0u, 0u, 0u, 0u);
-                        if (tok < p.M) xv = ldg_v4(p.X + (int64_t)tok * p.K + 128 * g + 8 * row);
+                        const int tok = 8 * j + g8;  // rows >= M are zero (TMA fill)
+                        const uint4 xv = *reinterpret_cast<const uint4*>(xs + tok * 128 + (((row & 7) ^ (tok & 7)) << 4));
                         xb[j][0] = prmt(xv.x, xv.z, 0x5410);
                         xb[j][1] = prmt(xv.x, xv.z, 0x7632);
                         xb[j][2] = prmt(xv.y, xv.w, 0x5410);
@@ -288,9 +328,9 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
             const int slot = first_piece ? 0 : 1;
             float* mine = p.partials + ((size_t)blockIdx.x * 2 + slot) * kDecBN * MP;
             for (int e = threadIdx.x; e < kDecBN * MP; e += 256) mine[e] = red[e];
-            __threadfence();
             named_bar_sync(1, 256);
             if (threadIdx.x == 0) {
+                __threadfence();  // the CTA's partial stores (ordered by the barrier) before the arrival
                 // CTAs that hold a piece of this slab: the ones containing its first and last unit
                 const int ufirst = slab * G, ulast = slab * G + G - 1;
                 int cf = (int)((int64_t)ufirst * p.grid / p.units);
@@ -304,11 +344,13 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
                 flag[0] = last ? 1 : 0;
                 flag[1] = cf;
                 flag[2] = cl;
-                if (last) p.counters[slab] = 0;
+                if (last) {
+                    p.counters[slab] = 0;
+                    __threadfence();  // acquire: the other pieces' partials are visible from here on
+                }
             }
             named_bar_sync(1, 256);
             if (flag[0]) {
-                __threadfence();
                 const int cf = flag[1], cl = flag[2];
                 for (int e = threadIdx.x; e < p.M * kDecBN; e += 256) {
                     const int tok = e / kDecBN, nn = e % kDecBN;
