@@ -208,7 +208,7 @@ DecodePlan decode_plan(int M, int K, int N)
     d.G = K / 128;
     d.nslabs = (N + qg::kDecBN - 1) / qg::kDecBN;
     d.units = d.G * d.nslabs;
-    d.grid = std::min(num_sms(), d.units);
+    d.grid = std::min(std::min(num_sms(), d.units), qg::kMaxPieces);
     d.partial_bytes = (size_t)d.grid * 2 * qg::kDecBN * d.MP * sizeof(float);
     // The counter region has one fixed size for every shape, so that the counters of
     // one call never overlap the partial tiles another shape wrote into the same buffer.

@@ -55,6 +55,7 @@ constexpr int kDecGroupW = 16 * 128 * 4;  // packed words of one group: 16 rows 
 constexpr int kDecScaleOff = 4 * kDecGroupW;
 constexpr int kDecZeroOff = kDecScaleOff + 4 * 256;
 constexpr int kDecXOff = kDecZeroOff + 4 * 128 + 512;  // 1 KB aligned
+constexpr int kMaxPieces = 160;         // >= grid: pieces of one slab (one per CTA at most)
 
 QG_DEV_INLINE int dec_first_unit(int c, int units, int grid) { return (int)((int64_t)c * units / grid); }
 
@@ -65,8 +66,9 @@ struct DecodeSmem {
     static constexpr int MP = 8 * MT;
     static constexpr int XG = MP * 256;  // X bytes per group
     static constexpr int STAGE = kDecXOff + 4 * XG;
-    static constexpr int RED = 4 * kDecBN * MP * 4;
-    static constexpr int TOTAL = ST * STAGE + RED + 2 * ST * 8 + 64 + 1024;
+    static constexpr int RS = kDecBN + 8;  // padded row of the [token][column] reduction tile
+    static constexpr int RED = 4 * MP * RS * 4;
+    static constexpr int TOTAL = ST * STAGE + RED + 2 * ST * 8 + 64 + 4 * kMaxPieces + 1024;
     static constexpr uint32_t GROUP_TX = kDecGroupW + 256 + 128 + XG;
 };
 
@@ -86,7 +88,8 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
     float* red = reinterpret_cast<float*>(smem + ST * L::STAGE);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * L::STAGE + L::RED);
     uint64_t* empty = full + ST;
-    int* flag = reinterpret_cast<int*>(empty + ST);
+    int* flag = reinterpret_cast<int*>(empty + ST);            // [16]
+    int* piece_off = flag + 16;                                   // [kMaxPieces] partial-tile offsets
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.G;
@@ -291,7 +294,10 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
             if (++stage == ST) { stage = 0; phase ^= 1; }
         }
         // ---------------- piece end: reduce the four group-warps, then write ----------------
-        float* myred = red + (size_t)wg * kDecBN * MP;
+        // Reduction tile layout [token][column] with a padded row, so that the fragment
+        // stores are at most 2-way conflicted and every later pass reads consecutive words.
+        constexpr int RS = L::RS;
+        float* myred = red + (size_t)wg * MP * RS;
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -300,18 +306,23 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
                 for (int j = 0; j < MT; ++j) {
                     const int nl = 64 * wn + 32 * h + 4 * g8 + 2 * cp;
                     const int tk = 8 * j + 2 * t4;
-                    *reinterpret_cast<float2*>(myred + (size_t)nl * MP + tk) = make_float2(acc[h][cp][j][0], acc[h][cp][j][1]);
-                    *reinterpret_cast<float2*>(myred + (size_t)(nl + 1) * MP + tk) =
-                        make_float2(acc[h][cp][j][2], acc[h][cp][j][3]);
+                    *reinterpret_cast<float2*>(myred + tk * RS + nl) = make_float2(acc[h][cp][j][0], acc[h][cp][j][2]);
+                    *reinterpret_cast<float2*>(myred + (tk + 1) * RS + nl) = make_float2(acc[h][cp][j][1], acc[h][cp][j][3]);
 #pragma unroll
                     for (int e = 0; e < 4; ++e) acc[h][cp][j][e] = 0.0f;
                 }
         named_bar_sync(1, 256);
-        for (int e = threadIdx.x; e < kDecBN * MP; e += 256) {
-            float v = red[e];
+        const int mrows = min(p.M, MP);
+        // sum the four group-warps: 4 consecutive columns per thread step
+        for (int e = threadIdx.x; e < mrows * (kDecBN / 4); e += 256) {
+            const int tok = e / (kDecBN / 4), c4 = 4 * (e % (kDecBN / 4));
+            float4 v = *reinterpret_cast<const float4*>(red + tok * RS + c4);
 #pragma unroll
-            for (int q = 1; q < 4; ++q) v += red[(size_t)q * kDecBN * MP + e];
-            red[e] = v;
+            for (int q = 1; q < 4; ++q) {
+                const float4 w = *reinterpret_cast<const float4*>(red + (size_t)q * MP * RS + tok * RS + c4);
+                v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
+            }
+            *reinterpret_cast<float4*>(red + tok * RS + c4) = v;
         }
         named_bar_sync(1, 256);
         const int nvalid = min(kDecBN, p.N - n0);
@@ -320,14 +331,18 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
         if (!all_ok) {
             ok = false;
         } else if (ga == 0 && gb == G) {
-            for (int e = threadIdx.x; e < p.M * kDecBN; e += 256) {
+            for (int e = threadIdx.x; e < mrows * kDecBN; e += 256) {
                 const int tok = e / kDecBN, nn = e % kDecBN;
-                if (nn < nvalid) p.Y[(int64_t)tok * p.N + n0 + nn] = H::to_bits(red[nn * MP + tok]);
+                if (nn < nvalid) p.Y[(int64_t)tok * p.N + n0 + nn] = H::to_bits(red[tok * RS + nn]);
             }
         } else {
+            // partial tile [token][128] in the workspace, then arrive on the slab's counter
             const int slot = first_piece ? 0 : 1;
             float* mine = p.partials + ((size_t)blockIdx.x * 2 + slot) * kDecBN * MP;
-            for (int e = threadIdx.x; e < kDecBN * MP; e += 256) mine[e] = red[e];
+            for (int e = threadIdx.x; e < mrows * (kDecBN / 4); e += 256) {
+                const int tok = e / (kDecBN / 4), c4 = 4 * (e % (kDecBN / 4));
+                *reinterpret_cast<float4*>(mine + tok * kDecBN + c4) = *reinterpret_cast<const float4*>(red + tok * RS + c4);
+            }
             named_bar_sync(1, 256);
             if (threadIdx.x == 0) {
                 __threadfence();  // the CTA's partial stores (ordered by the barrier) before the arrival
@@ -342,25 +357,39 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
                 const int old = atomicAdd(&p.counters[slab], 1);
                 const bool last = old == cl - cf;
                 flag[0] = last ? 1 : 0;
-                flag[1] = cf;
-                flag[2] = cl;
+                flag[1] = cl - cf + 1;
                 if (last) {
                     p.counters[slab] = 0;
+                    for (int c = cf; c <= cl; ++c) {
+                        const int sl = dec_first_unit(c, p.units, p.grid) >= slab * G ? 0 : 1;
+                        piece_off[c - cf] = (c * 2 + sl) * kDecBN * MP;
+                    }
                     __threadfence();  // acquire: the other pieces' partials are visible from here on
                 }
             }
             named_bar_sync(1, 256);
             if (flag[0]) {
-                const int cf = flag[1], cl = flag[2];
-                for (int e = threadIdx.x; e < p.M * kDecBN; e += 256) {
-                    const int tok = e / kDecBN, nn = e % kDecBN;
-                    if (nn >= nvalid) continue;
-                    float v = 0.0f;
-                    for (int c = cf; c <= cl; ++c) {
-                        const int sl = dec_first_unit(c, p.units, p.grid) >= slab * G ? 0 : 1;
-                        v += __ldcg(p.partials + ((size_t)c * 2 + sl) * kDecBN * MP + nn * MP + tok);
+                const int np = flag[1];
+                for (int e = threadIdx.x; e < mrows * (kDecBN / 4); e += 256) {
+                    const int tok = e / (kDecBN / 4), c4 = 4 * (e % (kDecBN / 4));
+                    const int off = tok * kDecBN + c4;
+                    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                    int i = 0;
+                    for (; i + 4 <= np; i += 4) {  // four independent loads in flight, summed in piece order
+                        float4 a[4];
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) a[r] = __ldcg(reinterpret_cast<const float4*>(p.partials + piece_off[i + r] + off));
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) { v.x += a[r].x; v.y += a[r].y; v.z += a[r].z; v.w += a[r].w; }
                     }
-                    p.Y[(int64_t)tok * p.N + n0 + nn] = H::to_bits(v);
+                    for (; i < np; ++i) {
+                        const float4 a = __ldcg(reinterpret_cast<const float4*>(p.partials + piece_off[i] + off));
+                        v.x += a.x; v.y += a.y; v.z += a.z; v.w += a.w;
+                    }
+                    const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int r = 0; r < 4; ++r)
+                        if (c4 + r < nvalid) p.Y[(int64_t)tok * p.N + n0 + c4 + r] = H::to_bits(vv[r]);
                 }
             }
         }
