@@ -292,6 +292,94 @@ qg_status w4a16_decode_dispatch(qg::SkinnyParams p, const uint32_t* packed, cons
 }
 
 // ---------------------------------------------------------------------------
+// tcgen05 tile kernels (M >= kTcMinM)
+// ---------------------------------------------------------------------------
+template <int KIND>
+qg_status launch_tc(const qg::TcParams& p, const CUtensorMap& ta, const CUtensorMap& tb, qg_stream_t stream)
+{
+    using C = qg::TcCfg<KIND>;
+    auto kern = qg::tc_gemm_kernel<KIND>;
+    const size_t smem = qg::TcSmem<KIND>::TOTAL;
+    static_assert(qg::TcSmem<KIND>::TOTAL <= 227 * 1024, "tile kernel shared memory");
+    static KernelInfo info;
+    int occ = 1;
+    qg_status st = prepare_kernel(info, kern, C::THREADS, smem, &occ);
+    if (st != QG_OK) return st;
+    const int tiles = p.m_tiles * p.n_tiles;
+    const int grid = std::min(tiles, num_sms());
+    kern<<<grid, C::THREADS, smem, reinterpret_cast<cudaStream_t>(stream)>>>(p, ta, tb);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+
+qg_status tc_w8a8(const qg::TcInt8Args& a, qg_stream_t stream)
+{
+    using C = qg::TcCfg<qg::TC_W8A8>;
+    CUtensorMap ta, tb;
+    qg_status st;
+    if ((st = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.Xq, a.K, a.M, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)))
+        return st;
+    if ((st = make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.Wq, a.N, a.K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)))
+        return st;
+    qg::TcParams p{};
+    p.t = a.t;
+    p.sw = a.sw;
+    p.Y = a.Y;
+    p.dbg = a.dbg;
+    p.M = a.M;
+    p.K = a.K;
+    p.N = a.N;
+    p.m_tiles = (a.M + C::BM - 1) / C::BM;
+    p.n_tiles = (a.N + C::BN - 1) / C::BN;
+    return launch_tc<qg::TC_W8A8>(p, ta, tb, stream);
+}
+
+qg_status tc_w4a8(const qg::TcInt8Args& a, qg_stream_t stream)
+{
+    using C = qg::TcCfg<qg::TC_W4A8>;
+    CUtensorMap ta, tb;
+    qg_status st;
+    if ((st = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.Xq, a.K, a.M, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)))
+        return st;
+    if ((st = make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, a.N, a.K / 8, 128, 16,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)))
+        return st;
+    qg::TcParams p{};
+    p.t = a.t;
+    p.sg = a.sg;
+    p.Y = a.Y;
+    p.dbg = a.dbg;
+    p.M = a.M;
+    p.K = a.K;
+    p.N = a.N;
+    p.m_tiles = (a.M + C::BM - 1) / C::BM;
+    p.n_tiles = (a.N + C::BN - 1) / C::BN;
+    return launch_tc<qg::TC_W4A8>(p, ta, tb, stream);
+}
+
+qg_status tc_w4a16(const qg::TcW4A16Args& a, qg_stream_t stream)
+{
+    using C = qg::TcCfg<qg::TC_W4A16>;
+    CUtensorMap ta, tb;
+    qg_status st;
+    if ((st = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.X, a.K, a.M, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)))
+        return st;
+    if ((st = make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, a.N, a.K / 8, 128, 8,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)))
+        return st;
+    qg::TcParams p{};
+    p.scales = a.scales;
+    p.zeros = a.zeros;
+    p.Y = a.Y;
+    p.M = a.M;
+    p.K = a.K;
+    p.N = a.N;
+    p.m_tiles = (a.M + C::BM - 1) / C::BM;
+    p.n_tiles = (a.N + C::BN - 1) / C::BN;
+    return launch_tc<qg::TC_W4A16>(p, ta, tb, stream);
+}
+
+// ---------------------------------------------------------------------------
 // int8 skinny paths
 // ---------------------------------------------------------------------------
 template <int MT>
@@ -418,7 +506,7 @@ qg_status qg_gemm_w4a16(const void* X, qg_dtype xdt, int M, int K, int N, const 
         return QG_ERR_ALIGN;
     if (xdt == QG_BF16 && M >= qg::kTcMinM) {
         qg::TcW4A16Args a{static_cast<const uint16_t*>(X), packed, scales, zeros, static_cast<uint16_t*>(Y), M, K, N};
-        return qg::tc_w4a16_launch(a, stream);
+        return tc_w4a16(a, stream);
     }
     qg::SkinnyParams p{static_cast<const uint16_t*>(X), packed, scales, zeros, static_cast<uint16_t*>(Y), M, K, N};
     if (workspace && decode_eligible(M, N)) {
@@ -454,7 +542,7 @@ qg_status qg_gemm_w8a8(const int8_t* Xq, const float* t, int M, int K, const int
         return QG_ERR_ALIGN;
     if (M >= qg::kTcMinM) {
         qg::TcInt8Args a{Xq, t, Wq, sw, nullptr, nullptr, Y, acc_dbg, M, K, N};
-        return qg::tc_w8a8_launch(a, stream);
+        return tc_w8a8(a, stream);
     }
     for (int m0 = 0; m0 < M; m0 += 16) {
         qg::Int8SkinnyParams p{Xq + (int64_t)m0 * K, t + m0, Wq, sw, nullptr, nullptr, Y + (int64_t)m0 * N,
@@ -479,7 +567,7 @@ qg_status qg_gemm_w4a8(const int8_t* Xq, const float* t, int M, int K, const uin
         return QG_ERR_ALIGN;
     if (M >= qg::kTcMinM) {
         qg::TcInt8Args a{Xq, t, nullptr, nullptr, packed, sg, Y, part_dbg, M, K, N};
-        return qg::tc_w4a8_launch(a, stream);
+        return tc_w4a8(a, stream);
     }
     const int G = K / 128;
     for (int m0 = 0; m0 < M; m0 += 32) {

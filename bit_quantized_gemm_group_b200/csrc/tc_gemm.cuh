@@ -1,4 +1,26 @@
-// tc_gemm.cuh -- tcgen05 (TMEM accumulator, TMA-fed) tile kernels for prefill shapes.
+// tc_gemm.cuh -- tcgen05 tile kernels for prefill-size M (tensor memory accumulators,
+// TMA-fed operands, warp-specialised, persistent).
+//
+// One template covers three products (KIND):
+//   W8A8  acc = Xq Wq (int8 x int8 -> int32 in TMEM), Y = bf16((acc * t[m]) * sw[n])
+//         ("AI Infra guide, ch.4 Quantization" sec. 2.2-2.3, SmoothQuant)
+//   W4A16 Y = X (q - z) s with the dequantized bf16 weight tile built in shared memory
+//         by dequant warps ("AI Infra guide" sec. 3.1, 3.5; group-wise scale/zero:
+//         "LLM inference cost: W8A8/W4A8 ..." sec. 2.2)
+//   W4A8  P_g = Xq q4 per group of 128 (int32 in TMEM, ping-pong), Y = bf16(t[m] sum_g P_g s[g][n])
+//         ("LLM inference cost: W8A8/W4A8 ..." sec. 2.2)
+//
+// Roles (one CTA per SM, persistent over output tiles, n-tile-major order so that
+// concurrently running CTAs share the weight tile through L2):
+//   warp 0        TMA producer: activation tile and (W8A8) weight tile, or the packed
+//                 weight words (W4A16, W4A8), into a ring of shared-memory stages.
+//   warp 1        TMEM allocator and MMA issuer (one elected lane issues tcgen05.mma
+//                 and tcgen05.commit; commits release ring stages and publish results).
+//   warps 2..5    epilogue: tcgen05.ld from TMEM, scale, convert, store.
+//   warps 6..9    (W4A16, W4A8) dequant: unpack nibbles from the raw stage and write the
+//                 K-major, 128-byte-swizzled B tile the MMA reads.
+// Every wait is bounded (mbar_wait); a wait that gives up records QG_ERR_TIMEOUT and
+// its role stops issuing work.  No TMA multicast is used anywhere.
 #pragma once
 #include <climits>
 
@@ -8,7 +30,9 @@
 namespace qg {
 
 // Smallest M routed to the tensor-memory tile kernels (smaller M uses the skinny paths).
-constexpr int kTcMinM = INT_MAX;
+constexpr int kTcMinM = 128;
+
+enum TcKind { TC_W8A8 = 0, TC_W4A16 = 1, TC_W4A8 = 2 };
 
 struct TcW4A16Args {
     const uint16_t* X;
@@ -31,9 +55,412 @@ struct TcInt8Args {
     int M, K, N;
 };
 
-inline qg_status tc_w4a16_launch(const TcW4A16Args&, qg_stream_t) { return QG_ERR_UNSUPPORTED; }
-inline qg_status tc_w8a8_launch(const TcInt8Args&, qg_stream_t) { return QG_ERR_UNSUPPORTED; }
-inline qg_status tc_w4a8_launch(const TcInt8Args&, qg_stream_t) { return QG_ERR_UNSUPPORTED; }
+template <int KIND>
+struct TcCfg;
+
+// W8A8: tile 128 x 256, k-block 128 int8; A 16 KB + B 32 KB per stage.
+template <>
+struct TcCfg<TC_W8A8> {
+    static constexpr int BM = 128, BN = 256, BK = 128;
+    static constexpr int A_BYTES = 128 * 128, B_BYTES = 256 * 128, RAW_BYTES = 0;
+    static constexpr int STAGE = A_BYTES + B_BYTES;
+    static constexpr int ST = 4;
+    static constexpr int THREADS = 192;
+    static constexpr int TMEM_COLS = 512;  // two 256-column accumulators
+    static constexpr int MH = 1;           // M=128 MMAs per tile
+};
+
+// W4A16: tile 256 x 128 (two M=128 MMAs share one dequantized B tile), k-block 64 bf16;
+// A 2 x 16 KB, raw packed words 8 x 128 x 4 B = 4 KB, B 128 x 64 bf16 = 16 KB per stage.
+template <>
+struct TcCfg<TC_W4A16> {
+    static constexpr int BM = 256, BN = 128, BK = 64;
+    static constexpr int A_BYTES = 2 * 128 * 128, RAW_BYTES = 8 * 128 * 4, B_BYTES = 128 * 128;
+    static constexpr int STAGE = A_BYTES + B_BYTES + 4096;  // raw area padded to 4 KB
+    static constexpr int ST = 4;
+    static constexpr int THREADS = 320;
+    static constexpr int TMEM_COLS = 512;  // two tiles x (2 halves x 128 columns)
+    static constexpr int MH = 2;
+};
+
+// W4A8: tile 128 x 128, k-block = one group of 128 int8; A 16 KB, raw 16 x 128 x 4 B = 8 KB,
+// B 128 x 128 int8 = 16 KB per stage; TMEM holds two group accumulators (ping-pong).
+template <>
+struct TcCfg<TC_W4A8> {
+    static constexpr int BM = 128, BN = 128, BK = 128;
+    static constexpr int A_BYTES = 128 * 128, RAW_BYTES = 16 * 128 * 4, B_BYTES = 128 * 128;
+    static constexpr int STAGE = A_BYTES + B_BYTES + RAW_BYTES;
+    static constexpr int ST = 4;
+    static constexpr int THREADS = 320;
+    static constexpr int TMEM_COLS = 256;
+    static constexpr int MH = 1;
+};
+
+template <int KIND>
+struct TcSmem {
+    using C = TcCfg<KIND>;
+    static constexpr int BAR_OFF = C::ST * C::STAGE;
+    static constexpr int TOTAL = BAR_OFF + 256 + 1024;  // barriers + tmem address + alignment slack
+};
+
+struct TcParams {
+    const float* t;     // W8A8, W4A8: per-token scale
+    const float* sw;    // W8A8: per-channel scale
+    const float* sg;    // W4A8: per-group scale [K/128][N]
+    const uint16_t* scales;  // W4A16: fp16 [K/128][N]
+    const uint8_t* zeros;    // W4A16: u8 [K/128][N]
+    uint16_t* Y;
+    int32_t* dbg;
+    int M, K, N;
+    int m_tiles, n_tiles;
+};
+
+// instruction descriptors (tcgen05 "kind::f16" / "kind::i8"), M = 128
+__host__ __device__ constexpr uint32_t idesc_bf16(int n)
+{
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+}
+__host__ __device__ constexpr uint32_t idesc_s8(int n, bool b_mn_major)
+{
+    return (2u << 4) | (1u << 7) | (1u << 10) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(n >> 3) << 17) |
+           ((uint32_t)(128 >> 4) << 24);
+}
+
+// bf16x2 of (128 + nibble j, 128 + nibble j+4) -> natural pairs after one subtract and
+// one multiply; see the decode kernel for the exponent trick.
+QG_DEV_INLINE uint32_t bf16x2_sub(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+QG_DEV_INLINE uint32_t bf16x2_mul(uint32_t a, uint32_t b)
+{
+    uint32_t r;
+    asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+template <int KIND>
+__global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
+    tc_gemm_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b)
+{
+    using C = TcCfg<KIND>;
+    using S = TcSmem<KIND>;
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::BAR_OFF);
+    uint64_t* empty = full + C::ST;
+    uint64_t* bready = empty + C::ST;      // dequant -> MMA
+    uint64_t* tfull = bready + C::ST;      // MMA -> epilogue (2)
+    uint64_t* tempty = tfull + 2;          // epilogue -> MMA (2)
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(tempty + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int KB = p.K / C::BK;
+    const int num_tiles = p.m_tiles * p.n_tiles;
+
+    if (threadIdx.x == 0) {
+        for (int i = 0; i < C::ST; ++i) {
+            mbar_init(&full[i], 1);
+            mbar_init(&empty[i], 1);
+            mbar_init(&bready[i], 4);
+        }
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&tfull[i], 1);
+            mbar_init(&tempty[i], 4);
+        }
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, C::TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+
+    if (warp == 0) {
+        // ------------------------------ TMA producer ------------------------------
+        if (lane == 0) {
+            tma_prefetch_desc(&tm_a);
+            tma_prefetch_desc(&tm_b);
+            int s = 0;
+            uint32_t ph = 0;
+            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+                const int m0 = (tile % p.m_tiles) * C::BM, n0 = (tile / p.m_tiles) * C::BN;
+                for (int kb = 0; kb < KB; ++kb) {
+                    if (!mbar_wait(&empty[s], ph ^ 1)) goto producer_done;
+                    uint8_t* st = smem + s * C::STAGE;
+                    if constexpr (KIND == TC_W8A8) {
+                        mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::B_BYTES);
+                        tma_load_2d(&tm_a, &full[s], st, kb * 128, m0);
+                        tma_load_2d(&tm_b, &full[s], st + C::A_BYTES, n0, kb * 128);
+                        tma_load_2d(&tm_b, &full[s], st + C::A_BYTES + 16384, n0 + 128, kb * 128);
+                    } else if constexpr (KIND == TC_W4A16) {
+                        mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::RAW_BYTES);
+                        tma_load_2d(&tm_a, &full[s], st, kb * 64, m0);
+                        tma_load_2d(&tm_a, &full[s], st + 16384, kb * 64, m0 + 128);
+                        tma_load_2d(&tm_b, &full[s], st + C::A_BYTES + C::B_BYTES, n0, kb * 8);
+                    } else {
+                        mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::RAW_BYTES);
+                        tma_load_2d(&tm_a, &full[s], st, kb * 128, m0);
+                        tma_load_2d(&tm_b, &full[s], st + C::A_BYTES + C::B_BYTES, n0, kb * 16);
+                    }
+                    if (++s == C::ST) { s = 0; ph ^= 1; }
+                }
+            }
+        }
+    producer_done:;
+    } else if (warp == 1) {
+        // ------------------------------ MMA issuer ------------------------------
+        if (lane == 0) {
+            int s = 0;
+            uint32_t ph = 0;
+            int li = 0;
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x, ++li) {
+                if constexpr (KIND == TC_W4A8) {
+                    // one TMEM buffer per group, alternating across all groups of all tiles
+                    for (int kb = 0; kb < KB; ++kb) {
+                        const int gi = li * KB + kb;
+                        const int buf = gi & 1;
+                        if (!mbar_wait(&tempty[buf], ((gi >> 1) & 1) ^ 1)) { ok = false; break; }
+                        if (!mbar_wait(&bready[s], ph)) { ok = false; break; }
+                        tc_fence_after();
+                        const uint32_t a0 = smem_u32(smem + s * C::STAGE);
+                        const uint32_t b0 = a0 + C::A_BYTES;
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_i8_ss(tmem + buf * 128, smem_desc(a0 + 32 * kk, 16, 1024, 2),
+                                      smem_desc(b0 + 32 * kk, 16, 1024, 2), idesc_s8(128, false), kk > 0 ? 1u : 0u);
+                        mma_commit(&empty[s]);
+                        mma_commit(&tfull[buf]);
+                        if (++s == C::ST) { s = 0; ph ^= 1; }
+                    }
+                } else {
+                    const int buf = li & 1;
+                    if (!mbar_wait(&tempty[buf], ((li >> 1) & 1) ^ 1)) break;
+                    tc_fence_after();
+                    for (int kb = 0; kb < KB; ++kb) {
+                        if constexpr (KIND == TC_W8A8) {
+                            if (!mbar_wait(&full[s], ph)) { ok = false; break; }
+                        } else {
+                            if (!mbar_wait(&bready[s], ph)) { ok = false; break; }
+                        }
+                        tc_fence_after();
+                        const uint32_t a0 = smem_u32(smem + s * C::STAGE);
+                        const uint32_t b0 = a0 + C::A_BYTES;
+                        if constexpr (KIND == TC_W8A8) {
+#pragma unroll
+                            for (int kk = 0; kk < 4; ++kk)
+                                mma_i8_ss(tmem + buf * 256, smem_desc(a0 + 32 * kk, 16, 1024, 2),
+                                          smem_desc(b0 + 4096 * kk, 16384, 1024, 2), idesc_s8(256, true),
+                                          (kb | kk) ? 1u : 0u);
+                        } else {
+#pragma unroll
+                            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                                for (int kk = 0; kk < 4; ++kk)
+                                    mma_f16_ss(tmem + buf * 256 + h * 128, smem_desc(a0 + h * 16384 + 32 * kk, 16, 1024, 2),
+                                               smem_desc(b0 + 32 * kk, 16, 1024, 2), idesc_bf16(128), (kb | kk) ? 1u : 0u);
+                        }
+                        mma_commit(&empty[s]);
+                        if (++s == C::ST) { s = 0; ph ^= 1; }
+                    }
+                    if (ok) mma_commit(&tfull[buf]);
+                }
+            }
+        }
+    } else if (warp < 6) {
+        // ------------------------------ epilogue ------------------------------
+        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        int li = 0;
+        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++li) {
+            const int m0 = (tile % p.m_tiles) * C::BM, n0 = (tile / p.m_tiles) * C::BN;
+            if constexpr (KIND == TC_W4A8) {
+                float accf[128];
+#pragma unroll
+                for (int i = 0; i < 128; ++i) accf[i] = 0.0f;
+                const int m = m0 + 32 * q + lane;
+                bool ok = true;
+                for (int kb = 0; kb < KB && ok; ++kb) {
+                    const int gi = li * KB + kb;
+                    const int buf = gi & 1;
+                    if (!mbar_wait(&tfull[buf], (gi >> 1) & 1)) { ok = false; break; }
+                    tc_fence_after();
+                    const float* sgrow = p.sg + (int64_t)kb * p.N + n0;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + buf * 128 + 32 * c, r);
+                        tmem_ld_wait();
+                        if (p.dbg && m < p.M) {
+                            int32_t* drow = p.dbg + ((int64_t)m * KB + kb) * p.N + n0 + 32 * c;
+#pragma unroll
+                            for (int i = 0; i < 32; i += 4)
+                                if (n0 + 32 * c + i < p.N)
+                                    *reinterpret_cast<int4*>(drow + i) = make_int4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+                        }
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4) {
+                            const float4 sv = (n0 + 32 * c + i < p.N) ? __ldg(reinterpret_cast<const float4*>(sgrow + 32 * c + i))
+                                                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+                            accf[32 * c + i + 0] = fmaf((float)(int)r[i + 0], sv.x, accf[32 * c + i + 0]);
+                            accf[32 * c + i + 1] = fmaf((float)(int)r[i + 1], sv.y, accf[32 * c + i + 1]);
+                            accf[32 * c + i + 2] = fmaf((float)(int)r[i + 2], sv.z, accf[32 * c + i + 2]);
+                            accf[32 * c + i + 3] = fmaf((float)(int)r[i + 3], sv.w, accf[32 * c + i + 3]);
+                        }
+                    }
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&tempty[buf]);
+                }
+                if (!ok) break;
+                if (m < p.M) {
+                    const float tm = __ldg(p.t + m);
+                    uint16_t* yrow = p.Y + (int64_t)m * p.N + n0;
+#pragma unroll
+                    for (int i = 0; i < 128; i += 8) {
+                        if (n0 + i < p.N) {
+                            uint4 v;
+                            v.x = pack_bf16x2_rn(__fmul_rn(tm, accf[i + 0]), __fmul_rn(tm, accf[i + 1]));
+                            v.y = pack_bf16x2_rn(__fmul_rn(tm, accf[i + 2]), __fmul_rn(tm, accf[i + 3]));
+                            v.z = pack_bf16x2_rn(__fmul_rn(tm, accf[i + 4]), __fmul_rn(tm, accf[i + 5]));
+                            v.w = pack_bf16x2_rn(__fmul_rn(tm, accf[i + 6]), __fmul_rn(tm, accf[i + 7]));
+                            *reinterpret_cast<uint4*>(yrow + i) = v;
+                        }
+                    }
+                }
+            } else {
+                const int buf = li & 1;
+                if (!mbar_wait(&tfull[buf], (li >> 1) & 1)) break;
+                tc_fence_after();
+#pragma unroll 1
+                for (int h = 0; h < C::MH; ++h) {
+                    const int m = m0 + h * 128 + 32 * q + lane;
+                    const float tm = (KIND == TC_W8A8 && m < p.M) ? __ldg(p.t + m) : 0.0f;
+#pragma unroll 1
+                    for (int c = 0; c < (KIND == TC_W8A8 ? 8 : 4); ++c) {
+                        uint32_t r[32];
+                        const uint32_t col = (KIND == TC_W8A8 ? buf * 256 : buf * 256 + h * 128) + 32 * c;
+                        tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + col, r);
+                        tmem_ld_wait();
+                        const int nb = n0 + 32 * c;
+                        if (m < p.M) {
+                            uint16_t* yrow = p.Y + (int64_t)m * p.N + nb;
+#pragma unroll
+                            for (int i = 0; i < 32; i += 8) {
+                                if (nb + i >= p.N) continue;
+                                float f[8];
+                                if constexpr (KIND == TC_W8A8) {
+                                    const float4 s0 = __ldg(reinterpret_cast<const float4*>(p.sw + nb + i));
+                                    const float4 s1 = __ldg(reinterpret_cast<const float4*>(p.sw + nb + i + 4));
+                                    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e)
+                                        f[e] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[i + e]), tm), sv[e]);
+                                    if (p.dbg) {
+                                        int32_t* d = p.dbg + (int64_t)m * p.N + nb + i;
+                                        *reinterpret_cast<int4*>(d) = make_int4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+                                        *reinterpret_cast<int4*>(d + 4) = make_int4(r[i + 4], r[i + 5], r[i + 6], r[i + 7]);
+                                    }
+                                } else {
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[i + e]);
+                                }
+                                uint4 v;
+                                v.x = pack_bf16x2_rn(f[0], f[1]);
+                                v.y = pack_bf16x2_rn(f[2], f[3]);
+                                v.z = pack_bf16x2_rn(f[4], f[5]);
+                                v.w = pack_bf16x2_rn(f[6], f[7]);
+                                *reinterpret_cast<uint4*>(yrow + i) = v;
+                            }
+                        }
+                    }
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&tempty[buf]);
+            }
+        }
+    } else {
+        // ------------------------------ dequant warps (W4A16, W4A8) ------------------------------
+        if constexpr (KIND != TC_W8A8) {
+            const int dt = threadIdx.x - 192;  // 0..127: the B tile row (column n) this thread fills
+            int s = 0;
+            uint32_t ph = 0;
+            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+                const int n0 = (tile / p.m_tiles) * C::BN;
+                const int n = n0 + dt;
+                for (int kb = 0; kb < KB; ++kb) {
+                    // per-column scale and zero of this k-block's group, fetched before the wait
+                    float sv = 0.0f, zv = 0.0f;
+                    if constexpr (KIND == TC_W4A16) {
+                        if (n < p.N) {
+                            sv = __half2float(__ushort_as_half(__ldg(p.scales + (int64_t)(kb >> 1) * p.N + n)));
+                            zv = (float)__ldg(p.zeros + (int64_t)(kb >> 1) * p.N + n);
+                        }
+                    }
+                    if (!mbar_wait(&full[s], ph)) goto dequant_done;
+                    uint8_t* st = smem + s * C::STAGE;
+                    const uint32_t* raw = reinterpret_cast<const uint32_t*>(st + C::A_BYTES + C::B_BYTES);
+                    uint8_t* brow = st + C::A_BYTES + dt * 128;  // row dt of the K-major B tile
+                    if constexpr (KIND == TC_W4A16) {
+                        // k-block of 64 = 8 words of column n, all in group kb / 2
+                        const uint32_t s2 = pack_bf16x2_rn(sv, sv);
+                        const uint32_t z2 = pack_bf16x2_rn(128.0f + zv, 128.0f + zv);
+#pragma unroll
+                        for (int w = 0; w < 8; ++w) {
+                            const uint32_t word = raw[w * 128 + dt];
+                            uint32_t R[4];
+#pragma unroll
+                            for (int r = 0; r < 4; ++r)
+                                R[r] = bf16x2_mul(bf16x2_sub(lop3_and_or(word >> (4 * r), 0x000F000Fu, 0x43004300u), z2), s2);
+                            uint4 v;  // natural k order: (0,1) (2,3) (4,5) (6,7)
+                            v.x = prmt(R[0], R[1], 0x5410);
+                            v.y = prmt(R[2], R[3], 0x5410);
+                            v.z = prmt(R[0], R[1], 0x7632);
+                            v.w = prmt(R[2], R[3], 0x7632);
+                            *reinterpret_cast<uint4*>(brow + ((w ^ (dt & 7)) << 4)) = v;
+                        }
+                    } else {
+                        // one group of 128 k = 16 words; two words per 16-byte chunk
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            uint32_t o[4];
+#pragma unroll
+                            for (int hw = 0; hw < 2; ++hw) {
+                                const uint32_t word = raw[(2 * c + hw) * 128 + dt];
+                                uint32_t ev, od;
+                                asm("lop3.b32 %0, %1, 0x0F0F0F0F, 0x08080808, 0x6A;" : "=r"(ev) : "r"(word));
+                                asm("lop3.b32 %0, %1, 0x0F0F0F0F, 0x08080808, 0x6A;" : "=r"(od) : "r"(word >> 4));
+                                ev = (ev + 0x78787878u) ^ 0x80808080u;
+                                od = (od + 0x78787878u) ^ 0x80808080u;
+                                o[2 * hw] = prmt(ev, od, 0x5140);
+                                o[2 * hw + 1] = prmt(ev, od, 0x7362);
+                            }
+                            *reinterpret_cast<uint4*>(brow + ((c ^ (dt & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                        }
+                    }
+                    fence_proxy_async_smem();  // generic-proxy stores -> visible to tcgen05.mma
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&bready[s]);
+                    if (++s == C::ST) { s = 0; ph ^= 1; }
+                }
+            }
+        }
+    dequant_done:;
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, C::TMEM_COLS);
+    }
+}
 
 // Self-test of the bounded wait: one warp waits on an mbarrier that nothing arrives
 // at.  mbar_wait gives up after the configured limit and records QG_ERR_TIMEOUT.

@@ -302,3 +302,55 @@ def test_nonfinite_weights_reported():
 @pytest.mark.parametrize("K,N", synth.CONFIGS["w4a16_prefill"]["KN"])
 def test_gemm_w4a16_prefill_sampled(K, N):
     _w4a16_case(K, N, "w4a16_prefill", [4096, 8192], "bf16", rows=lambda M: sample_rows(M, extra=3))
+
+
+# ---------------------------------------------------------------------------
+# tensor-memory tile kernels (M >= 128) on ragged shapes: partial M and N tiles
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("M,K,N", [(128, 256, 208), (130, 384, 144), (257, 256, 272), (300, 512, 400)])
+def test_tile_w8a8_ragged(M, K, N):
+    rng = np.random.default_rng(M + N)
+    Xq = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    Wq = rng.integers(-127, 128, (K, N)).astype(np.int8)
+    t = rng.uniform(0.01, 1.0, M).astype(np.float32)
+    sw = rng.uniform(0.001, 0.01, N).astype(np.float32)
+    q = qlib()
+    Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    acc = torch.full((M, N), -1, dtype=torch.int32, device="cuda")
+    q.qg_gemm_w8a8(cuda(Xq), cuda(t), cuda(Wq), cuda(sw), Y, acc)
+    _status_ok()
+    acc_o, y_o, yref, b = oracle.gemm_w8a8(Xq, t, Wq, sw)
+    np.testing.assert_array_equal(acc.cpu().numpy(), acc_o)
+    np.testing.assert_array_equal(u16(Y), y_o)
+
+
+@pytest.mark.parametrize("M,K,N", [(128, 256, 208), (130, 384, 144), (257, 256, 272), (300, 512, 400)])
+def test_tile_w4a8_ragged(M, K, N):
+    rng = np.random.default_rng(M * N)
+    Xq = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    codes = rng.integers(-7, 8, (K, N)).astype(np.int8)
+    sg = rng.uniform(0.001, 0.01, (K // 128, N)).astype(np.float32)
+    t = rng.uniform(0.01, 1.0, M).astype(np.float32)
+    p_o = oracle.pack_nibbles(codes)
+    q = qlib()
+    Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    part = torch.full((M, K // 128, N), -1, dtype=torch.int32, device="cuda")
+    q.qg_gemm_w4a8(cuda(Xq), cuda(t), cuda(p_o.view(np.int32)), cuda(sg), Y, part)
+    _status_ok()
+    part_o, yref, b = oracle.gemm_w4a8(Xq, t, p_o, sg)
+    np.testing.assert_array_equal(part.cpu().numpy(), part_o)
+    assert_tol(bf16_to_f32(u16(Y)), yref, b)
+
+
+@pytest.mark.parametrize("M,K,N", [(128, 256, 208), (130, 384, 144), (257, 256, 272), (513, 512, 400)])
+def test_tile_w4a16_ragged(M, K, N):
+    W = synth.weights(K, N, 0.02, 0.01, 8.0, seed=M)
+    codes, scales, zeros, packed = quant_w4_asym(W)
+    c_o, s_o, z_o, _ = oracle.quantize_w4_asym(W)
+    X, Xb = synth.activations(M, K, "bf16", seed=N)
+    q = qlib()
+    Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    q.qg_gemm_w4a16(x_device(Xb, torch.bfloat16), packed, scales, zeros, Y)
+    _status_ok()
+    yref, b = oracle.gemm_w4a16_ref(X, oracle.pack_nibbles(c_o), s_o, z_o)
+    assert_tol(bf16_to_f32(u16(Y)), yref, b)
