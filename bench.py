@@ -277,9 +277,10 @@ def e2e_decode(sweep, steps, warmup, world):
     return ms, h2d, d2h
 
 
-def cpu_baseline_decode(seconds_hint=15.0, col_frac=16):
+def cpu_baseline_decode(min_seconds=10.0, col_frac=1, max_reps=20):
     """The oracle, as it stands, on a bounded sample of the sweep: every (K, N, M)
-    call restricted to the first N/col_frac output columns."""
+    call restricted to the first N/col_frac output columns, the whole set repeated
+    until at least `min_seconds` of CPU time have been spent (at most `max_reps`)."""
     import oracle
     cfg = synth.CONFIGS["w4a16_decode"]
     prepared = []
@@ -293,26 +294,28 @@ def cpu_baseline_decode(seconds_hint=15.0, col_frac=16):
             prepared.append((K, Ns, M, X, packed, scales, zeros))
     t0 = time.perf_counter()
     by = 0
-    for K, Ns, M, X, packed, scales, zeros in prepared:
-        oracle.gemm_w4a16_ref(X, packed, scales, zeros)
-        by += w4_bytes(K, Ns) + 2 * M * (K + Ns)
+    reps = 0
+    while reps < max_reps and (reps == 0 or time.perf_counter() - t0 < min_seconds):
+        for K, Ns, M, X, packed, scales, zeros in prepared:
+            oracle.gemm_w4a16_ref(X, packed, scales, zeros)
+            by += w4_bytes(K, Ns) + 2 * M * (K + Ns)
+        reps += 1
     dt = time.perf_counter() - t0
-    cores = len(os.sched_getaffinity(0))
+    cores = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
     return dict(value=by / dt / 1e9, unit="GB/s", cores=cores, kind="oracle",
-                sample=f"all 16 decode-sweep calls on the first 1/{col_frac} of the output columns "
-                       f"({by / 1e6:.1f} MB algorithmic), fp64 reference GEMM, {dt:.2f} s"), dt
+                sample=f"{reps} pass(es) over all 16 decode-sweep calls on 1/{col_frac} of the output columns "
+                       f"({by / 1e6:.1f} MB algorithmic), fp64 reference GEMM with OpenMP, {dt:.2f} s"), dt
 
 
 def run_reference(args, world, rank):
     """--impl reference: the CPU oracle timed on a bounded sample of the workload."""
     if rank != 0:
         return
-    col_frac = 64
-    _, dt = cpu_baseline_decode(col_frac=col_frac)  # warm-up + size estimate
+    col_frac = 8
     times = []
     by = None
     for i in range(args.warmup + args.steps):
-        cb, dt = cpu_baseline_decode(col_frac=col_frac)
+        cb, dt = cpu_baseline_decode(min_seconds=0.0, col_frac=col_frac, max_reps=1)
         if i >= args.warmup:
             times.append(dt)
             by = cb["value"] * dt * 1e9
@@ -321,11 +324,164 @@ def run_reference(args, world, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / len(times) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "w4a16_decode sample: 16 calls on 1/64 of the columns"},
+            "config": {"workload": "w4a16_decode sample: 16 calls on 1/8 of the columns"},
             "cpu_baseline": {"value": value, "unit": "GB/s", "kind": "oracle", "cores": cb["cores"],
                              "sample": cb["sample"]},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------------------
+# the other workloads: W8A8 SmoothQuant, W4A16 prefill, W4A8, W4A16 tiny
+# ---------------------------------------------------------------------------
+def measure_int8_peak():
+    """Dense int8 tensor throughput of this GPU (torch._int_mm, cuBLASLt), 8192^3, best of 10.
+    Used only as the roofline denominator of the int8 products."""
+    a = torch.randint(-127, 127, (8192, 8192), dtype=torch.int8, device="cuda")
+    b = torch.randint(-127, 127, (8192, 8192), dtype=torch.int8, device="cuda")
+    for _ in range(3):
+        torch._int_mm(a, b)
+    torch.cuda.synchronize()
+    best = 1e30
+    for _ in range(10):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        torch._int_mm(a, b)
+        e1.record()
+        torch.cuda.synchronize()
+        best = min(best, e0.elapsed_time(e1))
+    return 2 * 8192 ** 3 / (best * 1e-3) / 1e12
+
+
+def time_calls(fn, reps, rotations=1):
+    """Device time per call: `reps` calls captured in one graph (rotation index passed in)."""
+    def body(i):
+        for r in range(reps):
+            fn((i * reps + r) % rotations)
+    gs = capture_graphs(body, 1)
+    return time_graphs(gs, 5, 2, 1) / 5 / reps
+
+
+def gpu_quant_w4(q, W, s=None, sym=False):
+    K, N = W.shape
+    codes = torch.empty(K, N, dtype=torch.uint8, device="cuda")
+    if sym:
+        scales = torch.empty(K // 128, N, dtype=torch.float32, device="cuda")
+        q.qg_quantize_w4_group(W, s, 128, True, codes, scales, None)
+        zeros = None
+    else:
+        scales = torch.empty(K // 128, N, dtype=torch.int16, device="cuda")
+        zeros = torch.empty(K // 128, N, dtype=torch.uint8, device="cuda")
+        q.qg_quantize_w4_group(W, s, 128, False, codes, scales, zeros)
+    packed = torch.empty(K // 8, N, dtype=torch.int32, device="cuda")
+    q.qg_pack_nibbles(codes, packed)
+    return packed, scales, zeros
+
+
+def x_bf16(name, M, K):
+    _, xb = synth.workload_activations(name, M, K)
+    return torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def bench_configs(q, pk, int8_peak):
+    out = {}
+    L2 = l2_bytes()
+    bf16_peak = pk["bf16_tflops"]
+    # --- W4A16 tiny (fp16 X) -------------------------------------------------
+    K, N = 1024, 1024
+    W = torch.from_numpy(synth.workload_weights("w4a16_tiny", K, N)).cuda()
+    pw, sc, z = gpu_quant_w4(q, W)
+    _, xb = synth.workload_activations("w4a16_tiny", 1, K)
+    X = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.float16)
+    Y = torch.empty(1, N, dtype=torch.float16, device="cuda")
+    ms = time_calls(lambda i: q.qg_gemm_w4a16(X, pw, sc, z, Y), 64)
+    by = w4_bytes(K, N) + 2 * (K + N)
+    out["w4a16_tiny"] = {"M=1": {"us": ms * 1e3, "gbs": by / (ms * 1e-3) / 1e9, "note": "parity-size case, L2-resident"}}
+    # --- W8A8 SmoothQuant: act quant + GEMM ---------------------------------
+    cfg = synth.CONFIGS["w8a8"]
+    K, N = cfg["KN"][0]
+    W = torch.from_numpy(synth.workload_weights("w8a8", K, N)).cuda()
+    _, xcb = synth.calibration(K, cfg)
+    Xc = torch.from_numpy(xcb.view(np.int16)).cuda().view(torch.bfloat16)
+    s = torch.empty(K, dtype=torch.float32, device="cuda")
+    inv = torch.empty_like(s)
+    q.qg_smooth_scales(Xc, W, 0.5, s, inv)
+    Wq = torch.empty(K, N, dtype=torch.int8, device="cuda")
+    sw = torch.empty(N, dtype=torch.float32, device="cuda")
+    q.qg_quantize_w8_channel(W, s, Wq, sw)
+    rot = max(1, math.ceil(2 * L2 / (K * N)))
+    wqs = [Wq] + [Wq.clone() for _ in range(rot - 1)]
+    res = {}
+    for M in cfg["M"]:
+        X = x_bf16("w8a8", M, K)
+        Xq = torch.empty(M, K, dtype=torch.int8, device="cuda")
+        t = torch.empty(M, dtype=torch.float32, device="cuda")
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        ms_a = time_calls(lambda i: q.qg_smooth_quant_act_i8(X, inv, Xq, t), 32)
+        ms_g = time_calls(lambda i: q.qg_gemm_w8a8(Xq, t, wqs[i], sw, Y), 32, rot)
+        ops = 2 * M * K * N
+        by_g = K * N + 4 * N + M * K + 4 * M + 2 * M * N
+        by_a = 3 * M * K + 4 * K + 4 * M
+        t_roof = max(by_g / (pk["hbm_gbs"] * 1e9), ops / (int8_peak * 1e12))
+        res[f"M={M}"] = {"act_quant_us": ms_a * 1e3, "act_quant_gbs": by_a / (ms_a * 1e-3) / 1e9,
+                         "gemm_us": ms_g * 1e3, "tops": ops / (ms_g * 1e-3) / 1e12, "gbs": by_g / (ms_g * 1e-3) / 1e9,
+                         "bound": "hbm" if by_g / (pk["hbm_gbs"] * 1e9) > ops / (int8_peak * 1e12) else "int8 tensor",
+                         "roofline_frac": t_roof / (ms_g * 1e-3)}
+    out["w8a8"] = res
+    del W, Wq, wqs
+    # --- W4A8: act quant + GEMM ------------------------------------------------
+    cfg = synth.CONFIGS["w4a8"]
+    K, N = cfg["KN"][0]
+    W = torch.from_numpy(synth.workload_weights("w4a8", K, N)).cuda()
+    _, xcb = synth.calibration(K, cfg)
+    Xc = torch.from_numpy(xcb.view(np.int16)).cuda().view(torch.bfloat16)
+    s = torch.empty(K, dtype=torch.float32, device="cuda")
+    inv = torch.empty_like(s)
+    q.qg_smooth_scales(Xc, W, 0.5, s, inv)
+    pw, sg, _ = gpu_quant_w4(q, W, s, sym=True)
+    del W
+    wb = K * N // 2 + 4 * (K // 128) * N
+    rot = max(1, math.ceil(2 * L2 / wb))
+    pws = [(pw, sg)] + [(pw.clone(), sg.clone()) for _ in range(rot - 1)]
+    res = {}
+    for M in cfg["M"]:
+        X = x_bf16("w4a8", M, K)
+        Xq = torch.empty(M, K, dtype=torch.int8, device="cuda")
+        t = torch.empty(M, dtype=torch.float32, device="cuda")
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        q.qg_smooth_quant_act_i8(X, inv, Xq, t)
+        ms_g = time_calls(lambda i: q.qg_gemm_w4a8(Xq, t, pws[i][0], pws[i][1], Y), 32, rot)
+        ops = 2 * M * K * N
+        by_g = wb + M * K + 4 * M + 2 * M * N
+        fma_rescale = M * N * (K // 128)
+        t_hbm, t_tc = by_g / (pk["hbm_gbs"] * 1e9), ops / (int8_peak * 1e12)
+        res[f"M={M}"] = {"gemm_us": ms_g * 1e3, "tops": ops / (ms_g * 1e-3) / 1e12, "gbs": by_g / (ms_g * 1e-3) / 1e9,
+                         "bound": "hbm" if t_hbm > t_tc else "int8 tensor + per-group fp32 rescale",
+                         "rescale_fma": fma_rescale, "roofline_frac": max(t_hbm, t_tc) / (ms_g * 1e-3)}
+    out["w4a8"] = res
+    del pws, pw, sg
+    # --- W4A16 prefill --------------------------------------------------------
+    cfg = synth.CONFIGS["w4a16_prefill"]
+    res = {}
+    for (K, N) in cfg["KN"]:
+        W = torch.from_numpy(synth.workload_weights("w4a16_prefill", K, N)).cuda()
+        pw, sc, z = gpu_quant_w4(q, W)
+        del W
+        torch.cuda.empty_cache()
+        for M in cfg["M"]:
+            X = x_bf16("w4a16_prefill", M, K)
+            Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+            ms = time_calls(lambda i: q.qg_gemm_w4a16(X, pw, sc, z, Y), 3)
+            fl = 2 * M * K * N
+            res[f"M={M} K={K} N={N}"] = {"ms": ms, "tflops": fl / (ms * 1e-3) / 1e12,
+                                         "frac_bf16_burst": fl / (ms * 1e-3) / 1e12 / pk["bf16_tflops"],
+                                         "frac_bf16_sustained": fl / (ms * 1e-3) / 1e12 / pk["bf16_tflops_sustained"]}
+            del X, Y
+        del pw, sc, z
+    out["w4a16_prefill"] = res
+    out["int8_peak_tops_measured"] = int8_peak
+    out["bf16_peak_tflops_measured"] = bf16_peak
+    return out
 
 
 def run_single(spec, reps, workspace="auto"):
@@ -370,6 +526,7 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--workload", default="w4a16_decode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--skip-configs", action="store_true", help="only the headline decode sweep")
     ap.add_argument("--single", default=None, help="K,N,M: time one decode call shape alone (profiling aid)")
     ap.add_argument("--reps", type=int, default=5)
     ap.add_argument("--no-workspace", action="store_true")
@@ -408,6 +565,9 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu, _ = cpu_baseline_decode()
+    configs = None
+    if rank == 0 and not args.skip_configs:
+        configs = bench_configs(q, pk, measure_int8_peak())
 
     if rank == 0:
         line = {
@@ -427,6 +587,7 @@ def main():
             "clocks": ck,
             "tflops": sweep.flops_per_step() / (ms_step * 1e-3) / 1e12,
             "per_call": [{k: (round(v, 3) if isinstance(v, float) else v) for k, v in c.items()} for c in calls],
+            "configs": configs,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
