@@ -34,7 +34,7 @@ class QgError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
         msg = f"{where}: {STATUS.get(status, status)}"
-        if status == QG_ERR_CUDA and _lib is not None:
+        if status in (QG_ERR_CUDA, QG_ERR_WORKSPACE, QG_ERR_UNSUPPORTED) and _lib is not None:
             msg += " (" + _lib.qg_last_error().decode() + ")"
         super().__init__(msg)
 
@@ -71,10 +71,14 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     return L
 
 
-_lib = load_library()
+_lib = None
 
 
 def lib() -> ctypes.CDLL:
+    """The loaded libqgemm.so (loaded on first use; raises ImportError if it was never built)."""
+    global _lib
+    if _lib is None:
+        _lib = load_library()
     return _lib
 
 
@@ -101,26 +105,26 @@ def _check(st: int, where: str):
 
 def qg_quantize_w4_group(W, s_smooth, group, symmetric, codes, scales, zeros, stream=None):
     K, N = W.shape
-    _check(_lib.qg_quantize_w4_group(_ptr(W), _ptr(s_smooth), K, N, group, int(bool(symmetric)), _ptr(codes),
+    _check(lib().qg_quantize_w4_group(_ptr(W), _ptr(s_smooth), K, N, group, int(bool(symmetric)), _ptr(codes),
                                      _ptr(scales), _ptr(zeros), _stream(stream)), "qg_quantize_w4_group")
 
 
 def qg_pack_nibbles(codes, packed, stream=None):
     K, N = codes.shape
-    _check(_lib.qg_pack_nibbles(_ptr(codes), K, N, _ptr(packed), _stream(stream)), "qg_pack_nibbles")
+    _check(lib().qg_pack_nibbles(_ptr(codes), K, N, _ptr(packed), _stream(stream)), "qg_pack_nibbles")
 
 
 _WS = {}
 
 
 def qg_workspace_size(op: int, M: int, K: int, N: int) -> int:
-    return _lib.qg_workspace_size(op, M, K, N)
+    return lib().qg_workspace_size(op, M, K, N)
 
 
 def default_workspace(op, M, K, N, device):
     """A zero-filled workspace for (op, M, K, N), cached per device and grown on demand.
     Calls that may run concurrently (different streams) need workspaces of their own."""
-    need = _lib.qg_workspace_size(op, M, K, N)
+    need = lib().qg_workspace_size(op, M, K, N)
     if need == 0:
         return None
     key = torch.device(device).index if torch.device(device).index is not None else torch.cuda.current_device()
@@ -145,50 +149,50 @@ def qg_gemm_w4a16(X, packed, scales, zeros, Y, group=128, workspace="auto", stre
     N = packed.shape[1]
     xdt = QG_BF16 if X.dtype == torch.bfloat16 else QG_F16 if X.dtype == torch.float16 else -1
     wp, wb = _ws(workspace, QG_OP_GEMM_W4A16, M, K, N, X.device)
-    _check(_lib.qg_gemm_w4a16(_ptr(X), xdt, M, K, N, _ptr(packed), _ptr(scales), _ptr(zeros), group, _ptr(Y), wp, wb,
+    _check(lib().qg_gemm_w4a16(_ptr(X), xdt, M, K, N, _ptr(packed), _ptr(scales), _ptr(zeros), group, _ptr(Y), wp, wb,
                               _stream(stream)), "qg_gemm_w4a16")
 
 
 def qg_smooth_quant_act_i8(X, inv_s, Xq, t, stream=None):
     M, K = X.shape
-    _check(_lib.qg_smooth_quant_act_i8(_ptr(X), M, K, _ptr(inv_s), _ptr(Xq), _ptr(t), _stream(stream)),
+    _check(lib().qg_smooth_quant_act_i8(_ptr(X), M, K, _ptr(inv_s), _ptr(Xq), _ptr(t), _stream(stream)),
            "qg_smooth_quant_act_i8")
 
 
 def qg_gemm_w8a8(Xq, t, Wq, sw, Y, acc_dbg=None, stream=None):
     M, K = Xq.shape
     N = Wq.shape[1]
-    _check(_lib.qg_gemm_w8a8(_ptr(Xq), _ptr(t), M, K, _ptr(Wq), _ptr(sw), N, _ptr(Y), _ptr(acc_dbg), None, 0,
+    _check(lib().qg_gemm_w8a8(_ptr(Xq), _ptr(t), M, K, _ptr(Wq), _ptr(sw), N, _ptr(Y), _ptr(acc_dbg), None, 0,
                              _stream(stream)), "qg_gemm_w8a8")
 
 
 def qg_gemm_w4a8(Xq, t, packed, sg, Y, part_dbg=None, group=128, stream=None):
     M, K = Xq.shape
     N = packed.shape[1]
-    _check(_lib.qg_gemm_w4a8(_ptr(Xq), _ptr(t), M, K, _ptr(packed), _ptr(sg), N, group, _ptr(Y), _ptr(part_dbg), None,
+    _check(lib().qg_gemm_w4a8(_ptr(Xq), _ptr(t), M, K, _ptr(packed), _ptr(sg), N, group, _ptr(Y), _ptr(part_dbg), None,
                              0, _stream(stream)), "qg_gemm_w4a8")
 
 
 def qg_smooth_scales(Xcal, W, alpha, s, inv_s, stream=None):
     Mc, K = Xcal.shape
     N = W.shape[1]
-    _check(_lib.qg_smooth_scales(_ptr(Xcal), Mc, _ptr(W), K, N, ctypes.c_float(alpha), _ptr(s), _ptr(inv_s),
+    _check(lib().qg_smooth_scales(_ptr(Xcal), Mc, _ptr(W), K, N, ctypes.c_float(alpha), _ptr(s), _ptr(inv_s),
                                  _stream(stream)), "qg_smooth_scales")
 
 
 def qg_quantize_w8_channel(W, s, Wq, sw, stream=None):
     K, N = W.shape
-    _check(_lib.qg_quantize_w8_channel(_ptr(W), _ptr(s), K, N, _ptr(Wq), _ptr(sw), _stream(stream)),
+    _check(lib().qg_quantize_w8_channel(_ptr(W), _ptr(s), K, N, _ptr(Wq), _ptr(sw), _stream(stream)),
            "qg_quantize_w8_channel")
 
 
 def qg_device_status(stream=None) -> int:
-    return _lib.qg_device_status(_stream(stream))
+    return lib().qg_device_status(_stream(stream))
 
 
 def qg_selftest_bounded_wait(limit_ns: int = 0, stream=None):
-    _check(_lib.qg_selftest_bounded_wait(limit_ns, _stream(stream)), "qg_selftest_bounded_wait")
+    _check(lib().qg_selftest_bounded_wait(limit_ns, _stream(stream)), "qg_selftest_bounded_wait")
 
 
 def qg_status_string(status: int) -> str:
-    return _lib.qg_status_string(status).decode()
+    return lib().qg_status_string(status).decode()
