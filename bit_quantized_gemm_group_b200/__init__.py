@@ -27,7 +27,7 @@ QG_OP_GEMM_W4A16, QG_OP_GEMM_W8A8, QG_OP_GEMM_W4A8 = 0, 1, 2
 
 EXPORTS = ["qg_quantize_w4_group", "qg_pack_nibbles", "qg_gemm_w4a16", "qg_smooth_quant_act_i8", "qg_gemm_w8a8",
            "qg_gemm_w4a8", "qg_smooth_scales", "qg_quantize_w8_channel", "qg_device_status", "qg_status_string",
-           "qg_last_error", "qg_selftest_bounded_wait", "qg_workspace_size"]
+           "qg_last_error", "qg_selftest_bounded_wait", "qg_workspace_size", "qg_gemm_w4a16_noalloc"]
 
 
 class QgError(RuntimeError):
@@ -44,6 +44,7 @@ _SIGS = {
     "qg_quantize_w4_group": [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P],
     "qg_pack_nibbles": [_P, _I, _I, _P, _P],
     "qg_gemm_w4a16": [_P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _P, _SZ, _P],
+    "qg_gemm_w4a16_noalloc": [_P, _I, _I, _I, _I, _P, _P, _P, _I, _P, _P],
     "qg_smooth_quant_act_i8": [_P, _I, _I, _P, _P, _P, _P],
     "qg_gemm_w8a8": [_P, _P, _I, _I, _P, _P, _I, _P, _P, _P, _SZ, _P],
     "qg_gemm_w4a8": [_P, _P, _I, _I, _P, _P, _I, _I, _P, _P, _P, _SZ, _P],
@@ -151,6 +152,15 @@ def qg_gemm_w4a16(X, packed, scales, zeros, Y, group=128, workspace="auto", stre
     wp, wb = _ws(workspace, QG_OP_GEMM_W4A16, M, K, N, X.device)
     _check(lib().qg_gemm_w4a16(_ptr(X), xdt, M, K, N, _ptr(packed), _ptr(scales), _ptr(zeros), group, _ptr(Y), wp, wb,
                               _stream(stream)), "qg_gemm_w4a16")
+
+
+def qg_gemm_w4a16_noalloc(X, packed, scales, zeros, Y, group=128, stream=None):
+    """W4A16 GEMM with no workspace and no allocation (scratch in a static device array)."""
+    M, K = X.shape
+    N = packed.shape[1]
+    xdt = QG_BF16 if X.dtype == torch.bfloat16 else QG_F16 if X.dtype == torch.float16 else -1
+    _check(lib().qg_gemm_w4a16_noalloc(_ptr(X), xdt, M, K, N, _ptr(packed), _ptr(scales), _ptr(zeros), group, _ptr(Y),
+                                      _stream(stream)), "qg_gemm_w4a16_noalloc")
 
 
 def qg_smooth_quant_act_i8(X, inv_s, Xq, t, stream=None):

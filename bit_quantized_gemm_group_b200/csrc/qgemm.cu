@@ -625,3 +625,68 @@ qg_status qg_selftest_bounded_wait(uint64_t limit_ns, qg_stream_t stream)
 }
 
 }  // extern "C"
+
+// ===========================================================================
+// Allocation-free W4A16 entry point
+//
+// Some callers cannot call cudaMalloc (or torch's allocator) at the point where they
+// run a GEMM: code being captured into a CUDA graph (allocation is not allowed
+// inside a capture), plugins and custom operators inside a host framework that owns
+// every device allocation and gives the operator no allocator, and latency-bound
+// paths where an allocation's implicit device synchronisation is unacceptable.
+// For them the decode kernel's scratch (arrival counters and partial tiles) lives
+// in one statically sized device array instead of a caller workspace.
+// ===========================================================================
+namespace {
+
+// 6 MiB per GPU that loads this library, held until the process exits.  The
+// largest decode launch (32 tokens, one CTA per SM, at most 160 CTAs) needs
+// 32 KiB of counters + 160 x 2 x 128 x 32 x 4 B of partial tiles = 5.3 MiB.
+constexpr size_t kNoAllocScratchBytes = size_t(6) << 20;
+static __device__ __align__(256) unsigned char qg_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of the array, per device.  In host code the array's name is only a
+// host-side stand-in, so the address must come from cudaGetSymbolAddress, called
+// with the device current.
+void* g_noalloc_addr[kMaxDevices] = {nullptr};
+
+qg_status noalloc_scratch(void** out)
+{
+    const int dev = current_device();
+    if (!g_noalloc_addr[dev]) {
+        void* ptr = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&ptr, qg_noalloc_scratch);
+        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(qg_noalloc_scratch)");
+        g_noalloc_addr[dev] = ptr;
+    }
+    *out = g_noalloc_addr[dev];
+    return QG_OK;
+}
+
+}  // namespace
+
+extern "C" qg_status qg_gemm_w4a16_noalloc(const void* X, qg_dtype xdt, int M, int K, int N,
+                                           const uint32_t* packed, const uint16_t* scales, const uint8_t* zeros,
+                                           int group, void* Y, qg_stream_t stream)
+{
+    const size_t need = qg_workspace_size(QG_OP_GEMM_W4A16, M, K, N);
+    if (need == 0)  // no scratch used for this shape (or invalid arguments): plain call
+        return qg_gemm_w4a16(X, xdt, M, K, N, packed, scales, zeros, group, Y, nullptr, 0, stream);
+    if (need > kNoAllocScratchBytes) {
+        snprintf(g_last_error, sizeof(g_last_error),
+                 "qg_gemm_w4a16_noalloc: this shape needs %zu bytes of scratch, the static buffer holds %zu", need,
+                 kNoAllocScratchBytes);
+        return QG_ERR_WORKSPACE;
+    }
+    if (xdt != QG_F16 && xdt != QG_BF16) return QG_ERR_DTYPE;
+    if (!X || !packed || !scales || !zeros || !Y) return QG_ERR_NULL;
+    if (group != 128) return QG_ERR_SHAPE;
+    if (misaligned(X) || misaligned(packed) || misaligned(scales) || misaligned(zeros) || misaligned(Y))
+        return QG_ERR_ALIGN;
+    void* ws = nullptr;
+    qg_status st = noalloc_scratch(&ws);
+    if (st != QG_OK) return st;
+    // the arrival counters must start at zero; the array keeps whatever the last call left
+    QG_CUDA(cudaMemsetAsync(ws, 0, (size_t)qg::kDecMaxSlabs * sizeof(int), reinterpret_cast<cudaStream_t>(stream)));
+    return qg_gemm_w4a16(X, xdt, M, K, N, packed, scales, zeros, group, Y, ws, kNoAllocScratchBytes, stream);
+}

@@ -123,6 +123,26 @@ qg_status qg_gemm_w4a16(const void* X, qg_dtype xdt, int M, int K, int N, const 
                         void* workspace, size_t ws_bytes, qg_stream_t stream);
 
 /* --------------------------------------------------------------------------
+ * W4A16 GEMM that allocates nothing and takes no workspace.  The pages have no
+ * counterpart to this call: it exists for callers that cannot allocate device
+ * memory where they run the GEMM -- code inside a CUDA graph capture, operators
+ * inside a framework that owns all device memory, latency-bound paths that cannot
+ * afford an allocation's synchronisation.
+ *
+ * Same arguments and result as qg_gemm_w4a16 without (workspace, ws_bytes).  The
+ * decode kernel's scratch lives in one static device array of 6 MiB per GPU
+ * that loads the library, kept until the process exits; a shape whose scratch
+ * would exceed it is refused with QG_ERR_WORKSPACE (see qg_last_error()).
+ * The first call on each device looks the array's address up; make that first
+ * call before any stream capture.  Each call clears the array's counters on
+ * `stream` before its kernel.  All calls share the one array: calls that may
+ * overlap on the GPU (other streams, other threads) race and must not be issued.
+ * ------------------------------------------------------------------------ */
+qg_status qg_gemm_w4a16_noalloc(const void* X, qg_dtype xdt, int M, int K, int N, const uint32_t* packed,
+                                const uint16_t* scales, const uint8_t* zeros, int group, void* Y,
+                                qg_stream_t stream);
+
+/* --------------------------------------------------------------------------
  * Fused smoothing + per-token dynamic symmetric INT8 quantization of
  * activations.   [S] sec. 2.2; [Q] sec. 1.2 (s = max|x|/127), sec. 1.3 (per token)
  *
