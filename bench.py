@@ -484,38 +484,51 @@ def bench_configs(q, pk, int8_peak):
     return out
 
 
-def run_single(spec, reps, workspace="auto"):
-    """--single K,N,M: one decode-sweep call shape, `reps` timed launches (no graph),
-    for profiling a kernel in isolation.  Prints per-launch device time."""
+def run_single(spec, reps, workspace="auto", op="w4a16"):
+    """--single K,N,M [--op w4a16|w8a8|w4a8]: one GEMM call shape, `reps` timed launches
+    (no graph, L2 flushed before each), for profiling a kernel in isolation."""
     import bit_quantized_gemm_group_b200 as q
     K, N, M = (int(x) for x in spec.split(","))
-    W = torch.from_numpy(synth.workload_weights("w4a16_decode", K, N)).cuda()
-    codes = torch.empty(K, N, dtype=torch.uint8, device="cuda")
-    scales = torch.empty(K // 128, N, dtype=torch.int16, device="cuda")
-    zeros = torch.empty(K // 128, N, dtype=torch.uint8, device="cuda")
-    packed = torch.empty(K // 8, N, dtype=torch.int32, device="cuda")
-    q.qg_quantize_w4_group(W, None, 128, False, codes, scales, zeros)
-    q.qg_pack_nibbles(codes, packed)
-    _, xb = synth.activations(M, K, "bf16", seed=M)
-    X = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
-    Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+    cfg = {"w4a16": "w4a16_decode" if M <= 64 else "w4a16_prefill", "w8a8": "w8a8", "w4a8": "w4a8"}[op]
+    W = torch.from_numpy(synth.workload_weights(cfg, K, N)).cuda()
+    if op == "w4a16":
+        packed, scales, zeros = gpu_quant_w4(q, W)
+        X = x_bf16(cfg, M, K)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        call = lambda: q.qg_gemm_w4a16(X, packed, scales, zeros, Y, workspace=workspace)  # noqa: E731
+        by = w4_bytes(K, N) + 2 * M * (K + N)
+    else:
+        Xq = torch.randint(-127, 128, (M, K), dtype=torch.int8, device="cuda")
+        t = torch.rand(M, device="cuda") * 0.01
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        if op == "w8a8":
+            Wq = torch.empty(K, N, dtype=torch.int8, device="cuda")
+            sw = torch.empty(N, dtype=torch.float32, device="cuda")
+            q.qg_quantize_w8_channel(W, None, Wq, sw)
+            call = lambda: q.qg_gemm_w8a8(Xq, t, Wq, sw, Y)  # noqa: E731
+            by = K * N + 4 * N + M * K + 4 * M + 2 * M * N
+        else:
+            packed, sg, _ = gpu_quant_w4(q, W, None, sym=True)
+            call = lambda: q.qg_gemm_w4a8(Xq, t, packed, sg, Y)  # noqa: E731
+            by = K * N // 2 + 4 * (K // 128) * N + M * K + 4 * M + 2 * M * N
+    del W
     flush = torch.empty(2 * l2_bytes(), dtype=torch.uint8, device="cuda")
     for _ in range(3):
-        q.qg_gemm_w4a16(X, packed, scales, zeros, Y, workspace=workspace)
+        call()
     torch.cuda.synchronize()
     ts = []
     for _ in range(reps):
         flush.zero_()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record()
-        q.qg_gemm_w4a16(X, packed, scales, zeros, Y, workspace=workspace)
+        call()
         b.record()
         torch.cuda.synchronize()
         ts.append(a.elapsed_time(b) * 1e3)
     assert q.qg_device_status() == q.QG_OK
-    by = w4_bytes(K, N) + 2 * M * (K + N)
     med = float(np.median(ts))
-    print(json.dumps({"single": [K, N, M], "us_median": med, "us_min": min(ts), "gbs": by / (med * 1e-6) / 1e9}))
+    print(json.dumps({"single": [op, K, N, M], "us_median": med, "us_min": min(ts), "gbs": by / (med * 1e-6) / 1e9,
+                      "tflops": 2 * M * K * N / (med * 1e-6) / 1e12}))
 
 
 def main():
@@ -529,12 +542,16 @@ def main():
     ap.add_argument("--skip-configs", action="store_true", help="only the headline decode sweep")
     ap.add_argument("--single", default=None, help="K,N,M: time one decode call shape alone (profiling aid)")
     ap.add_argument("--reps", type=int, default=5)
+    ap.add_argument("--op", default="w4a16", choices=["w4a16", "w8a8", "w4a8"])
+    ap.add_argument("--profile", action="store_true",
+                    help="only the timed decode steps (no e2e / per-call / baseline / other workloads): "
+                         "the command profiled for the kernel launch list")
     ap.add_argument("--no-workspace", action="store_true")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.single:
         torch.cuda.set_device(0)
-        run_single(args.single, args.reps, None if args.no_workspace else "auto")
+        run_single(args.single, args.reps, None if args.no_workspace else "auto", args.op)
         return
 
     if args.impl == "reference":
@@ -558,6 +575,10 @@ def main():
     value = by * world * args.steps / (ms * 1e-3) / 1e9
     achieved = by / (ms_step * 1e-3) / 1e9
 
+    if args.profile:
+        if rank == 0:
+            print(json.dumps({"profile_run": True, "ms_per_step": ms_step, "gbs": achieved}), flush=True)
+        return
     e2e_ms, h2d, d2h = e2e_decode(sweep, args.steps, args.warmup, world)
     e2e_val = by * world * args.steps / (e2e_ms * 1e-3) / 1e9
     calls = per_call_times(sweep) if rank == 0 else []

@@ -16,9 +16,11 @@
 //                 weight words (W4A16, W4A8), into a ring of shared-memory stages.
 //   warp 1        TMEM allocator and MMA issuer (one elected lane issues tcgen05.mma
 //                 and tcgen05.commit; commits release ring stages and publish results).
-//   warps 2..5    epilogue: tcgen05.ld from TMEM, scale, convert, store.
-//   warps 6..9    (W4A16, W4A8) dequant: unpack nibbles from the raw stage and write the
-//                 K-major, 128-byte-swizzled B tile the MMA reads.
+//   warps 4..7    epilogue (warpgroup 1): tcgen05.ld from TMEM, scale, convert, store;
+//                 warp 4 + q reads TMEM lanes 32q..32q+31.
+//   warps 8..11   (W4A16, W4A8) dequant (warpgroup 2): unpack nibbles from the raw stage
+//                 and write the K-major, 128-byte-swizzled B tile the MMA reads.
+// Waits on mbarriers are done by one lane per warp, then __syncwarp.
 // Every wait is bounded (mbar_wait); a wait that gives up records QG_ERR_TIMEOUT and
 // its role stops issuing work.  No TMA multicast is used anywhere.
 #pragma once
@@ -65,7 +67,7 @@ struct TcCfg<TC_W8A8> {
     static constexpr int A_BYTES = 128 * 128, B_BYTES = 256 * 128, RAW_BYTES = 0;
     static constexpr int STAGE = A_BYTES + B_BYTES;
     static constexpr int ST = 4;
-    static constexpr int THREADS = 192;
+    static constexpr int THREADS = 256;
     static constexpr int TMEM_COLS = 512;  // two 256-column accumulators
     static constexpr int MH = 1;           // M=128 MMAs per tile
 };
@@ -78,21 +80,22 @@ struct TcCfg<TC_W4A16> {
     static constexpr int A_BYTES = 2 * 128 * 128, RAW_BYTES = 8 * 128 * 4, B_BYTES = 128 * 128;
     static constexpr int STAGE = A_BYTES + B_BYTES + 4096;  // raw area padded to 4 KB
     static constexpr int ST = 4;
-    static constexpr int THREADS = 320;
+    static constexpr int THREADS = 384;
     static constexpr int TMEM_COLS = 512;  // two tiles x (2 halves x 128 columns)
     static constexpr int MH = 2;
 };
 
 // W4A8: tile 128 x 128, k-block = one group of 128 int8; A 16 KB, raw 16 x 128 x 4 B = 8 KB,
-// B 128 x 128 int8 = 16 KB per stage; TMEM holds two group accumulators (ping-pong).
+// B 128 x 128 int8 = 16 KB per stage; TMEM holds two group accumulators (ping-pong) and
+// the tile's running fp32 sum (so the epilogue holds no accumulators in registers).
 template <>
 struct TcCfg<TC_W4A8> {
     static constexpr int BM = 128, BN = 128, BK = 128;
     static constexpr int A_BYTES = 128 * 128, RAW_BYTES = 16 * 128 * 4, B_BYTES = 128 * 128;
     static constexpr int STAGE = A_BYTES + B_BYTES + RAW_BYTES;
     static constexpr int ST = 4;
-    static constexpr int THREADS = 320;
-    static constexpr int TMEM_COLS = 256;
+    static constexpr int THREADS = 384;
+    static constexpr int TMEM_COLS = 512;  // group buffers at 0 and 128, running fp32 sum at 256
     static constexpr int MH = 1;
 };
 
@@ -100,7 +103,8 @@ template <int KIND>
 struct TcSmem {
     using C = TcCfg<KIND>;
     static constexpr int BAR_OFF = C::ST * C::STAGE;
-    static constexpr int TOTAL = BAR_OFF + 256 + 1024;  // barriers + tmem address + alignment slack
+    static constexpr int EPI_OFF = BAR_OFF + 256;         // W4A8: per-epilogue-warp group scales [4][2][128] fp32
+    static constexpr int TOTAL = EPI_OFF + (KIND == TC_W4A8 ? 4 * 2 * 128 * 4 : 0) + 1024;
 };
 
 struct TcParams {
@@ -140,6 +144,17 @@ QG_DEV_INLINE uint32_t bf16x2_mul(uint32_t a, uint32_t b)
     asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
     return r;
 }
+
+// one lane waits, the warp follows; returns the wait's result to every lane
+QG_DEV_INLINE bool warp_wait(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok = 1;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity) ? 1u : 0u;
+    return __shfl_sync(0xffffffffu, ok, 0) != 0;
+}
+
+// exact int32 -> fp32 for |v| < 2^22: add into the mantissa of 1.5 * 2^23, subtract it back
+QG_DEV_INLINE float i2f_small(uint32_t v) { return __uint_as_float(v + 0x4B400000u) - 12582912.0f; }
 
 template <int KIND>
 __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
@@ -273,28 +288,47 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
                 }
             }
         }
-    } else if (warp < 6) {
+    } else if (warp < 4) {
+        // warps 2, 3: no role
+    } else if (warp < 8) {
         // ------------------------------ epilogue ------------------------------
         const int q = warp & 3;  // TMEM lane quarter this warp may access
         int li = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++li) {
             const int m0 = (tile % p.m_tiles) * C::BM, n0 = (tile / p.m_tiles) * C::BN;
             if constexpr (KIND == TC_W4A8) {
-                float accf[128];
-#pragma unroll
-                for (int i = 0; i < 128; ++i) accf[i] = 0.0f;
+                // Per group: drain the int32 partial P from its TMEM buffer and fold it into
+                // the tile's running fp32 sum, also kept in TMEM (columns 256..383):
+                //     sum += P * s_g        (exact int32 -> fp32, one fma)
+                // The next group's scale row is staged in this warp's smem slot (one float4
+                // per lane) while the current one is used.  After the last group the sum is
+                // scaled by t[m] and stored as bf16.
+                float* sgs = reinterpret_cast<float*>(smem + S::EPI_OFF) + q * 256;
                 const int m = m0 + 32 * q + lane;
+                const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16);
+                auto stage_scales = [&](int g, int slot) {
+                    const int n = n0 + 4 * lane;
+                    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (g < KB && n < p.N) v = __ldg(reinterpret_cast<const float4*>(p.sg + (int64_t)g * p.N + n));
+                    *reinterpret_cast<float4*>(sgs + slot * 128 + 4 * lane) = v;
+                };
+                stage_scales(0, 0);
                 bool ok = true;
-                for (int kb = 0; kb < KB && ok; ++kb) {
+                for (int kb = 0; kb < KB; ++kb) {
                     const int gi = li * KB + kb;
                     const int buf = gi & 1;
-                    if (!mbar_wait(&tfull[buf], (gi >> 1) & 1)) { ok = false; break; }
+                    stage_scales(kb + 1, (kb + 1) & 1);  // next group's row, other slot
+                    if (!warp_wait(&tfull[buf], (gi >> 1) & 1)) { ok = false; break; }
                     tc_fence_after();
-                    const float* sgrow = p.sg + (int64_t)kb * p.N + n0;
-#pragma unroll
+                    __syncwarp();
+                    const float* sv = sgs + (kb & 1) * 128;
+                    const bool last = kb == KB - 1;
+                    const float tm = (last && m < p.M) ? __ldg(p.t + m) : 0.0f;
+#pragma unroll 1
                     for (int c = 0; c < 4; ++c) {
-                        uint32_t r[32];
-                        tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + buf * 128 + 32 * c, r);
+                        uint32_t r[32], a[32];
+                        tmem_ld_32x32b_x32(trow + buf * 128 + 32 * c, r);
+                        if (kb > 0) tmem_ld_32x32b_x32(trow + 256 + 32 * c, a);
                         tmem_ld_wait();
                         if (p.dbg && m < p.M) {
                             int32_t* drow = p.dbg + ((int64_t)m * KB + kb) * p.N + n0 + 32 * c;
@@ -305,37 +339,40 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
                         }
 #pragma unroll
                         for (int i = 0; i < 32; i += 4) {
-                            const float4 sv = (n0 + 32 * c + i < p.N) ? __ldg(reinterpret_cast<const float4*>(sgrow + 32 * c + i))
-                                                                       : make_float4(0.f, 0.f, 0.f, 0.f);
-                            accf[32 * c + i + 0] = fmaf((float)(int)r[i + 0], sv.x, accf[32 * c + i + 0]);
-                            accf[32 * c + i + 1] = fmaf((float)(int)r[i + 1], sv.y, accf[32 * c + i + 1]);
-                            accf[32 * c + i + 2] = fmaf((float)(int)r[i + 2], sv.z, accf[32 * c + i + 2]);
-                            accf[32 * c + i + 3] = fmaf((float)(int)r[i + 3], sv.w, accf[32 * c + i + 3]);
+                            const float4 s4 = *reinterpret_cast<const float4*>(sv + 32 * c + i);  // broadcast
+                            const float sc[4] = {s4.x, s4.y, s4.z, s4.w};
+#pragma unroll
+                            for (int e = 0; e < 4; ++e) {
+                                const float prev = kb > 0 ? __uint_as_float(a[i + e]) : 0.0f;
+                                a[i + e] = __float_as_uint(fmaf(i2f_small(r[i + e]), sc[e], prev));
+                            }
+                        }
+                        if (!last) {
+                            tmem_st_32x32b_x32(trow + 256 + 32 * c, a);
+                        } else if (m < p.M) {
+                            uint16_t* yrow = p.Y + (int64_t)m * p.N + n0 + 32 * c;
+#pragma unroll
+                            for (int i = 0; i < 32; i += 8) {
+                                if (n0 + 32 * c + i < p.N) {
+                                    uint4 v;
+                                    v.x = pack_bf16x2_rn(__fmul_rn(tm, __uint_as_float(a[i + 0])), __fmul_rn(tm, __uint_as_float(a[i + 1])));
+                                    v.y = pack_bf16x2_rn(__fmul_rn(tm, __uint_as_float(a[i + 2])), __fmul_rn(tm, __uint_as_float(a[i + 3])));
+                                    v.z = pack_bf16x2_rn(__fmul_rn(tm, __uint_as_float(a[i + 4])), __fmul_rn(tm, __uint_as_float(a[i + 5])));
+                                    v.w = pack_bf16x2_rn(__fmul_rn(tm, __uint_as_float(a[i + 6])), __fmul_rn(tm, __uint_as_float(a[i + 7])));
+                                    *reinterpret_cast<uint4*>(yrow + i) = v;
+                                }
+                            }
                         }
                     }
+                    tmem_st_wait();
                     tc_fence_before();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(&tempty[buf]);
                 }
                 if (!ok) break;
-                if (m < p.M) {
-                    const float tm = __ldg(p.t + m);
-                    uint16_t* yrow = p.Y + (int64_t)m * p.N + n0;
-#pragma unroll
-                    for (int i = 0; i < 128; i += 8) {
-                        if (n0 + i < p.N) {
-                            uint4 v;
-                            v.x = pack_bf16x2_rn(__fmul_rn(tm, accf[i + 0]), __fmul_rn(tm, accf[i + 1]));
-                            v.y = pack_bf16x2_rn(__fmul_rn(tm, accf[i + 2]), __fmul_rn(tm, accf[i + 3]));
-                            v.z = pack_bf16x2_rn(__fmul_rn(tm, accf[i + 4]), __fmul_rn(tm, accf[i + 5]));
-                            v.w = pack_bf16x2_rn(__fmul_rn(tm, accf[i + 6]), __fmul_rn(tm, accf[i + 7]));
-                            *reinterpret_cast<uint4*>(yrow + i) = v;
-                        }
-                    }
-                }
             } else {
                 const int buf = li & 1;
-                if (!mbar_wait(&tfull[buf], (li >> 1) & 1)) break;
+                if (!warp_wait(&tfull[buf], (li >> 1) & 1)) break;
                 tc_fence_after();
 #pragma unroll 1
                 for (int h = 0; h < C::MH; ++h) {
@@ -388,22 +425,41 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
     } else {
         // ------------------------------ dequant warps (W4A16, W4A8) ------------------------------
         if constexpr (KIND != TC_W8A8) {
-            const int dt = threadIdx.x - 192;  // 0..127: the B tile row (column n) this thread fills
+            const int dt = threadIdx.x - 256;  // 0..127: the B tile row (column n) this thread fills
             int s = 0;
             uint32_t ph = 0;
             for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
                 const int n0 = (tile / p.m_tiles) * C::BN;
                 const int n = n0 + dt;
-                for (int kb = 0; kb < KB; ++kb) {
-                    // per-column scale and zero of this k-block's group, fetched before the wait
-                    float sv = 0.0f, zv = 0.0f;
-                    if constexpr (KIND == TC_W4A16) {
-                        if (n < p.N) {
-                            sv = __half2float(__ushort_as_half(__ldg(p.scales + (int64_t)(kb >> 1) * p.N + n)));
-                            zv = (float)__ldg(p.zeros + (int64_t)(kb >> 1) * p.N + n);
+                // W4A16: per-column scale and zero, fetched one group ahead of their use
+                uint16_t s_cur = 0, s_nxt = 0;
+                uint8_t z_cur = 0, z_nxt = 0;
+                if constexpr (KIND == TC_W4A16) {
+                    if (n < p.N) {
+                        s_cur = __ldg(p.scales + n);
+                        z_cur = __ldg(p.zeros + n);
+                        if (KB > 2) {
+                            s_nxt = __ldg(p.scales + (int64_t)p.N + n);
+                            z_nxt = __ldg(p.zeros + (int64_t)p.N + n);
                         }
                     }
-                    if (!mbar_wait(&full[s], ph)) goto dequant_done;
+                }
+                for (int kb = 0; kb < KB; ++kb) {
+                    float sv = 0.0f, zv = 0.0f;
+                    if constexpr (KIND == TC_W4A16) {
+                        if (kb > 0 && (kb & 1) == 0) {  // a new group starts: rotate and prefetch the next
+                            s_cur = s_nxt;
+                            z_cur = z_nxt;
+                            const int gn = (kb >> 1) + 1;
+                            if (n < p.N && 2 * gn < KB) {
+                                s_nxt = __ldg(p.scales + (int64_t)gn * p.N + n);
+                                z_nxt = __ldg(p.zeros + (int64_t)gn * p.N + n);
+                            }
+                        }
+                        sv = __half2float(__ushort_as_half(s_cur));
+                        zv = (float)z_cur;
+                    }
+                    if (!warp_wait(&full[s], ph)) goto dequant_done;
                     uint8_t* st = smem + s * C::STAGE;
                     const uint32_t* raw = reinterpret_cast<const uint32_t*>(st + C::A_BYTES + C::B_BYTES);
                     uint8_t* brow = st + C::A_BYTES + dt * 128;  // row dt of the K-major B tile
