@@ -471,7 +471,7 @@ def bench_configs(q, pk, int8_peak):
         for M in cfg["M"]:
             X = x_bf16("w4a16_prefill", M, K)
             Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
-            ms = time_calls(lambda i: q.qg_gemm_w4a16(X, pw, sc, z, Y), 3)
+            ms = time_calls(lambda i: q.qg_gemm_w4a16(X, pw, sc, z, Y), 10)
             fl = 2 * M * K * N
             res[f"M={M} K={K} N={N}"] = {"ms": ms, "tflops": fl / (ms * 1e-3) / 1e12,
                                          "frac_bf16_burst": fl / (ms * 1e-3) / 1e12 / pk["bf16_tflops"],
@@ -588,7 +588,10 @@ def main():
         cpu, _ = cpu_baseline_decode()
     configs = None
     if rank == 0 and not args.skip_configs:
+        cs = ClockSampler(local)
+        cs.start()
         configs = bench_configs(q, pk, measure_int8_peak())
+        configs["clocks"] = cs.stop()
 
     if rank == 0:
         line = {

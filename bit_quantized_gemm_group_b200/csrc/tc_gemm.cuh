@@ -16,10 +16,11 @@
 //                 weight words (W4A16, W4A8), into a ring of shared-memory stages.
 //   warp 1        TMEM allocator and MMA issuer (one elected lane issues tcgen05.mma
 //                 and tcgen05.commit; commits release ring stages and publish results).
-//   warps 4..7    epilogue (warpgroup 1): tcgen05.ld from TMEM, scale, convert, store;
-//                 warp 4 + q reads TMEM lanes 32q..32q+31.
-//   warps 8..11   (W4A16, W4A8) dequant (warpgroup 2): unpack nibbles from the raw stage
-//                 and write the K-major, 128-byte-swizzled B tile the MMA reads.
+//   warps 4..     EPI epilogue warps: tcgen05.ld from TMEM, scale, convert, store; epilogue
+//                 warp e reads TMEM lanes 32(e%4)..+31 and the e/4-th share of the columns.
+//   then          DQ dequant warps (W4A16, W4A8): unpack nibbles from the raw stage and write
+//                 the K-major, 128-byte-swizzled B tile the MMA reads; dequant thread d fills
+//                 B row d%128 and the (d/128)-th share of the k-block's words.
 // Waits on mbarriers are done by one lane per warp, then __syncwarp.
 // Every wait is bounded (mbar_wait); a wait that gives up records QG_ERR_TIMEOUT and
 // its role stops issuing work.  No TMA multicast is used anywhere.
@@ -67,7 +68,8 @@ struct TcCfg<TC_W8A8> {
     static constexpr int A_BYTES = 128 * 128, B_BYTES = 256 * 128, RAW_BYTES = 0;
     static constexpr int STAGE = A_BYTES + B_BYTES;
     static constexpr int ST = 4;
-    static constexpr int THREADS = 256;
+    static constexpr int EPI = 8, DQ = 0;  // epilogue / dequant warps
+    static constexpr int THREADS = 32 * (4 + EPI + DQ);
     static constexpr int TMEM_COLS = 512;  // two 256-column accumulators
     static constexpr int MH = 1;           // M=128 MMAs per tile
 };
@@ -80,7 +82,8 @@ struct TcCfg<TC_W4A16> {
     static constexpr int A_BYTES = 2 * 128 * 128, RAW_BYTES = 8 * 128 * 4, B_BYTES = 128 * 128;
     static constexpr int STAGE = A_BYTES + B_BYTES + 4096;  // raw area padded to 4 KB
     static constexpr int ST = 4;
-    static constexpr int THREADS = 384;
+    static constexpr int EPI = 8, DQ = 8;
+    static constexpr int THREADS = 32 * (4 + EPI + DQ);
     static constexpr int TMEM_COLS = 512;  // two tiles x (2 halves x 128 columns)
     static constexpr int MH = 2;
 };
@@ -94,7 +97,8 @@ struct TcCfg<TC_W4A8> {
     static constexpr int A_BYTES = 128 * 128, RAW_BYTES = 16 * 128 * 4, B_BYTES = 128 * 128;
     static constexpr int STAGE = A_BYTES + B_BYTES + RAW_BYTES;
     static constexpr int ST = 4;
-    static constexpr int THREADS = 384;
+    static constexpr int EPI = 8, DQ = 4;
+    static constexpr int THREADS = 32 * (4 + EPI + DQ);
     static constexpr int TMEM_COLS = 512;  // group buffers at 0 and 128, running fp32 sum at 256
     static constexpr int MH = 1;
 };
@@ -104,7 +108,7 @@ struct TcSmem {
     using C = TcCfg<KIND>;
     static constexpr int BAR_OFF = C::ST * C::STAGE;
     static constexpr int EPI_OFF = BAR_OFF + 256;         // W4A8: per-epilogue-warp group scales [4][2][128] fp32
-    static constexpr int TOTAL = EPI_OFF + (KIND == TC_W4A8 ? 4 * 2 * 128 * 4 : 0) + 1024;
+    static constexpr int TOTAL = EPI_OFF + (KIND == TC_W4A8 ? C::EPI * 2 * 128 * 4 : 0) + 1024;
 };
 
 struct TcParams {
@@ -179,11 +183,11 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
         for (int i = 0; i < C::ST; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], 1);
-            mbar_init(&bready[i], 4);
+            mbar_init(&bready[i], C::DQ > 0 ? C::DQ : 1);
         }
         for (int i = 0; i < 2; ++i) {
             mbar_init(&tfull[i], 1);
-            mbar_init(&tempty[i], 4);
+            mbar_init(&tempty[i], C::EPI);
         }
         fence_mbar_init();
     }
@@ -290,9 +294,12 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
         }
     } else if (warp < 4) {
         // warps 2, 3: no role
-    } else if (warp < 8) {
+    } else if (warp < 4 + C::EPI) {
         // ------------------------------ epilogue ------------------------------
-        const int q = warp & 3;  // TMEM lane quarter this warp may access
+        const int e = warp - 4;
+        const int q = e & 3;  // TMEM lane quarter this warp may access
+        constexpr int CSPLIT = C::EPI / 4;               // warps sharing one lane quarter
+        const int cs = e >> 2;                           // this warp's share of the columns
         int li = 0;
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++li) {
             const int m0 = (tile % p.m_tiles) * C::BM, n0 = (tile / p.m_tiles) * C::BN;
@@ -303,14 +310,18 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
                 // The next group's scale row is staged in this warp's smem slot (one float4
                 // per lane) while the current one is used.  After the last group the sum is
                 // scaled by t[m] and stored as bf16.
-                float* sgs = reinterpret_cast<float*>(smem + S::EPI_OFF) + q * 256;
+                float* sgs = reinterpret_cast<float*>(smem + S::EPI_OFF) + e * 256;
+                constexpr int CW = C::BN / CSPLIT;           // columns per warp
+                const int cb = cs * CW;                      // first column of this warp
                 const int m = m0 + 32 * q + lane;
                 const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16);
                 auto stage_scales = [&](int g, int slot) {
-                    const int n = n0 + 4 * lane;
-                    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (g < KB && n < p.N) v = __ldg(reinterpret_cast<const float4*>(p.sg + (int64_t)g * p.N + n));
-                    *reinterpret_cast<float4*>(sgs + slot * 128 + 4 * lane) = v;
+                    if (4 * lane < CW) {
+                        const int n = n0 + cb + 4 * lane;
+                        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                        if (g < KB && n < p.N) v = __ldg(reinterpret_cast<const float4*>(p.sg + (int64_t)g * p.N + n));
+                        *reinterpret_cast<float4*>(sgs + slot * 128 + 4 * lane) = v;
+                    }
                 };
                 stage_scales(0, 0);
                 bool ok = true;
@@ -325,7 +336,8 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
                     const bool last = kb == KB - 1;
                     const float tm = (last && m < p.M) ? __ldg(p.t + m) : 0.0f;
 #pragma unroll 1
-                    for (int c = 0; c < 4; ++c) {
+                    for (int cc = 0; cc < CW / 32; ++cc) {
+                        const int c = cb / 32 + cc;  // chunk of 32 columns within the tile
                         uint32_t r[32], a[32];
                         tmem_ld_32x32b_x32(trow + buf * 128 + 32 * c, r);
                         if (kb > 0) tmem_ld_32x32b_x32(trow + 256 + 32 * c, a);
@@ -339,7 +351,7 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
                         }
 #pragma unroll
                         for (int i = 0; i < 32; i += 4) {
-                            const float4 s4 = *reinterpret_cast<const float4*>(sv + 32 * c + i);  // broadcast
+                            const float4 s4 = *reinterpret_cast<const float4*>(sv + 32 * cc + i);  // broadcast
                             const float sc[4] = {s4.x, s4.y, s4.z, s4.w};
 #pragma unroll
                             for (int e = 0; e < 4; ++e) {
@@ -374,12 +386,13 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
                 const int buf = li & 1;
                 if (!warp_wait(&tfull[buf], (li >> 1) & 1)) break;
                 tc_fence_after();
+                constexpr int NCH = (KIND == TC_W8A8 ? 8 : 4) / CSPLIT;  // 32-column chunks per warp
 #pragma unroll 1
                 for (int h = 0; h < C::MH; ++h) {
                     const int m = m0 + h * 128 + 32 * q + lane;
                     const float tm = (KIND == TC_W8A8 && m < p.M) ? __ldg(p.t + m) : 0.0f;
 #pragma unroll 1
-                    for (int c = 0; c < (KIND == TC_W8A8 ? 8 : 4); ++c) {
+                    for (int c = cs * NCH; c < (cs + 1) * NCH; ++c) {
                         uint32_t r[32];
                         const uint32_t col = (KIND == TC_W8A8 ? buf * 256 : buf * 256 + h * 128) + 32 * c;
                         tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + col, r);
@@ -425,7 +438,10 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
     } else {
         // ------------------------------ dequant warps (W4A16, W4A8) ------------------------------
         if constexpr (KIND != TC_W8A8) {
-            const int dt = threadIdx.x - 256;  // 0..127: the B tile row (column n) this thread fills
+            const int dthr = threadIdx.x - 32 * (4 + C::EPI);
+            const int dt = dthr & 127;                 // the B tile row (column n) this thread fills
+            constexpr int WSPLIT = C::DQ / 4;           // threads sharing one B row
+            const int ws = dthr >> 7;                   // this thread's share of the k-block's words
             int s = 0;
             uint32_t ph = 0;
             for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
@@ -468,7 +484,8 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
                         const uint32_t s2 = pack_bf16x2_rn(sv, sv);
                         const uint32_t z2 = pack_bf16x2_rn(128.0f + zv, 128.0f + zv);
 #pragma unroll
-                        for (int w = 0; w < 8; ++w) {
+                        for (int wi = 0; wi < 8 / WSPLIT; ++wi) {
+                            const int w = ws * (8 / WSPLIT) + wi;
                             const uint32_t word = raw[w * 128 + dt];
                             uint32_t R[4];
 #pragma unroll
@@ -484,7 +501,8 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
                     } else {
                         // one group of 128 k = 16 words; two words per 16-byte chunk
 #pragma unroll
-                        for (int c = 0; c < 8; ++c) {
+                        for (int ci = 0; ci < 8 / WSPLIT; ++ci) {
+                            const int c = ws * (8 / WSPLIT) + ci;
                             uint32_t o[4];
 #pragma unroll
                             for (int hw = 0; hw < 2; ++hw) {
