@@ -565,7 +565,7 @@ qg_status qg_gemm_w4a8(const int8_t* Xq, const float* t, int M, int K, const uin
     if (misaligned(Xq) || misaligned(t) || misaligned(packed) || misaligned(sg) || misaligned(Y) ||
         misaligned(part_dbg))
         return QG_ERR_ALIGN;
-    if (M >= qg::kTcMinM) {
+    if (M >= qg::kTcMinMW4A8) {
         qg::TcInt8Args a{Xq, t, nullptr, nullptr, packed, sg, Y, part_dbg, M, K, N};
         return tc_w4a8(a, stream);
     }
