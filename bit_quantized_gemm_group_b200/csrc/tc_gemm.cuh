@@ -318,23 +318,29 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
                 const int c = cs;                            // this warp's 32-column chunk
                 const int m = m0 + 32 * q + lane;
                 const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16);
-                auto stage_scales = [&](int g, int slot) {
-                    if (lane < 8) {
-                        const int n = n0 + 32 * c + 4 * lane;
-                        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                        if (g < KB && n < p.N) v = __ldg(reinterpret_cast<const float4*>(p.sg + (int64_t)g * p.N + n));
-                        *reinterpret_cast<float4*>(sgs + slot * 128 + 4 * lane) = v;
-                    }
+                // group scales travel global -> register (two groups ahead) -> smem slot (one
+                // group ahead) -> broadcast reads, so no load latency sits on the group loop
+                auto load_scales = [&](int g) {
+                    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+                    const int n = n0 + 32 * c + 4 * lane;
+                    if (lane < 8 && g < KB && n < p.N) v = __ldg(reinterpret_cast<const float4*>(p.sg + (int64_t)g * p.N + n));
+                    return v;
+                };
+                auto store_scales = [&](const float4& v, int slot) {
+                    if (lane < 8) *reinterpret_cast<float4*>(sgs + slot * 128 + 4 * lane) = v;
                 };
                 float sum[32];
 #pragma unroll
                 for (int i = 0; i < 32; ++i) sum[i] = 0.0f;
-                stage_scales(0, 0);
+                store_scales(load_scales(0), 0);
+                float4 s_ahead = load_scales(1);
                 bool ok = true;
                 for (int kb = 0; kb < KB; ++kb) {
                     const int gi = li * KB + kb;
                     const int buf = gi & 1;
-                    stage_scales(kb + 1, (kb + 1) & 1);  // next group's row, other slot
+                    store_scales(s_ahead, (kb + 1) & 1);  // group kb+1, loaded one group ago
+                    s_ahead = load_scales(kb + 2);
+                    __syncwarp();
                     if (!warp_wait(&tfull[buf], (gi >> 1) & 1)) { ok = false; break; }
                     tc_fence_after();
                     uint32_t r[32];
