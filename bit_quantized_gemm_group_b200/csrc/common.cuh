@@ -151,6 +151,26 @@ QG_DEV_INLINE bool mbar_wait(uint64_t* bar, uint32_t parity)
     }
 }
 
+// Same bounded wait, but backing off with nanosleep between polls (32 ns doubling to
+// 256 ns).  For roles with many warps waiting at once (epilogue, dequant, consumers):
+// their polling then leaves the issue slots to the warps doing the work.
+QG_DEV_INLINE bool mbar_wait_backoff(uint64_t* bar, uint32_t parity)
+{
+    if (mbar_try_wait(bar, parity)) return true;
+    const unsigned long long t0 = globaltimer_ns();
+    const unsigned long long lim = g_wait_limit_ns;
+    uint32_t ns = 32;
+    for (uint32_t it = 1;; ++it) {
+        __nanosleep(ns);
+        if (mbar_try_wait(bar, parity)) return true;
+        if (ns < 256) ns <<= 1;
+        if ((it & 15u) == 0u && globaltimer_ns() - t0 > lim) {
+            set_status(7u);
+            return false;
+        }
+    }
+}
+
 // Named barrier `id` over `count` threads that also ANDs a predicate across them.
 QG_DEV_INLINE int named_bar_and(uint32_t id, uint32_t count, bool v)
 {

@@ -156,7 +156,7 @@ QG_DEV_INLINE uint32_t bf16x2_mul(uint32_t a, uint32_t b)
 QG_DEV_INLINE bool warp_wait(uint64_t* bar, uint32_t parity)
 {
     uint32_t ok = 1;
-    if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity) ? 1u : 0u;
+    if ((threadIdx.x & 31) == 0) ok = mbar_wait_backoff(bar, parity) ? 1u : 0u;
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 

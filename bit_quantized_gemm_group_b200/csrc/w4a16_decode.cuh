@@ -201,7 +201,7 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
         const int n0 = slab * kDecBN;
         for (int g0 = ga; g0 < gb; g0 += kDecGroupsPerStage) {
             const int ng = min(kDecGroupsPerStage, gb - g0);
-            if (ok && !mbar_wait(&full[stage], phase)) ok = false;
+            if (ok && !mbar_wait_backoff(&full[stage], phase)) ok = false;
             const uint8_t* st = ring + stage * L::STAGE;
             if (ok && wg < ng) {
                 const int g = g0 + wg;
