@@ -93,14 +93,14 @@ struct TcCfg<TC_W4A16> {
 
 // W4A8: tile 128 x 128, k-block = one group of 128 int8; A 16 KB, raw 16 x 128 x 4 B = 8 KB,
 // B 128 x 128 int8 = 16 KB per stage; TMEM holds two group accumulators (ping-pong); each
-// of the 16 epilogue warps keeps the running fp32 sum of its 32 columns in registers.
+// of the 8 epilogue warps keeps the running fp32 sum of its 64 columns in registers.
 template <>
 struct TcCfg<TC_W4A8> {
     static constexpr int BM = 128, BN = 128, BK = 128;
     static constexpr int A_BYTES = 128 * 128, RAW_BYTES = 16 * 128 * 4, B_BYTES = 128 * 128;
     static constexpr int STAGE = A_BYTES + B_BYTES + RAW_BYTES;
     static constexpr int ST = 4;
-    static constexpr int EPI = 16, DQ = 4;  // 16 epilogue warps: each owns 32 columns of a lane quarter
+    static constexpr int EPI = 8, DQ = 4;   // 8 epilogue warps: each owns 64 columns of a lane quarter
     static constexpr int THREADS = 32 * (4 + EPI + DQ);
     static constexpr int TMEM_COLS = 256;   // two group buffers (ping-pong) of 128 columns
     static constexpr int MH = 1;
@@ -307,31 +307,29 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
         for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x, ++li) {
             const int m0 = (tile % p.m_tiles) * C::BM, n0 = (tile / p.m_tiles) * C::BN;
             if constexpr (KIND == TC_W4A8) {
-                // Per group: drain the int32 partial P of this warp's 32 columns from its TMEM
+                // Per group: drain the int32 partial P of this warp's CW columns from its TMEM
                 // buffer and fold it into the running fp32 sum held in registers:
                 //     sum += P * s_g        (exact int32 -> fp32, one fma)
-                // The next group's scale row is staged in this warp's smem slot (one float4 per
-                // lane) while the current one is used.  After the last group the sum is scaled
-                // by t[m] and stored as bf16.
-                static_assert(C::BN / CSPLIT == 32, "one 32-column chunk per epilogue warp");
+                // Group scales travel global -> register (two groups ahead) -> smem slot (one
+                // group ahead) -> broadcast reads, so no load latency sits on the group loop.
+                // After the last group the sum is scaled by t[m] and stored as bf16.
+                constexpr int CW = C::BN / CSPLIT;   // columns of this warp
                 float* sgs = reinterpret_cast<float*>(smem + S::EPI_OFF) + e * 256;
-                const int c = cs;                            // this warp's 32-column chunk
+                const int cb = cs * CW;
                 const int m = m0 + 32 * q + lane;
                 const uint32_t trow = tmem + ((uint32_t)(32 * q) << 16);
-                // group scales travel global -> register (two groups ahead) -> smem slot (one
-                // group ahead) -> broadcast reads, so no load latency sits on the group loop
                 auto load_scales = [&](int g) {
                     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                    const int n = n0 + 32 * c + 4 * lane;
-                    if (lane < 8 && g < KB && n < p.N) v = __ldg(reinterpret_cast<const float4*>(p.sg + (int64_t)g * p.N + n));
+                    const int n = n0 + cb + 4 * lane;
+                    if (4 * lane < CW && g < KB && n < p.N) v = __ldg(reinterpret_cast<const float4*>(p.sg + (int64_t)g * p.N + n));
                     return v;
                 };
                 auto store_scales = [&](const float4& v, int slot) {
-                    if (lane < 8) *reinterpret_cast<float4*>(sgs + slot * 128 + 4 * lane) = v;
+                    if (4 * lane < CW) *reinterpret_cast<float4*>(sgs + slot * 128 + 4 * lane) = v;
                 };
-                float sum[32];
+                float sum[CW];
 #pragma unroll
-                for (int i = 0; i < 32; ++i) sum[i] = 0.0f;
+                for (int i = 0; i < CW; ++i) sum[i] = 0.0f;
                 store_scales(load_scales(0), 0);
                 float4 s_ahead = load_scales(1);
                 bool ok = true;
@@ -343,36 +341,42 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
                     __syncwarp();
                     if (!warp_wait(&tfull[buf], (gi >> 1) & 1)) { ok = false; break; }
                     tc_fence_after();
-                    uint32_t r[32];
-                    tmem_ld_32x32b_x32(trow + buf * 128 + 32 * c, r);
-                    tmem_ld_wait();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(&tempty[buf]);  // the partial is in registers now
-                    if (p.dbg && m < p.M) {
-                        int32_t* drow = p.dbg + ((int64_t)m * KB + kb) * p.N + n0 + 32 * c;
-#pragma unroll
-                        for (int i = 0; i < 32; i += 4)
-                            if (n0 + 32 * c + i < p.N)
-                                *reinterpret_cast<int4*>(drow + i) = make_int4(r[i], r[i + 1], r[i + 2], r[i + 3]);
-                    }
                     const float* sv = sgs + (kb & 1) * 128;
 #pragma unroll
-                    for (int i = 0; i < 32; i += 4) {
-                        const float4 s4 = *reinterpret_cast<const float4*>(sv + i);  // broadcast
-                        sum[i + 0] = fmaf(i2f_small(r[i + 0]), s4.x, sum[i + 0]);
-                        sum[i + 1] = fmaf(i2f_small(r[i + 1]), s4.y, sum[i + 1]);
-                        sum[i + 2] = fmaf(i2f_small(r[i + 2]), s4.z, sum[i + 2]);
-                        sum[i + 3] = fmaf(i2f_small(r[i + 3]), s4.w, sum[i + 3]);
+                    for (int cc = 0; cc < CW / 32; ++cc) {
+                        const int c = cb / 32 + cc;
+                        uint32_t r[32];
+                        tmem_ld_32x32b_x32(trow + buf * 128 + 32 * c, r);
+                        tmem_ld_wait();
+                        if (cc == CW / 32 - 1) {       // the whole partial is in registers now
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&tempty[buf]);
+                        }
+                        if (p.dbg && m < p.M) {
+                            int32_t* drow = p.dbg + ((int64_t)m * KB + kb) * p.N + n0 + 32 * c;
+#pragma unroll
+                            for (int i = 0; i < 32; i += 4)
+                                if (n0 + 32 * c + i < p.N)
+                                    *reinterpret_cast<int4*>(drow + i) = make_int4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+                        }
+#pragma unroll
+                        for (int i = 0; i < 32; i += 4) {
+                            const float4 s4 = *reinterpret_cast<const float4*>(sv + 32 * cc + i);  // broadcast
+                            sum[32 * cc + i + 0] = fmaf(i2f_small(r[i + 0]), s4.x, sum[32 * cc + i + 0]);
+                            sum[32 * cc + i + 1] = fmaf(i2f_small(r[i + 1]), s4.y, sum[32 * cc + i + 1]);
+                            sum[32 * cc + i + 2] = fmaf(i2f_small(r[i + 2]), s4.z, sum[32 * cc + i + 2]);
+                            sum[32 * cc + i + 3] = fmaf(i2f_small(r[i + 3]), s4.w, sum[32 * cc + i + 3]);
+                        }
                     }
                 }
                 if (!ok) break;
                 if (m < p.M) {
                     const float tm = __ldg(p.t + m);
-                    uint16_t* yrow = p.Y + (int64_t)m * p.N + n0 + 32 * c;
+                    uint16_t* yrow = p.Y + (int64_t)m * p.N + n0 + cb;
 #pragma unroll
-                    for (int i = 0; i < 32; i += 8) {
-                        if (n0 + 32 * c + i < p.N) {
+                    for (int i = 0; i < CW; i += 8) {
+                        if (n0 + cb + i < p.N) {
                             uint4 v;
                             v.x = pack_bf16x2_rn(__fmul_rn(tm, sum[i + 0]), __fmul_rn(tm, sum[i + 1]));
                             v.y = pack_bf16x2_rn(__fmul_rn(tm, sum[i + 2]), __fmul_rn(tm, sum[i + 3]));
