@@ -197,7 +197,7 @@ qg_status make_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, size_t elem_bytes
 // ---------------------------------------------------------------------------
 struct DecodePlan {
     int MP, G, nslabs, units, grid;
-    size_t partial_bytes, counter_bytes;
+    size_t partial_bytes;
 };
 
 DecodePlan decode_plan(int M, int K, int N)
@@ -210,28 +210,46 @@ DecodePlan decode_plan(int M, int K, int N)
     d.units = d.G * d.nslabs;
     d.grid = std::min(std::min(num_sms(), d.units), qg::kMaxPieces);
     d.partial_bytes = (size_t)d.grid * 2 * qg::kDecBN * d.MP * sizeof(float);
-    // The counter region has one fixed size for every shape, so that the counters of
-    // one call never overlap the partial tiles another shape wrote into the same buffer.
-    d.counter_bytes = (size_t)qg::kDecMaxSlabs * sizeof(int);
     return d;
 }
 
-bool decode_eligible(int M, int N) { return M >= 1 && N % 16 == 0 && (N + qg::kDecBN - 1) / qg::kDecBN <= qg::kDecMaxSlabs; }
+bool decode_eligible(int M, int N) { return M >= 1 && N % 16 == 0; }
+
+template <typename Kern, typename... Args>
+qg_status launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, qg_stream_t stream, Args... args)
+{
+    // programmatic dependent launch: the grid may start while the previous kernel in the
+    // stream drains; the kernel orders itself with griddepcontrol.wait
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    QG_CUDA(cudaLaunchKernelEx(&cfg, kern, args...));
+    return QG_OK;
+}
 
 template <int MT, bool BF16>
 qg_status launch_w4a16_decode(const qg::SkinnyParams& sp, const uint32_t* packed, const uint16_t* scales,
                               const uint8_t* zeros, void* ws, qg_stream_t stream)
 {
-    constexpr int ST = MT == 1 ? 4 : MT == 2 ? 3 : 2;  // ring depth that fits next to the reduction buffer
-    static_assert(qg::DecodeSmem<MT, ST>::TOTAL <= 227 * 1024, "decode kernel shared memory");
-    auto kern = qg::w4a16_decode_kernel<MT, BF16, ST>;
-    const size_t smem = qg::DecodeSmem<MT, ST>::TOTAL;
+    constexpr int WS = MT == 1 ? 2 : 1;                 // two warps per group at M <= 8
+    constexpr int ST = MT == 1 ? 4 : MT == 2 ? 3 : 2;  // ring depth that fits next to the reduction tile
+    using L = qg::DecodeSmem<MT, ST, WS>;
+    static_assert(L::TOTAL <= 227 * 1024, "decode kernel shared memory");
+    auto kern = qg::w4a16_decode_kernel<MT, BF16, ST, WS>;
+    const size_t smem = L::TOTAL;
     static KernelInfo info;
     int occ = 1;
-    qg_status st = prepare_kernel(info, kern, 384, smem, &occ);
+    qg_status st = prepare_kernel(info, kern, L::THREADS, smem, &occ);
     if (st != QG_OK) return st;
     const DecodePlan d = decode_plan(sp.M, sp.K, sp.N);
-    CUtensorMap tw, ts, tz;
+    CUtensorMap tw, ts, tz, tx;
     if ((st = make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, sp.N, sp.K / 8, 32, 16,
                            CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
         return st;
@@ -241,15 +259,13 @@ qg_status launch_w4a16_decode(const qg::SkinnyParams& sp, const uint32_t* packed
     if ((st = make_tmap_2d(&tz, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, zeros, sp.N, d.G, 128, 1,
                            CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK)
         return st;
-    CUtensorMap tx;
     if ((st = make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, sp.X, sp.K, sp.M, 64, 8 * MT,
                            CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
         return st;
     qg::DecodeParams p;
     p.X = sp.X;
     p.Y = sp.Y;
-    p.counters = static_cast<int*>(ws);
-    p.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + d.counter_bytes);
+    p.partials = static_cast<float*>(ws);
     p.M = sp.M;
     p.K = sp.K;
     p.N = sp.N;
@@ -257,20 +273,8 @@ qg_status launch_w4a16_decode(const qg::SkinnyParams& sp, const uint32_t* packed
     p.nslabs = d.nslabs;
     p.units = d.units;
     p.grid = d.grid;
-    // programmatic dependent launch: this grid may start while the previous kernel in
-    // the stream drains; the kernel orders itself with griddepcontrol.wait.
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(d.grid);
-    cfg.blockDim = dim3(384);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = reinterpret_cast<cudaStream_t>(stream);
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    QG_CUDA(cudaLaunchKernelEx(&cfg, kern, p, tw, ts, tz, tx));
-    return QG_OK;
+    if ((st = launch_pdl(kern, dim3(d.grid), dim3(L::THREADS), smem, stream, p, tw, ts, tz, tx)) != QG_OK) return st;
+    return launch_pdl(qg::w4a16_decode_fixup_kernel<BF16>, dim3(d.nslabs), dim3(256), 0, stream, p, 8 * MT);
 }
 
 template <bool BF16>
@@ -447,8 +451,7 @@ size_t qg_workspace_size(qg_op op, int M, int K, int N)
     switch (op) {
         case QG_OP_GEMM_W4A16: {
             if (!decode_eligible(M, N)) return 0;
-            const DecodePlan d = decode_plan(M, K, N);
-            return d.counter_bytes + d.partial_bytes;
+            return decode_plan(M, K, N).partial_bytes;
         }
         default: return 0;
     }
@@ -634,14 +637,14 @@ qg_status qg_selftest_bounded_wait(uint64_t limit_ns, qg_stream_t stream)
 // inside a capture), plugins and custom operators inside a host framework that owns
 // every device allocation and gives the operator no allocator, and latency-bound
 // paths where an allocation's implicit device synchronisation is unacceptable.
-// For them the decode kernel's scratch (arrival counters and partial tiles) lives
+// For them the decode kernel's scratch (the partial tiles of split column slabs) lives
 // in one statically sized device array instead of a caller workspace.
 // ===========================================================================
 namespace {
 
 // 6 MiB per GPU that loads this library, held until the process exits.  The
 // largest decode launch (32 tokens, one CTA per SM, at most 160 CTAs) needs
-// 32 KiB of counters + 160 x 2 x 128 x 32 x 4 B of partial tiles = 5.3 MiB.
+// 160 x 2 x 128 x 32 x 4 B of partial tiles = 5 MiB.
 constexpr size_t kNoAllocScratchBytes = size_t(6) << 20;
 static __device__ __align__(256) unsigned char qg_noalloc_scratch[kNoAllocScratchBytes];
 
@@ -686,7 +689,7 @@ extern "C" qg_status qg_gemm_w4a16_noalloc(const void* X, qg_dtype xdt, int M, i
     void* ws = nullptr;
     qg_status st = noalloc_scratch(&ws);
     if (st != QG_OK) return st;
-    // the arrival counters must start at zero; the array keeps whatever the last call left
-    QG_CUDA(cudaMemsetAsync(ws, 0, (size_t)qg::kDecMaxSlabs * sizeof(int), reinterpret_cast<cudaStream_t>(stream)));
+    // The decode kernel writes every partial tile before the fixup kernel reads it, so
+    // nothing in the array has to start at zero; it keeps the last call's contents.
     return qg_gemm_w4a16(X, xdt, M, K, N, packed, scales, zeros, group, Y, ws, kNoAllocScratchBytes, stream);
 }

@@ -9,30 +9,37 @@
 // Work split (stream-K).  The N columns form slabs of 128; one unit is one group
 // (128 k) of one slab.  The persistent grid (one CTA per SM) divides the
 // nslabs x G units into equal contiguous ranges, so every SM streams the same
-// number of bytes.  A CTA's range is a list of slab pieces; a piece that covers a
-// whole slab writes Y directly, a partial piece writes its fp32 tile to the
-// workspace and bumps the slab's counter; the CTA that brings the counter to the
-// number of pieces sums all pieces in CTA order (deterministic) and writes Y, then
-// resets the counter to zero.
+// number of bytes.  A CTA's range is a list of slab pieces: a piece that covers a
+// whole slab writes Y directly; a partial piece writes its fp32 tile to the workspace
+// (slot 0 for the CTA's first piece, 1 for its last).  The follow-up kernel
+// `w4a16_decode_fixup_kernel` sums the pieces of every split slab in CTA order
+// (deterministic; no atomics, no counters) and writes Y.
 //
-// Data movement.  One producer warp streams each group's packed words (16 rows of
+// Data movement.  One producer thread streams each group's packed words (16 rows of
 // the [K/8][N] matrix x 128 columns, as four 128-byte-wide boxes with 128-byte
-// swizzle), fp16 scales and u8 zeros into a ring of shared-memory stages with TMA;
-// a stage holds up to four groups of one slab.  Eight consumer warps: warp (wn, wg)
-// takes columns 64wn..64wn+63 of group wg of each stage.
+// swizzle), fp16 scales, u8 zeros and the group's activation tile into a ring of
+// shared-memory stages with TMA; a stage holds up to four groups of one slab.
+// Consumer warp (wn, wg, ws) takes columns 64wn..64wn+63 of group wg of each stage and
+// the ws-th share of its four 32-k steps (WS = 1 or 2 warps per group).
 //
 // Math.  Swap-AB mma.sync (weights are the m16 operand, up to 32 tokens are n8
 // tiles).  A lane's 128-bit read gives 4 columns x 8 k; OR-ing a nibble pair into
 // the exponent field of a bf16 (fp16) pair yields exactly 128 + q (1024 + q) with
 // one LOP3, so the MMA accumulates D = sum (128 + q) x per group.  The zero point and
 // scale are applied once per group and output element:
-//     acc += s * (D - (128 + z) * sum_{k in g} x)
+//     acc += s * (D - (128 + z) * sum_{k} x)
 // where sum x comes from one extra MMA tile whose A operand is all ones, already in
-// the accumulator layout.  Inside a 32-k step the k order is permuted so that a
+// the accumulator layout (the correction is linear, so each warp applies it to its
+// own share of the steps).  Inside a 32-k step the k order is permuted so that a
 // lane's own word feeds its fragment slots; the activation pairs get the same
-// permutation with two byte permutes per register.  Shared-memory rows are visited
-// in the order 0,2,4,6 | 1,3,5,7 | 8,... so the eight lanes of each 128-bit access
-// phase hit eight different 16-byte bank groups under the 128-byte swizzle.
+// permutation with byte permutes.  Shared-memory rows are visited in the order
+// 0,2,4,6 | 1,3,5,7 | 8,... so the eight lanes of each 128-bit access phase hit eight
+// different 16-byte bank groups under the 128-byte swizzle.
+//
+// Programmatic dependent launch: the kernel lets the next grid launch at once; the
+// producer requests the first ring-full of weights before waiting for the previous
+// grid (griddepcontrol.wait), and nothing that depends on it (X, Y, the workspace)
+// is touched before that wait.
 #pragma once
 #include "common.cuh"
 #include "w4a16_skinny.cuh"
@@ -42,77 +49,84 @@ namespace qg {
 struct DecodeParams {
     const uint16_t* X;
     uint16_t* Y;
-    float* partials;  // [grid][2][128][MP]
-    int* counters;    // [kDecMaxSlabs], zero between calls
+    float* partials;  // [grid][2][MP][128]
     int M, K, N;
     int G, nslabs, units, grid;
 };
 
-constexpr int kDecBN = 128;             // columns per slab
-constexpr int kDecMaxSlabs = 8192;      // counters at the start of the workspace: N <= 8192 * 128
+constexpr int kDecBN = 128;               // columns per slab
 constexpr int kDecGroupsPerStage = 4;
 constexpr int kDecGroupW = 16 * 128 * 4;  // packed words of one group: 16 rows x 128 columns x 4 B
 constexpr int kDecScaleOff = 4 * kDecGroupW;
 constexpr int kDecZeroOff = kDecScaleOff + 4 * 256;
 constexpr int kDecXOff = kDecZeroOff + 4 * 128 + 512;  // 1 KB aligned
-constexpr int kMaxPieces = 160;         // >= grid: pieces of one slab (one per CTA at most)
+constexpr int kMaxPieces = 160;           // grid cap: pieces of one slab (one per CTA at most)
 
 QG_DEV_INLINE int dec_first_unit(int c, int units, int grid) { return (int)((int64_t)c * units / grid); }
 
+// CTA holding unit u of the static split
+QG_DEV_INLINE int dec_cta_of_unit(int u, int units, int grid)
+{
+    int c = (int)((int64_t)u * grid / units);
+    while (c > 0 && dec_first_unit(c, units, grid) > u) --c;
+    while (dec_first_unit(c + 1, units, grid) <= u) ++c;
+    return c;
+}
+
 // Stage: 4 groups x {packed words 8 KB, fp16 scales 256 B, u8 zeros 128 B, X tile
 // MP tokens x 128 k bf16 as two 128-byte-swizzled boxes of 64 k}.
-template <int MT, int ST>
+template <int MT, int ST, int WS>
 struct DecodeSmem {
     static constexpr int MP = 8 * MT;
     static constexpr int XG = MP * 256;  // X bytes per group
     static constexpr int STAGE = kDecXOff + 4 * XG;
     static constexpr int RS = kDecBN + 8;  // padded row of the [token][column] reduction tile
-    static constexpr int RED = 4 * MP * RS * 4;
-    static constexpr int TOTAL = ST * STAGE + RED + 2 * ST * 8 + 64 + 4 * kMaxPieces + 1024;
+    static constexpr int NRED = 4 * WS;    // warps adding into one column half
+    static constexpr int RED = NRED * MP * RS * 4;
+    static constexpr int TOTAL = ST * STAGE + RED + 2 * ST * 8 + 1024;
     static constexpr uint32_t GROUP_TX = kDecGroupW + 256 + 128 + XG;
+    static constexpr int NC = 8 * WS;      // consumer warps
+    static constexpr int THREADS = 32 * NC + 128;
 };
 
-template <int MT, bool BF16, int ST>
-__global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams p,
-                                                               const __grid_constant__ CUtensorMap tm_w,
-                                                               const __grid_constant__ CUtensorMap tm_s,
-                                                               const __grid_constant__ CUtensorMap tm_z,
-                                                               const __grid_constant__ CUtensorMap tm_x)
+template <int MT, bool BF16, int ST, int WS>
+__global__ void __launch_bounds__(DecodeSmem<MT, ST, WS>::THREADS, 1)
+    w4a16_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_w,
+                        const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_z,
+                        const __grid_constant__ CUtensorMap tm_x)
 {
     using H = HalfOps<BF16>;
+    using L = DecodeSmem<MT, ST, WS>;
     constexpr int MP = 8 * MT;
+    constexpr int NC = L::NC;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    using L = DecodeSmem<MT, ST>;
     uint8_t* ring = smem;
     float* red = reinterpret_cast<float*>(smem + ST * L::STAGE);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * L::STAGE + L::RED);
     uint64_t* empty = full + ST;
-    int* flag = reinterpret_cast<int*>(empty + ST);            // [16]
-    int* piece_off = flag + 16;                                   // [kMaxPieces] partial-tile offsets
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.G;
     const int u0 = dec_first_unit(blockIdx.x, p.units, p.grid), u1 = dec_first_unit(blockIdx.x + 1, p.units, p.grid);
 
-    // The next grid in the stream may start launching now; it waits for this one to
-    // finish (griddepcontrol.wait) before it touches X, Y or the workspace.
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     if (threadIdx.x == 0) {
         for (int i = 0; i < ST; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], 8);
+            mbar_init(&empty[i], NC);
         }
         fence_mbar_init();
     }
     __syncthreads();
 
-    if (warp >= 8) {
+    if (warp >= NC) {
         // ---------------- producer warpgroup (one thread issues TMA) ----------------
-        // Registers: launched with 384 x 168; this warpgroup gives up 128 x 128 and the
-        // two consumer warpgroups take 256 x 64 (168 -> 232).
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");
-        if (warp == 8 && lane == 0) {
+        // Register split (setmaxnreg works per warpgroup): this warpgroup keeps few
+        // registers and hands the rest to the consumer warpgroups.
+        if constexpr (WS == 1) asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");   // 384 x 168 at launch
+        else asm volatile("setmaxnreg.dec.sync.aligned.u32 24;");                    // 640 x 96 at launch
+        if (warp == NC && lane == 0) {
             tma_prefetch_desc(&tm_w);
             tma_prefetch_desc(&tm_s);
             tma_prefetch_desc(&tm_z);
@@ -173,9 +187,11 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
     }
 
     // ---------------- consumers ----------------
-    asm volatile("setmaxnreg.inc.sync.aligned.u32 232;");
+    if constexpr (WS == 1) asm volatile("setmaxnreg.inc.sync.aligned.u32 232;");
+    else asm volatile("setmaxnreg.inc.sync.aligned.u32 112;");
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int wn = warp & 1, wg = warp >> 1;
+    const int wn = warp & 1, wg = (warp >> 1) & 3, ws = warp >> 3;
+    constexpr int SPW = 4 / WS;  // 32-k steps per warp per group
     const int g8 = lane >> 2, t4 = lane & 3;
     const uint32_t ONE = BF16 ? 0x3F803F80u : 0x3C003C00u;
     float acc[2][2][MT][4];
@@ -194,7 +210,7 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
     bool first_piece = true;
     // After a wait gives up (status already recorded) the warp keeps walking the same
     // schedule without waiting or computing, so that every named barrier still sees
-    // all 256 consumer threads; nothing is written to global memory after that.
+    // all consumer threads; nothing is written to global memory after that.
     for (int u = u0; u < u1;) {
         const int slab = u / G, ga = u % G;
         const int gb = min(G, ga + (u1 - u));
@@ -204,7 +220,6 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
             if (ok && !mbar_wait_backoff(&full[stage], phase)) ok = false;
             const uint8_t* st = ring + stage * L::STAGE;
             if (ok && wg < ng) {
-                const int g = g0 + wg;
                 // per-column scale and (128 + z) of the lane's 8 columns
                 float sc[2][4], zc[2][4];
 #pragma unroll
@@ -232,8 +247,10 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
                             for (int e = 0; e < 4; ++e) D[h][c][j][e] = 0.0f;
                 }
                 const uint8_t* wbase = st + wg * kDecGroupW;
+                const uint8_t* xg = st + kDecXOff + wg * L::XG;
 #pragma unroll
-                for (int s = 0; s < 4; ++s) {
+                for (int si = 0; si < SPW; ++si) {
+                    const int s = ws * SPW + si;
                     const int row = 8 * (s >> 1) + 2 * t4 + (s & 1);  // kb row within the group
                     uint4 wv[2];
 #pragma unroll
@@ -241,7 +258,7 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
                         wv[h] = *reinterpret_cast<const uint4*>(wbase + (2 * wn + h) * 2048 + row * 128 +
                                                                 ((g8 ^ (row & 7)) << 4));
                     uint32_t xb[MT][4];
-                    const uint8_t* xs = st + kDecXOff + wg * L::XG + (row >> 3) * (L::XG / 2);
+                    const uint8_t* xs = xg + (row >> 3) * (L::XG / 2);
 #pragma unroll
                     for (int j = 0; j < MT; ++j) {
                         const int tok = 8 * j + g8;  // rows >= M are zero (TMA fill)
@@ -275,7 +292,7 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
                         mma_16816<BF16>(Dx[j], ONE, ONE, ONE, ONE, xb[j][2], xb[j][3]);
                     }
                 }
-                // group epilogue: acc += s * (D - (128 + z) * sum x)
+                // group epilogue (this warp's steps): acc += s * (D - (128 + z) * sum x)
 #pragma unroll
                 for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -293,11 +310,12 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
             if (lane == 0) mbar_arrive(&empty[stage]);
             if (++stage == ST) { stage = 0; phase ^= 1; }
         }
-        // ---------------- piece end: reduce the four group-warps, then write ----------------
+
+        // ---------------- piece end: reduce the group-warps of each column half ----------------
         // Reduction tile layout [token][column] with a padded row, so that the fragment
         // stores are at most 2-way conflicted and every later pass reads consecutive words.
         constexpr int RS = L::RS;
-        float* myred = red + (size_t)wg * MP * RS;
+        float* myred = red + (size_t)(wg * WS + ws) * MP * RS;
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
@@ -311,91 +329,85 @@ __global__ void __launch_bounds__(384, 1) w4a16_decode_kernel(const DecodeParams
 #pragma unroll
                     for (int e = 0; e < 4; ++e) acc[h][cp][j][e] = 0.0f;
                 }
-        named_bar_sync(1, 256);
+        named_bar_sync(1, 32 * NC);
         const int mrows = min(p.M, MP);
-        // sum the four group-warps: 4 consecutive columns per thread step
-        for (int e = threadIdx.x; e < mrows * (kDecBN / 4); e += 256) {
-            const int tok = e / (kDecBN / 4), c4 = 4 * (e % (kDecBN / 4));
-            float4 v = *reinterpret_cast<const float4*>(red + tok * RS + c4);
-#pragma unroll
-            for (int q = 1; q < 4; ++q) {
-                const float4 w = *reinterpret_cast<const float4*>(red + (size_t)q * MP * RS + tok * RS + c4);
-                v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
-            }
-            *reinterpret_cast<float4*>(red + tok * RS + c4) = v;
-        }
-        named_bar_sync(1, 256);
-        const int nvalid = min(kDecBN, p.N - n0);
         // any warp that gave up makes the whole CTA skip its global writes
-        const int all_ok = named_bar_and(1, 256, ok);
+        const int all_ok = named_bar_and(1, 32 * NC, ok);
         if (!all_ok) {
             ok = false;
-        } else if (ga == 0 && gb == G) {
-            for (int e = threadIdx.x; e < mrows * kDecBN; e += 256) {
-                const int tok = e / kDecBN, nn = e % kDecBN;
-                if (nn < nvalid) p.Y[(int64_t)tok * p.N + n0 + nn] = H::to_bits(red[tok * RS + nn]);
-            }
         } else {
-            // partial tile [token][128] in the workspace, then arrive on the slab's counter
-            const int slot = first_piece ? 0 : 1;
-            float* mine = p.partials + ((size_t)blockIdx.x * 2 + slot) * kDecBN * MP;
-            for (int e = threadIdx.x; e < mrows * (kDecBN / 4); e += 256) {
+            const bool whole = ga == 0 && gb == G;
+            const int nvalid = min(kDecBN, p.N - n0);
+            float* mine = p.partials + ((size_t)blockIdx.x * 2 + (first_piece ? 0 : 1)) * MP * kDecBN;
+            // sum the group-warps, 4 consecutive columns per thread step; write Y (whole
+            // slab) or this piece's partial tile [token][128] (split slab)
+            for (int e = threadIdx.x; e < mrows * (kDecBN / 4); e += 32 * NC) {
                 const int tok = e / (kDecBN / 4), c4 = 4 * (e % (kDecBN / 4));
-                *reinterpret_cast<float4*>(mine + tok * kDecBN + c4) = *reinterpret_cast<const float4*>(red + tok * RS + c4);
-            }
-            named_bar_sync(1, 256);
-            if (threadIdx.x == 0) {
-                __threadfence();  // the CTA's partial stores (ordered by the barrier) before the arrival
-                // CTAs that hold a piece of this slab: the ones containing its first and last unit
-                const int ufirst = slab * G, ulast = slab * G + G - 1;
-                int cf = (int)((int64_t)ufirst * p.grid / p.units);
-                while (cf > 0 && dec_first_unit(cf, p.units, p.grid) > ufirst) --cf;
-                while (dec_first_unit(cf + 1, p.units, p.grid) <= ufirst) ++cf;
-                int cl = (int)((int64_t)ulast * p.grid / p.units);
-                while (cl > 0 && dec_first_unit(cl, p.units, p.grid) > ulast) --cl;
-                while (dec_first_unit(cl + 1, p.units, p.grid) <= ulast) ++cl;
-                const int old = atomicAdd(&p.counters[slab], 1);
-                const bool last = old == cl - cf;
-                flag[0] = last ? 1 : 0;
-                flag[1] = cl - cf + 1;
-                if (last) {
-                    p.counters[slab] = 0;
-                    for (int c = cf; c <= cl; ++c) {
-                        const int sl = dec_first_unit(c, p.units, p.grid) >= slab * G ? 0 : 1;
-                        piece_off[c - cf] = (c * 2 + sl) * kDecBN * MP;
-                    }
-                    __threadfence();  // acquire: the other pieces' partials are visible from here on
+                float4 v = *reinterpret_cast<const float4*>(red + tok * RS + c4);
+#pragma unroll
+                for (int q = 1; q < L::NRED; ++q) {
+                    const float4 w = *reinterpret_cast<const float4*>(red + (size_t)q * MP * RS + tok * RS + c4);
+                    v.x += w.x; v.y += w.y; v.z += w.z; v.w += w.w;
                 }
-            }
-            named_bar_sync(1, 256);
-            if (flag[0]) {
-                const int np = flag[1];
-                for (int e = threadIdx.x; e < mrows * (kDecBN / 4); e += 256) {
-                    const int tok = e / (kDecBN / 4), c4 = 4 * (e % (kDecBN / 4));
-                    const int off = tok * kDecBN + c4;
-                    float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-                    int i = 0;
-                    for (; i + 4 <= np; i += 4) {  // four independent loads in flight, summed in piece order
-                        float4 a[4];
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) a[r] = __ldcg(reinterpret_cast<const float4*>(p.partials + piece_off[i + r] + off));
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) { v.x += a[r].x; v.y += a[r].y; v.z += a[r].z; v.w += a[r].w; }
-                    }
-                    for (; i < np; ++i) {
-                        const float4 a = __ldcg(reinterpret_cast<const float4*>(p.partials + piece_off[i] + off));
-                        v.x += a.x; v.y += a.y; v.z += a.z; v.w += a.w;
-                    }
+                if (whole) {
                     const float vv[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
                     for (int r = 0; r < 4; ++r)
                         if (c4 + r < nvalid) p.Y[(int64_t)tok * p.N + n0 + c4 + r] = H::to_bits(vv[r]);
+                } else {
+                    *reinterpret_cast<float4*>(mine + tok * kDecBN + c4) = v;
                 }
             }
         }
-        named_bar_sync(1, 256);
+        named_bar_sync(1, 32 * NC);
         first_piece = false;
         u += gb - ga;
+    }
+}
+
+// Sums the pieces of every slab that the decode grid split between CTAs, in CTA order,
+// and writes Y.  One CTA per slab; slabs held by one CTA were written directly.
+template <bool BF16>
+__global__ void __launch_bounds__(256) w4a16_decode_fixup_kernel(const DecodeParams p, int MP)
+{
+    using H = HalfOps<BF16>;
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    const int slab = blockIdx.x;
+    const int G = p.G;
+    const int cf = dec_cta_of_unit(slab * G, p.units, p.grid);
+    const int cl = dec_cta_of_unit(slab * G + G - 1, p.units, p.grid);
+    if (cf == cl) return;  // the whole slab was one piece: written by the decode kernel
+    __shared__ int off[kMaxPieces];
+    for (int c = cf + threadIdx.x; c <= cl; c += blockDim.x) {
+        const int sl = dec_first_unit(c, p.units, p.grid) >= slab * G ? 0 : 1;  // first piece of CTA c?
+        off[c - cf] = (c * 2 + sl) * MP * kDecBN;
+    }
+    __syncthreads();
+    asm volatile("griddepcontrol.wait;" ::: "memory");  // the decode grid's partial tiles are complete
+    const int np = cl - cf + 1;
+    const int n0 = slab * kDecBN;
+    const int nvalid = min(kDecBN, p.N - n0);
+    const int mrows = min(p.M, MP);
+    for (int e = threadIdx.x; e < mrows * (kDecBN / 4); e += blockDim.x) {
+        const int tok = e / (kDecBN / 4), c4 = 4 * (e % (kDecBN / 4));
+        const int o = tok * kDecBN + c4;
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        int i = 0;
+        for (; i + 4 <= np; i += 4) {  // four independent loads in flight, summed in piece order
+            float4 a[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) a[r] = __ldcg(reinterpret_cast<const float4*>(p.partials + off[i + r] + o));
+#pragma unroll
+            for (int r = 0; r < 4; ++r) { v.x += a[r].x; v.y += a[r].y; v.z += a[r].z; v.w += a[r].w; }
+        }
+        for (; i < np; ++i) {
+            const float4 a = __ldcg(reinterpret_cast<const float4*>(p.partials + off[i] + o));
+            v.x += a.x; v.y += a.y; v.z += a.z; v.w += a.w;
+        }
+        const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int r = 0; r < 4; ++r)
+            if (c4 + r < nvalid) p.Y[(int64_t)tok * p.N + n0 + c4 + r] = H::to_bits(vv[r]);
     }
 }
 

@@ -110,13 +110,12 @@ qg_status qg_pack_nibbles(const uint8_t* codes, int K, int N, uint32_t* packed, 
  * group    128 (the only group size the GEMM kernels take).
  * Rules: K % 128 == 0, N % 8 == 0.  Accumulation is fp32.
  * workspace: NULL, or a device buffer of at least
- *   qg_workspace_size(QG_OP_GEMM_W4A16, M, K, N) bytes that was zero-filled before
- *   its first use.  With a workspace, decode shapes (N % 16 == 0, N <= 2^20)
- *   use the stream-K kernel, which keeps per-slab partial tiles and arrival
- *   counters there; every call that completes leaves the counters at zero again.
- *   After a device error (qg_device_status() != QG_OK) zero-fill it again.
- *   The workspace must not be shared by calls that may run concurrently.
- *   Without one, the split-K reduction runs in distributed shared memory (slower).
+ *   qg_workspace_size(QG_OP_GEMM_W4A16, M, K, N) bytes (contents irrelevant).  With
+ *   a workspace, decode shapes (N % 16 == 0) use the stream-K kernel, which writes
+ *   the partial tiles of split column slabs there and sums them in a second kernel,
+ *   in a fixed order.  The workspace must not be shared by calls that may run
+ *   concurrently.  Without one, the split-K reduction runs in distributed shared
+ *   memory (slower).
  * ------------------------------------------------------------------------ */
 qg_status qg_gemm_w4a16(const void* X, qg_dtype xdt, int M, int K, int N, const uint32_t* packed,
                         const uint16_t* scales, const uint8_t* zeros, int group, void* Y,
@@ -134,9 +133,9 @@ qg_status qg_gemm_w4a16(const void* X, qg_dtype xdt, int M, int K, int N, const 
  * that loads the library, kept until the process exits; a shape whose scratch
  * would exceed it is refused with QG_ERR_WORKSPACE (see qg_last_error()).
  * The first call on each device looks the array's address up; make that first
- * call before any stream capture.  Each call clears the array's counters on
- * `stream` before its kernel.  All calls share the one array: calls that may
- * overlap on the GPU (other streams, other threads) race and must not be issued.
+ * call before any stream capture.  Nothing in the array needs to start at zero.
+ * All calls share the one array: calls that may overlap on the GPU (other
+ * streams, other threads) race and must not be issued.
  * ------------------------------------------------------------------------ */
 qg_status qg_gemm_w4a16_noalloc(const void* X, qg_dtype xdt, int M, int K, int N, const uint32_t* packed,
                                 const uint16_t* scales, const uint8_t* zeros, int group, void* Y,
