@@ -16,6 +16,7 @@
 #include "quantize.cuh"
 #include "tc_gemm.cuh"
 #include "w4a16_decode.cuh"
+#include "w4a16_tile.cuh"
 #include "w4a16_skinny.cuh"
 
 namespace {
@@ -363,24 +364,33 @@ qg_status tc_w4a8(const qg::TcInt8Args& a, qg_stream_t stream)
 
 qg_status tc_w4a16(const qg::TcW4A16Args& a, qg_stream_t stream)
 {
-    using C = qg::TcCfg<qg::TC_W4A16>;
-    CUtensorMap ta, tb;
+    using C = qg::W4TileCfg;
+    static_assert(C::TOTAL <= 227 * 1024, "W4A16 tile kernel shared memory");
+    CUtensorMap tx, tw;
     qg_status st;
-    if ((st = make_tmap_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.X, a.K, a.M, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B)))
+    if ((st = make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, a.X, a.K, a.M, C::BK, C::BT,
+                           CU_TENSOR_MAP_SWIZZLE_128B)))
         return st;
-    if ((st = make_tmap_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, a.N, a.K / 8, 128, 8,
+    if ((st = make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.packed, a.N, a.K / 8, C::BW, C::BK / 8,
                            CU_TENSOR_MAP_SWIZZLE_NONE)))
         return st;
-    qg::TcParams p{};
+    qg::W4TileParams p{};
     p.scales = a.scales;
     p.zeros = a.zeros;
     p.Y = a.Y;
     p.M = a.M;
     p.K = a.K;
     p.N = a.N;
-    p.m_tiles = (a.M + C::BM - 1) / C::BM;
-    p.n_tiles = (a.N + C::BN - 1) / C::BN;
-    return launch_tc<qg::TC_W4A16>(p, ta, tb, stream);
+    p.t_tiles = (a.M + C::BT - 1) / C::BT;
+    p.w_tiles = (a.N + C::BW - 1) / C::BW;
+    auto kern = qg::w4a16_tile_kernel;
+    static KernelInfo info;
+    int occ = 1;
+    if ((st = prepare_kernel(info, kern, C::THREADS, C::TOTAL, &occ)) != QG_OK) return st;
+    const int grid = std::min(p.t_tiles * p.w_tiles, num_sms());
+    kern<<<grid, C::THREADS, C::TOTAL, reinterpret_cast<cudaStream_t>(stream)>>>(p, tx, tw);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
 }
 
 // ---------------------------------------------------------------------------
