@@ -174,9 +174,24 @@ __global__ void __launch_bounds__(W4TileCfg::THREADS, 1)
                 uint32_t r[32];
                 tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + t0, r);
                 tmem_ld_wait();
-                if (n < p.N) {
+                const int nt = min(32, p.M - m0 - t0);
+                if ((p.N & 1) == 0) {
+                    // 2 x 2 transpose between lane pairs, then one 4-byte store of two
+                    // adjacent columns per lane: the even lane writes token t, the odd
+                    // lane token t + 1 (half the store instructions of 2-byte stores)
+                    const bool even = (lane & 1) == 0;
+                    const int c0 = even ? n : n - 1;
+#pragma unroll
+                    for (int t = 0; t < 32; t += 2) {
+                        const float a = __uint_as_float(r[t]), b = __uint_as_float(r[t + 1]);
+                        const float recv = __shfl_xor_sync(0xffffffffu, even ? b : a, 1);
+                        const int row = t + (even ? 0 : 1);
+                        const uint32_t v = even ? pack_bf16x2_rn(a, recv) : pack_bf16x2_rn(recv, b);
+                        if (row < nt && c0 + 1 < p.N)
+                            *reinterpret_cast<uint32_t*>(p.Y + (int64_t)(m0 + t0 + row) * p.N + c0) = v;
+                    }
+                } else if (n < p.N) {  // odd N: rows are not 4-byte aligned
                     uint16_t* y = p.Y + (int64_t)(m0 + t0) * p.N + n;
-                    const int nt = min(32, p.M - m0 - t0);
 #pragma unroll
                     for (int t = 0; t < 32; ++t)
                         if (t < nt) y[(int64_t)t * p.N] = f32_to_bf16_bits(__uint_as_float(r[t]));
