@@ -193,6 +193,29 @@ qg_status make_tmap_2d(CUtensorMap* m, CUtensorMapDataType dt, size_t elem_bytes
     return QG_OK;
 }
 
+// 3-D tiled map: dims {d0, d1, d2} with byte strides {stride1, stride2} for d1, d2.
+qg_status make_tmap_3d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, uint64_t d0, uint64_t d1,
+                       uint64_t d2, uint64_t stride1, uint64_t stride2, uint32_t b0, uint32_t b1, uint32_t b2,
+                       CUtensorMapSwizzle sw)
+{
+    auto enc = tmap_encoder();
+    if (!enc) {
+        snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled unavailable");
+        return QG_ERR_UNSUPPORTED;
+    }
+    cuuint64_t dims[3] = {d0, d1, d2};
+    cuuint64_t strides[2] = {stride1, stride2};
+    cuuint32_t box[3] = {b0, b1, b2};
+    cuuint32_t estr[3] = {1, 1, 1};
+    CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled (3-D) failed (%d)", (int)r);
+        return QG_ERR_CUDA;
+    }
+    return QG_OK;
+}
+
 // ---------------------------------------------------------------------------
 // W4A16 decode (stream-K, TMA-fed, workspace)
 // ---------------------------------------------------------------------------
@@ -250,17 +273,25 @@ qg_status launch_w4a16_decode(const qg::SkinnyParams& sp, const uint32_t* packed
     qg_status st = prepare_kernel(info, kern, L::THREADS, smem, &occ);
     if (st != QG_OK) return st;
     const DecodePlan d = decode_plan(sp.M, sp.K, sp.N);
-    CUtensorMap tw, ts, tz, tx;
-    if ((st = make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, sp.N, sp.K / 8, 32, 16,
-                           CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
-        return st;
-    if ((st = make_tmap_2d(&ts, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, scales, sp.N, d.G, 128, 1,
+    qg::DecodeMaps m;
+    const uint64_t N = sp.N, KW = sp.K / 8, G = d.G, K = sp.K;
+    if ((st = make_tmap_2d(&m.w4, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, N, KW, 32, 64,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK ||
+        (st = make_tmap_2d(&m.w1, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, N, KW, 32, 16,
+                           CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK ||
+        (st = make_tmap_2d(&m.s4, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, scales, N, G, 128, 4,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK ||
+        (st = make_tmap_2d(&m.s1, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, scales, N, G, 128, 1,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK ||
+        (st = make_tmap_2d(&m.z4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, zeros, N, G, 128, 4,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK ||
+        (st = make_tmap_2d(&m.z1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, zeros, N, G, 128, 1,
                            CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK)
         return st;
-    if ((st = make_tmap_2d(&tz, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, zeros, sp.N, d.G, 128, 1,
-                           CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK)
-        return st;
-    if ((st = make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, sp.X, sp.K, sp.M, 64, 8 * MT,
+    // X as {64 k, M rows, K / 64 halves}: row stride K * 2 bytes, half stride 128 bytes
+    if ((st = make_tmap_3d(&m.x4, CU_TENSOR_MAP_DATA_TYPE_UINT16, sp.X, 64, sp.M, K / 64, K * 2, 128, 64, 8 * MT,
+                           2 * qg::kDecGroupsPerStage, CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK ||
+        (st = make_tmap_3d(&m.x1, CU_TENSOR_MAP_DATA_TYPE_UINT16, sp.X, 64, sp.M, K / 64, K * 2, 128, 64, 8 * MT, 2,
                            CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
         return st;
     qg::DecodeParams p;
@@ -274,7 +305,7 @@ qg_status launch_w4a16_decode(const qg::SkinnyParams& sp, const uint32_t* packed
     p.nslabs = d.nslabs;
     p.units = d.units;
     p.grid = d.grid;
-    if ((st = launch_pdl(kern, dim3(d.grid), dim3(L::THREADS), smem, stream, p, tw, ts, tz, tx)) != QG_OK) return st;
+    if ((st = launch_pdl(kern, dim3(d.grid), dim3(L::THREADS), smem, stream, p, m)) != QG_OK) return st;
     return launch_pdl(qg::w4a16_decode_fixup_kernel<BF16>, dim3(d.nslabs), dim3(256), 0, stream, p, 8 * MT);
 }
 

@@ -57,6 +57,7 @@ struct DecodeParams {
 constexpr int kDecBN = 128;               // columns per slab
 constexpr int kDecGroupsPerStage = 4;
 constexpr int kDecGroupW = 16 * 128 * 4;  // packed words of one group: 16 rows x 128 columns x 4 B
+// (a stage holds them as [column block of 32][group][16 rows][128 B], 128-byte swizzled)
 constexpr int kDecScaleOff = 4 * kDecGroupW;
 constexpr int kDecZeroOff = kDecScaleOff + 4 * 256;
 constexpr int kDecXOff = kDecZeroOff + 4 * 128 + 512;  // 1 KB aligned
@@ -89,11 +90,23 @@ struct DecodeSmem {
     static constexpr int THREADS = 32 * NC + 128;
 };
 
+// Tensor maps.  A full stage (four groups of one slab) comes in four copies: the
+// packed words as four 32-column x 64-row boxes (128-byte swizzle), the scales and zeros
+// as 4-row boxes, and the activation tile as one 3-D box {64 k, MP rows, 8 halves}
+// that lands as [group][half][row][128 B].  A thread's bulk copies are issued one after
+// another at a cost of roughly a hundred cycles each, so few large copies keep the
+// producer ahead of the weight stream.  Stages of fewer groups (a piece's last) use
+// one-group boxes into the same layout.
+struct DecodeMaps {
+    CUtensorMap w4, w1;  // packed words: {32 columns, 64 | 16 rows}
+    CUtensorMap s4, s1;  // fp16 scales:  {128 columns, 4 | 1 groups}
+    CUtensorMap z4, z1;  // u8 zeros:     {128 columns, 4 | 1 groups}
+    CUtensorMap x4, x1;  // activations:  {64 k, MP rows, 8 | 2 halves}
+};
+
 template <int MT, bool BF16, int ST, int WS>
 __global__ void __launch_bounds__(DecodeSmem<MT, ST, WS>::THREADS, 1)
-    w4a16_decode_kernel(const DecodeParams p, const __grid_constant__ CUtensorMap tm_w,
-                        const __grid_constant__ CUtensorMap tm_s, const __grid_constant__ CUtensorMap tm_z,
-                        const __grid_constant__ CUtensorMap tm_x)
+    w4a16_decode_kernel(const DecodeParams p, const __grid_constant__ DecodeMaps maps)
 {
     using H = HalfOps<BF16>;
     using L = DecodeSmem<MT, ST, WS>;
@@ -127,32 +140,45 @@ __global__ void __launch_bounds__(DecodeSmem<MT, ST, WS>::THREADS, 1)
         if constexpr (WS == 1) asm volatile("setmaxnreg.dec.sync.aligned.u32 40;");   // 384 x 168 at launch
         else asm volatile("setmaxnreg.dec.sync.aligned.u32 24;");                    // 640 x 96 at launch
         if (warp == NC && lane == 0) {
-            tma_prefetch_desc(&tm_w);
-            tma_prefetch_desc(&tm_s);
-            tma_prefetch_desc(&tm_z);
-            tma_prefetch_desc(&tm_x);
+            tma_prefetch_desc(&maps.w4);
+            tma_prefetch_desc(&maps.s4);
+            tma_prefetch_desc(&maps.z4);
+            tma_prefetch_desc(&maps.x4);
+            // activation tiles of a stage: one 3-D box for four groups, else per group
+            auto load_x = [&](uint64_t* bar, uint8_t* st, int g0, int ng) {
+                if (ng == kDecGroupsPerStage)
+                    tma_load_3d(&maps.x4, bar, st + kDecXOff, 0, 0, 2 * g0);
+                else
+                    for (int i = 0; i < ng; ++i) tma_load_3d(&maps.x1, bar, st + kDecXOff + i * L::XG, 0, 0, 2 * (g0 + i));
+            };
             // Weights, scales and zeros do not depend on the previous grid: the first
             // ring-full of them is requested before waiting for it; X after.
             int stage = 0, issued = 0;
             uint32_t phase = 0;
-            bool waited = false;
+            bool waited = false, ok = true;
             int pend_g0[ST], pend_ng[ST];
-            for (int u = u0; u < u1;) {
+            for (int u = u0; u < u1 && ok;) {
                 const int slab = u / G, ga = u % G;
                 const int gb = min(G, ga + (u1 - u));
                 for (int g0 = ga; g0 < gb; g0 += kDecGroupsPerStage) {
                     const int ng = min(kDecGroupsPerStage, gb - g0);
-                    if (!mbar_wait(&empty[stage], phase ^ 1)) return;
+                    if (!mbar_wait(&empty[stage], phase ^ 1)) { ok = false; break; }
                     mbar_arrive_expect_tx(&full[stage], (uint32_t)ng * L::GROUP_TX);
                     uint8_t* st = ring + stage * L::STAGE;
-                    for (int i = 0; i < ng; ++i) {
-                        const int g = g0 + i;
+                    const int x = slab * kDecBN;
+                    if (ng == kDecGroupsPerStage) {
 #pragma unroll
-                        for (int b = 0; b < 4; ++b)
-                            tma_load_2d(&tm_w, &full[stage], st + i * kDecGroupW + b * 2048, slab * kDecBN + 32 * b,
-                                        16 * g);
-                        tma_load_2d(&tm_s, &full[stage], st + kDecScaleOff + i * 256, slab * kDecBN, g);
-                        tma_load_2d(&tm_z, &full[stage], st + kDecZeroOff + i * 128, slab * kDecBN, g);
+                        for (int b = 0; b < 4; ++b) tma_load_2d(&maps.w4, &full[stage], st + b * 4 * 2048, x + 32 * b, 16 * g0);
+                        tma_load_2d(&maps.s4, &full[stage], st + kDecScaleOff, x, g0);
+                        tma_load_2d(&maps.z4, &full[stage], st + kDecZeroOff, x, g0);
+                    } else {
+                        for (int i = 0; i < ng; ++i) {
+#pragma unroll
+                            for (int b = 0; b < 4; ++b)
+                                tma_load_2d(&maps.w1, &full[stage], st + b * 4 * 2048 + i * 2048, x + 32 * b, 16 * (g0 + i));
+                            tma_load_2d(&maps.s1, &full[stage], st + kDecScaleOff + i * 256, x, g0 + i);
+                            tma_load_2d(&maps.z1, &full[stage], st + kDecZeroOff + i * 128, x, g0 + i);
+                        }
                     }
                     if (!waited && issued < ST) {
                         pend_g0[issued] = g0;
@@ -162,26 +188,23 @@ __global__ void __launch_bounds__(DecodeSmem<MT, ST, WS>::THREADS, 1)
                         // ring full (or schedule done): now wait for the previous grid, then load X
                         asm volatile("griddepcontrol.wait;" ::: "memory");
                         waited = true;
-                        for (int j = 0; j <= issued; ++j) {
-                            uint8_t* sj = ring + j * L::STAGE;
-                            for (int i = 0; i < pend_ng[j]; ++i)
-#pragma unroll
-                                for (int b = 0; b < 2; ++b)
-                                    tma_load_2d(&tm_x, &full[j], sj + kDecXOff + i * L::XG + b * (L::XG / 2),
-                                                128 * (pend_g0[j] + i) + 64 * b, 0);
-                        }
+                        for (int j = 0; j <= issued; ++j) load_x(&full[j], ring + j * L::STAGE, pend_g0[j], pend_ng[j]);
                     } else if (waited) {
-                        for (int i = 0; i < ng; ++i)
-#pragma unroll
-                            for (int b = 0; b < 2; ++b)
-                                tma_load_2d(&tm_x, &full[stage], st + kDecXOff + i * L::XG + b * (L::XG / 2),
-                                            128 * (g0 + i) + 64 * b, 0);
+                        load_x(&full[stage], st, g0, ng);
                     }
                     ++issued;
                     if (++stage == ST) { stage = 0; phase ^= 1; }
                 }
                 u += gb - ga;
             }
+            if (!waited) {
+                // gave up inside the first ring-full: complete the stages requested so
+                // far, so that every copy in flight can land
+                asm volatile("griddepcontrol.wait;" ::: "memory");
+                for (int j = 0; j < issued; ++j) load_x(&full[j], ring + j * L::STAGE, pend_g0[j], pend_ng[j]);
+            }
+            // every copy still in flight lands before the CTA exits
+            for (int j = issued - ST > 0 ? issued - ST : 0; j < issued; ++j) mbar_wait(&full[j % ST], (j / ST) & 1);
         }
         return;
     }
@@ -246,7 +269,7 @@ __global__ void __launch_bounds__(DecodeSmem<MT, ST, WS>::THREADS, 1)
 #pragma unroll
                             for (int e = 0; e < 4; ++e) D[h][c][j][e] = 0.0f;
                 }
-                const uint8_t* wbase = st + wg * kDecGroupW;
+                const uint8_t* wbase = st + wg * 2048;  // column block b of group wg at b * 8 KB + wg * 2 KB
                 const uint8_t* xg = st + kDecXOff + wg * L::XG;
 #pragma unroll
                 for (int si = 0; si < SPW; ++si) {
@@ -255,7 +278,7 @@ __global__ void __launch_bounds__(DecodeSmem<MT, ST, WS>::THREADS, 1)
                     uint4 wv[2];
 #pragma unroll
                     for (int h = 0; h < 2; ++h)
-                        wv[h] = *reinterpret_cast<const uint4*>(wbase + (2 * wn + h) * 2048 + row * 128 +
+                        wv[h] = *reinterpret_cast<const uint4*>(wbase + (2 * wn + h) * 8192 + row * 128 +
                                                                 ((g8 ^ (row & 7)) << 4));
                     uint32_t xb[MT][4];
                     const uint8_t* xs = xg + (row >> 3) * (L::XG / 2);
