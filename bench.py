@@ -36,6 +36,12 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "quantized GEMM TFLOPS/TOPS and HBM GB/s (% of roofline) at M=1..8192"
+# DRAM bytes (read + write) of one decode launch over its algorithmic bytes, from an ncu
+# capture of one w4a16_decode_kernel launch at K=4096, N=22016, M=1 (47.237 MB read +
+# 0.016 MB written against 47.255 MB algorithmic; the weight stream is read exactly once,
+# so traffic scales with the algorithmic bytes of each call).  Take it again whenever the
+# decode kernel changes.
+DECODE_TRAFFIC_RATIO = (47.236608e6 + 15.616e3) / (4096 * 22016 // 2 + 4096 // 128 * 22016 * 3 + 2 * 4096 + 2 * 22016)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
@@ -187,7 +193,9 @@ class DecodeSweep:
         return sum(2 * c["M"] * sh["K"] * sh["N"] for sh, c in self.calls())
 
     def launches_per_step(self):
-        return sum(1 for _ in self.calls())
+        # every decode call is two kernels: w4a16_decode_kernel and its fixup (all sweep
+        # shapes have N % 16 == 0, the workspace path)
+        return 2 * sum(1 for _ in self.calls())
 
     def step(self, s):
         q = self.q
@@ -603,8 +611,9 @@ def main():
                        "l2": "weights rotate over copies totalling >= 2x L2 per shape (no L2 reuse across calls)",
                        "launch": "one CUDA graph per step (16 launches)"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / pk["hbm_gbs"], "traffic": None, "peak_source": pk["source"],
-                         "kernel": "w4a16_skinny_kernel (whole step)"},
+                         "frac": achieved / pk["hbm_gbs"], "traffic": by * DECODE_TRAFFIC_RATIO,
+                         "traffic_unit": "bytes per step", "peak_source": pk["source"],
+                         "kernel": "w4a16_decode_kernel + w4a16_decode_fixup_kernel, 16 calls per step"},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
             "gpu_launches": sweep.launches_per_step() * args.steps,

@@ -1,24 +1,22 @@
 // tc_gemm.cuh -- tcgen05 tile kernels for prefill-size M (tensor memory accumulators,
 // TMA-fed operands, warp-specialised, persistent).
 //
-// One template covers three products (KIND):
+// One template covers the two int8 products (KIND); the W4A16 tile kernel, which keeps
+// its dequantized weights in tensor memory, is in w4a16_tile.cuh.
 //   W8A8  acc = Xq Wq (int8 x int8 -> int32 in TMEM), Y = bf16((acc * t[m]) * sw[n])
 //         ("AI Infra guide, ch.4 Quantization" sec. 2.2-2.3, SmoothQuant)
-//   W4A16 Y = X (q - z) s with the dequantized bf16 weight tile built in shared memory
-//         by dequant warps ("AI Infra guide" sec. 3.1, 3.5; group-wise scale/zero:
-//         "LLM inference cost: W8A8/W4A8 ..." sec. 2.2)
 //   W4A8  P_g = Xq q4 per group of 128 (int32 in TMEM, ping-pong), Y = bf16(t[m] sum_g P_g s[g][n])
 //         ("LLM inference cost: W8A8/W4A8 ..." sec. 2.2)
 //
 // Roles (one CTA per SM, persistent over output tiles, n-tile-major order so that
 // concurrently running CTAs share the weight tile through L2):
 //   warp 0        TMA producer: activation tile and (W8A8) weight tile, or the packed
-//                 weight words (W4A16, W4A8), into a ring of shared-memory stages.
+//                 weight words (W4A8), into a ring of shared-memory stages.
 //   warp 1        TMEM allocator and MMA issuer (one elected lane issues tcgen05.mma
 //                 and tcgen05.commit; commits release ring stages and publish results).
 //   warps 4..     EPI epilogue warps: tcgen05.ld from TMEM, scale, convert, store; epilogue
 //                 warp e reads TMEM lanes 32(e%4)..+31 and the e/4-th share of the columns.
-//   then          DQ dequant warps (W4A16, W4A8): unpack nibbles from the raw stage and write
+//   then          DQ dequant warps (W4A8): unpack nibbles from the raw stage and write
 //                 the K-major, 128-byte-swizzled B tile the MMA reads; dequant thread d fills
 //                 B row d%128 and the (d/128)-th share of the k-block's words.
 // Waits on mbarriers are done by one lane per warp, then __syncwarp.
@@ -37,7 +35,7 @@ constexpr int kTcMinM = 128;
 // W4A8 below 128 tokens stays on the skinny kernel (measured faster at 64 tokens).
 constexpr int kTcMinMW4A8 = 128;
 
-enum TcKind { TC_W8A8 = 0, TC_W4A16 = 1, TC_W4A8 = 2 };
+enum TcKind { TC_W8A8 = 0, TC_W4A8 = 2 };
 
 struct TcW4A16Args {
     const uint16_t* X;
@@ -73,21 +71,6 @@ struct TcCfg<TC_W8A8> {
     static constexpr int EPI = 8, DQ = 0;  // epilogue / dequant warps
     static constexpr int THREADS = 32 * (4 + EPI + DQ);
     static constexpr int TMEM_COLS = 512;  // two 256-column accumulators
-    static constexpr int MH = 1;           // M=128 MMAs per tile
-};
-
-// W4A16: tile 256 x 128 (two M=128 MMAs share one dequantized B tile), k-block 64 bf16;
-// A 2 x 16 KB, raw packed words 8 x 128 x 4 B = 4 KB, B 128 x 64 bf16 = 16 KB per stage.
-template <>
-struct TcCfg<TC_W4A16> {
-    static constexpr int BM = 256, BN = 128, BK = 64;
-    static constexpr int A_BYTES = 2 * 128 * 128, RAW_BYTES = 8 * 128 * 4, B_BYTES = 128 * 128;
-    static constexpr int STAGE = A_BYTES + B_BYTES + 4096;  // raw area padded to 4 KB
-    static constexpr int ST = 4;
-    static constexpr int EPI = 8, DQ = 8;
-    static constexpr int THREADS = 32 * (4 + EPI + DQ);
-    static constexpr int TMEM_COLS = 512;  // two tiles x (2 halves x 128 columns)
-    static constexpr int MH = 2;
 };
 
 // W4A8: tile 128 x 128, k-block = one group of 128 int8; A 16 KB, raw 16 x 128 x 4 B = 8 KB,
@@ -102,7 +85,6 @@ struct TcCfg<TC_W4A8> {
     static constexpr int EPI = 8, DQ = 4;   // 8 epilogue warps: each owns 64 columns of a lane quarter
     static constexpr int THREADS = 32 * (4 + EPI + DQ);
     static constexpr int TMEM_COLS = 256;   // two group buffers (ping-pong) of 128 columns
-    static constexpr int MH = 1;
 };
 
 template <int KIND>
@@ -117,8 +99,6 @@ struct TcParams {
     const float* t;     // W8A8, W4A8: per-token scale
     const float* sw;    // W8A8: per-channel scale
     const float* sg;    // W4A8: per-group scale [K/128][N]
-    const uint16_t* scales;  // W4A16: fp16 [K/128][N]
-    const uint8_t* zeros;    // W4A16: u8 [K/128][N]
     uint16_t* Y;
     int32_t* dbg;
     int M, K, N;
@@ -219,11 +199,6 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
                         tma_load_2d(&tm_a, &full[s], st, kb * 128, m0);
                         tma_load_2d(&tm_b, &full[s], st + C::A_BYTES, n0, kb * 128);
                         tma_load_2d(&tm_b, &full[s], st + C::A_BYTES + 16384, n0 + 128, kb * 128);
-                    } else if constexpr (KIND == TC_W4A16) {
-                        mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::RAW_BYTES);
-                        tma_load_2d(&tm_a, &full[s], st, kb * 64, m0);
-                        tma_load_2d(&tm_a, &full[s], st + 16384, kb * 64, m0 + 128);
-                        tma_load_2d(&tm_b, &full[s], st + C::A_BYTES + C::B_BYTES, n0, kb * 8);
                     } else {
                         mbar_arrive_expect_tx(&full[s], C::A_BYTES + C::RAW_BYTES);
                         tma_load_2d(&tm_a, &full[s], st, kb * 128, m0);
@@ -264,29 +239,15 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
                     const int buf = li & 1;
                     if (!mbar_wait(&tempty[buf], ((li >> 1) & 1) ^ 1)) break;
                     tc_fence_after();
-                    for (int kb = 0; kb < KB; ++kb) {
-                        if constexpr (KIND == TC_W8A8) {
-                            if (!mbar_wait(&full[s], ph)) { ok = false; break; }
-                        } else {
-                            if (!mbar_wait(&bready[s], ph)) { ok = false; break; }
-                        }
+                    for (int kb = 0; kb < KB; ++kb) {  // W8A8
+                        if (!mbar_wait(&full[s], ph)) { ok = false; break; }
                         tc_fence_after();
                         const uint32_t a0 = smem_u32(smem + s * C::STAGE);
                         const uint32_t b0 = a0 + C::A_BYTES;
-                        if constexpr (KIND == TC_W8A8) {
 #pragma unroll
-                            for (int kk = 0; kk < 4; ++kk)
-                                mma_i8_ss(tmem + buf * 256, smem_desc(a0 + 32 * kk, 16, 1024, 2),
-                                          smem_desc(b0 + 4096 * kk, 16384, 1024, 2), idesc_s8(256, true),
-                                          (kb | kk) ? 1u : 0u);
-                        } else {
-#pragma unroll
-                            for (int h = 0; h < 2; ++h)
-#pragma unroll
-                                for (int kk = 0; kk < 4; ++kk)
-                                    mma_f16_ss(tmem + buf * 256 + h * 128, smem_desc(a0 + h * 16384 + 32 * kk, 16, 1024, 2),
-                                               smem_desc(b0 + 32 * kk, 16, 1024, 2), idesc_bf16(128), (kb | kk) ? 1u : 0u);
-                        }
+                        for (int kk = 0; kk < 4; ++kk)
+                            mma_i8_ss(tmem + buf * 256, smem_desc(a0 + 32 * kk, 16, 1024, 2),
+                                      smem_desc(b0 + 4096 * kk, 16384, 1024, 2), idesc_s8(256, true), (kb | kk) ? 1u : 0u);
                         mma_commit(&empty[s]);
                         if (++s == C::ST) { s = 0; ph ^= 1; }
                     }
@@ -389,47 +350,37 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
                 const int buf = li & 1;
                 if (!warp_wait(&tfull[buf], (li >> 1) & 1)) break;
                 tc_fence_after();
-                constexpr int NCH = (KIND == TC_W8A8 ? 8 : 4) / CSPLIT;  // 32-column chunks per warp
+                constexpr int NCH = 8 / CSPLIT;  // W8A8: 32-column chunks per warp
+                const int m = m0 + 32 * q + lane;
+                const float tm = m < p.M ? __ldg(p.t + m) : 0.0f;
 #pragma unroll 1
-                for (int h = 0; h < C::MH; ++h) {
-                    const int m = m0 + h * 128 + 32 * q + lane;
-                    const float tm = (KIND == TC_W8A8 && m < p.M) ? __ldg(p.t + m) : 0.0f;
-#pragma unroll 1
-                    for (int c = cs * NCH; c < (cs + 1) * NCH; ++c) {
-                        uint32_t r[32];
-                        const uint32_t col = (KIND == TC_W8A8 ? buf * 256 : buf * 256 + h * 128) + 32 * c;
-                        tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + col, r);
-                        tmem_ld_wait();
-                        const int nb = n0 + 32 * c;
-                        if (m < p.M) {
-                            uint16_t* yrow = p.Y + (int64_t)m * p.N + nb;
+                for (int c = cs * NCH; c < (cs + 1) * NCH; ++c) {
+                    uint32_t r[32];
+                    tmem_ld_32x32b_x32(tmem + ((uint32_t)(32 * q) << 16) + buf * 256 + 32 * c, r);
+                    tmem_ld_wait();
+                    const int nb = n0 + 32 * c;
+                    if (m < p.M) {
+                        uint16_t* yrow = p.Y + (int64_t)m * p.N + nb;
 #pragma unroll
-                            for (int i = 0; i < 32; i += 8) {
-                                if (nb + i >= p.N) continue;
-                                float f[8];
-                                if constexpr (KIND == TC_W8A8) {
-                                    const float4 s0 = __ldg(reinterpret_cast<const float4*>(p.sw + nb + i));
-                                    const float4 s1 = __ldg(reinterpret_cast<const float4*>(p.sw + nb + i + 4));
-                                    const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+                        for (int i = 0; i < 32; i += 8) {
+                            if (nb + i >= p.N) continue;
+                            const float4 s0 = __ldg(reinterpret_cast<const float4*>(p.sw + nb + i));
+                            const float4 s1 = __ldg(reinterpret_cast<const float4*>(p.sw + nb + i + 4));
+                            const float sv[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+                            float f[8];
 #pragma unroll
-                                    for (int e = 0; e < 8; ++e)
-                                        f[e] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[i + e]), tm), sv[e]);
-                                    if (p.dbg) {
-                                        int32_t* d = p.dbg + (int64_t)m * p.N + nb + i;
-                                        *reinterpret_cast<int4*>(d) = make_int4(r[i], r[i + 1], r[i + 2], r[i + 3]);
-                                        *reinterpret_cast<int4*>(d + 4) = make_int4(r[i + 4], r[i + 5], r[i + 6], r[i + 7]);
-                                    }
-                                } else {
-#pragma unroll
-                                    for (int e = 0; e < 8; ++e) f[e] = __uint_as_float(r[i + e]);
-                                }
-                                uint4 v;
-                                v.x = pack_bf16x2_rn(f[0], f[1]);
-                                v.y = pack_bf16x2_rn(f[2], f[3]);
-                                v.z = pack_bf16x2_rn(f[4], f[5]);
-                                v.w = pack_bf16x2_rn(f[6], f[7]);
-                                *reinterpret_cast<uint4*>(yrow + i) = v;
+                            for (int e = 0; e < 8; ++e) f[e] = __fmul_rn(__fmul_rn(__int2float_rn((int)r[i + e]), tm), sv[e]);
+                            if (p.dbg) {
+                                int32_t* d = p.dbg + (int64_t)m * p.N + nb + i;
+                                *reinterpret_cast<int4*>(d) = make_int4(r[i], r[i + 1], r[i + 2], r[i + 3]);
+                                *reinterpret_cast<int4*>(d + 4) = make_int4(r[i + 4], r[i + 5], r[i + 6], r[i + 7]);
                             }
+                            uint4 v;
+                            v.x = pack_bf16x2_rn(f[0], f[1]);
+                            v.y = pack_bf16x2_rn(f[2], f[3]);
+                            v.z = pack_bf16x2_rn(f[4], f[5]);
+                            v.w = pack_bf16x2_rn(f[6], f[7]);
+                            *reinterpret_cast<uint4*>(yrow + i) = v;
                         }
                     }
                 }
@@ -439,69 +390,22 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
             }
         }
     } else {
-        // ------------------------------ dequant warps (W4A16, W4A8) ------------------------------
-        if constexpr (KIND != TC_W8A8) {
+        // ------------------------------ dequant warps (W4A8) ------------------------------
+        if constexpr (KIND == TC_W4A8) {
             const int dthr = threadIdx.x - 32 * (4 + C::EPI);
             const int dt = dthr & 127;                 // the B tile row (column n) this thread fills
             constexpr int WSPLIT = C::DQ / 4;           // threads sharing one B row
             const int ws = dthr >> 7;                   // this thread's share of the k-block's words
             int s = 0;
             uint32_t ph = 0;
-            for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
-                const int n0 = (tile / p.m_tiles) * C::BN;
-                const int n = n0 + dt;
-                // W4A16: per-column scale and zero, fetched one group ahead of their use
-                uint16_t s_cur = 0, s_nxt = 0;
-                uint8_t z_cur = 0, z_nxt = 0;
-                if constexpr (KIND == TC_W4A16) {
-                    if (n < p.N) {
-                        s_cur = __ldg(p.scales + n);
-                        z_cur = __ldg(p.zeros + n);
-                        if (KB > 2) {
-                            s_nxt = __ldg(p.scales + (int64_t)p.N + n);
-                            z_nxt = __ldg(p.zeros + (int64_t)p.N + n);
-                        }
-                    }
-                }
+            bool ok = true;
+            for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
                 for (int kb = 0; kb < KB; ++kb) {
-                    float sv = 0.0f, zv = 0.0f;
-                    if constexpr (KIND == TC_W4A16) {
-                        if (kb > 0 && (kb & 1) == 0) {  // a new group starts: rotate and prefetch the next
-                            s_cur = s_nxt;
-                            z_cur = z_nxt;
-                            const int gn = (kb >> 1) + 1;
-                            if (n < p.N && 2 * gn < KB) {
-                                s_nxt = __ldg(p.scales + (int64_t)gn * p.N + n);
-                                z_nxt = __ldg(p.zeros + (int64_t)gn * p.N + n);
-                            }
-                        }
-                        sv = __half2float(__ushort_as_half(s_cur));
-                        zv = (float)z_cur;
-                    }
-                    if (!warp_wait(&full[s], ph)) goto dequant_done;
+                    if (!warp_wait(&full[s], ph)) { ok = false; break; }
                     uint8_t* st = smem + s * C::STAGE;
                     const uint32_t* raw = reinterpret_cast<const uint32_t*>(st + C::A_BYTES + C::B_BYTES);
                     uint8_t* brow = st + C::A_BYTES + dt * 128;  // row dt of the K-major B tile
-                    if constexpr (KIND == TC_W4A16) {
-                        // k-block of 64 = 8 words of column n, all in group kb / 2
-                        const uint32_t s2 = pack_bf16x2_rn(sv, sv);
-                        const uint32_t z2 = pack_bf16x2_rn(128.0f + zv, 128.0f + zv);
-#pragma unroll
-                        for (int wi = 0; wi < 8 / WSPLIT; ++wi) {
-                            const int w = ws * (8 / WSPLIT) + wi;
-                            const uint32_t word = raw[w * 128 + dt];
-                            uint32_t R[4];
-#pragma unroll
-                            for (int r = 0; r < 4; ++r)
-                                R[r] = bf16x2_mul(bf16x2_sub(lop3_and_or(word >> (4 * r), 0x000F000Fu, 0x43004300u), z2), s2);
-                            uint4 v;  // natural k order: (0,1) (2,3) (4,5) (6,7)
-                            v.x = prmt(R[0], R[1], 0x5410);
-                            v.y = prmt(R[2], R[3], 0x5410);
-                            v.z = prmt(R[0], R[1], 0x7632);
-                            v.w = prmt(R[2], R[3], 0x7632);
-                            *reinterpret_cast<uint4*>(brow + ((w ^ (dt & 7)) << 4)) = v;
-                        }
-                    } else {
+                    {
                         // one group of 128 k = 16 words; two words per 16-byte chunk
 #pragma unroll
                         for (int ci = 0; ci < 8 / WSPLIT; ++ci) {
@@ -528,7 +432,6 @@ __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
                 }
             }
         }
-    dequant_done:;
     }
 
     tc_fence_before();

@@ -15,10 +15,10 @@
 // `w4a16_decode_fixup_kernel` sums the pieces of every split slab in CTA order
 // (deterministic; no atomics, no counters) and writes Y.
 //
-// Data movement.  One producer thread streams each group's packed words (16 rows of
-// the [K/8][N] matrix x 128 columns, as four 128-byte-wide boxes with 128-byte
-// swizzle), fp16 scales, u8 zeros and the group's activation tile into a ring of
-// shared-memory stages with TMA; a stage holds up to four groups of one slab.
+// Data movement.  One producer thread streams the packed words (16 rows of the [K/8][N]
+// matrix x 128 columns per group, 128-byte swizzled), fp16 scales, u8 zeros and the
+// activation tiles into a ring of shared-memory stages with TMA; a stage holds up to
+// four groups of one slab and, when full, arrives in four bulk copies (DecodeMaps).
 // Consumer warp (wn, wg, ws) takes columns 64wn..64wn+63 of group wg of each stage and
 // the ws-th share of its four 32-k steps (WS = 1 or 2 warps per group).
 //
