@@ -169,10 +169,11 @@ def qg_smooth_quant_act_i8(X, inv_s, Xq, t, stream=None):
            "qg_smooth_quant_act_i8")
 
 
-def qg_gemm_w8a8(Xq, t, Wq, sw, Y, acc_dbg=None, stream=None):
+def qg_gemm_w8a8(Xq, t, Wq, sw, Y, acc_dbg=None, workspace="auto", stream=None):
     M, K = Xq.shape
     N = Wq.shape[1]
-    _check(lib().qg_gemm_w8a8(_ptr(Xq), _ptr(t), M, K, _ptr(Wq), _ptr(sw), N, _ptr(Y), _ptr(acc_dbg), None, 0,
+    wp, wb = _ws(workspace, QG_OP_GEMM_W8A8, M, K, N, Xq.device)
+    _check(lib().qg_gemm_w8a8(_ptr(Xq), _ptr(t), M, K, _ptr(Wq), _ptr(sw), N, _ptr(Y), _ptr(acc_dbg), wp, wb,
                              _stream(stream)), "qg_gemm_w8a8")
 
 

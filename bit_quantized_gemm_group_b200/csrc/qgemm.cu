@@ -17,6 +17,7 @@
 #include "tc_gemm.cuh"
 #include "w4a16_decode.cuh"
 #include "w4a16_tile.cuh"
+#include "int8_decode.cuh"
 #include "w4a16_skinny.cuh"
 
 namespace {
@@ -425,6 +426,47 @@ qg_status tc_w4a16(const qg::TcW4A16Args& a, qg_stream_t stream)
 }
 
 // ---------------------------------------------------------------------------
+// W8A8 decode (M < kTcMinM, stream-K on tcgen05, workspace)
+// ---------------------------------------------------------------------------
+struct I8Plan {
+    int NT, KB, nslabs, units, grid;
+    size_t partial_bytes;
+};
+
+I8Plan i8_plan(int M, int K, int N)
+{
+    I8Plan d;
+    d.NT = M <= 16 ? 16 : M <= 32 ? 32 : M <= 64 ? 64 : 128;
+    d.KB = K / 128;
+    d.nslabs = (N + 127) / 128;
+    d.units = d.KB * d.nslabs;
+    d.grid = std::min(std::min(num_sms(), d.units), 160);
+    d.partial_bytes = (size_t)d.grid * 2 * 128 * d.NT * sizeof(int32_t);
+    return d;
+}
+
+template <int NT>
+qg_status launch_w8a8_decode(const int8_t* Xq, const float* t, int M, int K, const int8_t* Wq, const float* sw,
+                             int N, uint16_t* Y, int32_t* acc_dbg, void* ws, qg_stream_t stream)
+{
+    using C = qg::I8DecCfg<NT>;
+    static_assert(C::TOTAL <= 227 * 1024, "W8A8 decode kernel shared memory");
+    auto kern = qg::w8a8_decode_kernel<NT>;
+    static KernelInfo info;
+    int occ = 1;
+    qg_status st = prepare_kernel(info, kern, C::THREADS, C::TOTAL, &occ);
+    if (st != QG_OK) return st;
+    const I8Plan d = i8_plan(M, K, N);
+    CUtensorMap tw, tx;
+    if ((st = make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Wq, N, K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)) ||
+        (st = make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Xq, K, M, 128, NT, CU_TENSOR_MAP_SWIZZLE_128B)))
+        return st;
+    qg::I8DecodeParams p{t, sw, Y, acc_dbg, static_cast<int32_t*>(ws), M, K, N, d.KB, d.nslabs, d.units, d.grid};
+    if ((st = launch_pdl(kern, dim3(d.grid), dim3(C::THREADS), C::TOTAL, stream, p, tw, tx)) != QG_OK) return st;
+    return launch_pdl(qg::w8a8_decode_fixup_kernel, dim3(d.nslabs), dim3(256), 0, stream, p, NT);
+}
+
+// ---------------------------------------------------------------------------
 // int8 skinny paths
 // ---------------------------------------------------------------------------
 template <int MT>
@@ -493,6 +535,10 @@ size_t qg_workspace_size(qg_op op, int M, int K, int N)
         case QG_OP_GEMM_W4A16: {
             if (!decode_eligible(M, N)) return 0;
             return decode_plan(M, K, N).partial_bytes;
+        }
+        case QG_OP_GEMM_W8A8: {
+            if (M >= qg::kTcMinM || N % 16) return 0;
+            return i8_plan(M, K, N).partial_bytes;
         }
         default: return 0;
     }
@@ -577,16 +623,23 @@ qg_status qg_smooth_quant_act_i8(const uint16_t* X, int M, int K, const float* i
 qg_status qg_gemm_w8a8(const int8_t* Xq, const float* t, int M, int K, const int8_t* Wq, const float* sw, int N,
                        uint16_t* Y, int32_t* acc_dbg, void* workspace, size_t ws_bytes, qg_stream_t stream)
 {
-    (void)workspace;
-    (void)ws_bytes;
     if (M < 0 || K < 128 || N < 16 || K % 128 || N % 16) return QG_ERR_SHAPE;
     if (M == 0) return QG_OK;
     if (!Xq || !t || !Wq || !sw || !Y) return QG_ERR_NULL;
-    if (misaligned(Xq) || misaligned(t) || misaligned(Wq) || misaligned(sw) || misaligned(Y) || misaligned(acc_dbg))
+    if (misaligned(Xq) || misaligned(t) || misaligned(Wq) || misaligned(sw) || misaligned(Y) || misaligned(acc_dbg) ||
+        misaligned(workspace))
         return QG_ERR_ALIGN;
     if (M >= qg::kTcMinM) {
         qg::TcInt8Args a{Xq, t, Wq, sw, nullptr, nullptr, Y, acc_dbg, M, K, N};
         return tc_w8a8(a, stream);
+    }
+    if (workspace) {
+        if (ws_bytes < qg_workspace_size(QG_OP_GEMM_W8A8, M, K, N)) return QG_ERR_WORKSPACE;
+        const int nt = i8_plan(M, K, N).NT;
+        return nt == 16   ? launch_w8a8_decode<16>(Xq, t, M, K, Wq, sw, N, Y, acc_dbg, workspace, stream)
+               : nt == 32 ? launch_w8a8_decode<32>(Xq, t, M, K, Wq, sw, N, Y, acc_dbg, workspace, stream)
+               : nt == 64 ? launch_w8a8_decode<64>(Xq, t, M, K, Wq, sw, N, Y, acc_dbg, workspace, stream)
+                          : launch_w8a8_decode<128>(Xq, t, M, K, Wq, sw, N, Y, acc_dbg, workspace, stream);
     }
     for (int m0 = 0; m0 < M; m0 += 16) {
         qg::Int8SkinnyParams p{Xq + (int64_t)m0 * K, t + m0, Wq, sw, nullptr, nullptr, Y + (int64_t)m0 * N,

@@ -164,7 +164,13 @@ qg_status qg_smooth_quant_act_i8(const uint16_t* X, int M, int K, const float* i
  * Xq int8 [M][K], t fp32 [M] (from qg_smooth_quant_act_i8); Wq int8 [K][N],
  * sw fp32 [N] (from qg_quantize_w8_channel); Y bf16 [M][N].
  * acc_dbg: NULL, or int32 [M][N] that also receives the exact accumulators.
- * Rules: K % 128 == 0, N % 16 == 0.  workspace / ws_bytes unused (NULL, 0).
+ * Rules: K % 128 == 0, N % 16 == 0.
+ * workspace: NULL, or (M < 128) a device buffer of at least
+ *   qg_workspace_size(QG_OP_GEMM_W8A8, M, K, N) bytes (contents irrelevant; it holds
+ *   the int32 partial sums of column slabs split between CTAs).  With it, M < 128 runs
+ *   the stream-K tensor-core kernel; without it, the cluster split-K kernel.  Both give
+ *   the same bits.  A workspace smaller than required -> QG_ERR_WORKSPACE before any
+ *   launch.  Calls that may run concurrently need workspaces of their own.
  * ------------------------------------------------------------------------ */
 qg_status qg_gemm_w8a8(const int8_t* Xq, const float* t, int M, int K, const int8_t* Wq,
                        const float* sw, int N, uint16_t* Y, int32_t* acc_dbg, void* workspace,

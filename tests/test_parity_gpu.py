@@ -212,15 +212,18 @@ def w8a8_weights():
     return K, N, inv_o, Wq_o, sw_o
 
 
-@pytest.mark.parametrize("M", [16, 256, 2048, 1, 3, 17])
-def test_gemm_w8a8_bitexact(M, w8a8_weights):
+@pytest.mark.parametrize("M,workspace", [(16, "auto"), (256, "auto"), (2048, "auto"), (1, "auto"), (3, "auto"),
+                                         (17, "auto"), (16, None), (1, None), (17, None)])
+def test_gemm_w8a8_bitexact(M, workspace, w8a8_weights):
+    """Below 128 tokens the stream-K kernel (workspace) and the cluster split-K kernel
+    (no workspace) both give the oracle's bits."""
     K, N, inv_o, Wq_o, sw_o = w8a8_weights
     X, Xb = synth.workload_activations("w8a8", M, K)
     Xq_o, t_o, _ = oracle.smooth_quant_act_i8(X, inv_o)
     q = qlib()
     Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
     acc = torch.empty(M, N, dtype=torch.int32, device="cuda")
-    q.qg_gemm_w8a8(cuda(Xq_o), cuda(t_o), cuda(Wq_o), cuda(sw_o), Y, acc)
+    q.qg_gemm_w8a8(cuda(Xq_o), cuda(t_o), cuda(Wq_o), cuda(sw_o), Y, acc, workspace=workspace)
     _status_ok()
     rows = sample_rows(M) if M > 256 else None
     acc_o, y_o, yref, b = oracle.gemm_w8a8(Xq_o, t_o, Wq_o, sw_o, rows=rows)
@@ -233,8 +236,30 @@ def test_gemm_w8a8_bitexact(M, w8a8_weights):
     assert_tol(bf16_to_f32(y), yref, b)
     # without the debug output the result is the same
     Y2 = torch.empty_like(Y)
-    q.qg_gemm_w8a8(cuda(Xq_o), cuda(t_o), cuda(Wq_o), cuda(sw_o), Y2, None)
+    q.qg_gemm_w8a8(cuda(Xq_o), cuda(t_o), cuda(Wq_o), cuda(sw_o), Y2, None, workspace=workspace)
     assert torch.equal(Y2.view(torch.int16), Y.view(torch.int16))
+
+
+@pytest.mark.parametrize("K,N", [(512, 144), (1024, 272), (128, 16), (2048, 1296)])
+def test_gemm_w8a8_stream_k_edges(K, N):
+    """The stream-K kernel across every token tile (16, 32, 64, 128 tokens) and its
+    boundaries, on ragged column slabs, one-block K and slabs split between CTAs; the
+    workspace starts with garbage (its contents must not matter)."""
+    rng = np.random.default_rng(K + N)
+    q = qlib()
+    ws = torch.full((q.qg_workspace_size(q.QG_OP_GEMM_W8A8, 127, K, N),), 0x5A, dtype=torch.uint8, device="cuda")
+    for M in [1, 2, 15, 16, 17, 31, 32, 33, 63, 64, 65, 100, 127]:
+        Xq = rng.integers(-127, 128, (M, K)).astype(np.int8)
+        Wq = rng.integers(-127, 128, (K, N)).astype(np.int8)
+        t = rng.uniform(0.01, 1.0, M).astype(np.float32)
+        sw = rng.uniform(0.001, 0.01, N).astype(np.float32)
+        Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        acc = torch.full((M, N), -1, dtype=torch.int32, device="cuda")
+        q.qg_gemm_w8a8(cuda(Xq), cuda(t), cuda(Wq), cuda(sw), Y, acc, workspace=ws)
+        _status_ok()
+        acc_o, y_o, _, _ = oracle.gemm_w8a8(Xq, t, Wq, sw)
+        np.testing.assert_array_equal(acc.cpu().numpy(), acc_o, err_msg=f"M={M}")
+        np.testing.assert_array_equal(u16(Y), y_o, err_msg=f"M={M}")
 
 
 # ---------------------------------------------------------------------------
