@@ -36,6 +36,12 @@ sys.path.insert(0, ROOT)
 import synth  # noqa: E402
 
 METRIC = "quantized GEMM TFLOPS/TOPS and HBM GB/s (% of roofline) at M=1..8192"
+# the workload both arms report on (the reference arm times a bounded sample of it and
+# says which in its cpu_baseline.sample)
+CONFIG = {"workload": "w4a16_decode: M in {1,4,16,32} x (K,N) in {(4096,12288),(4096,4096),"
+                      "(4096,22016),(11008,4096)}, group-128 asym INT4, bf16 X/Y",
+          "l2": "weights rotate over copies totalling >= 2x L2 per shape (no L2 reuse across calls)",
+          "launch": "one CUDA graph per step (16 calls, each a decode and a fixup kernel)"}
 # DRAM bytes (read + write) of one decode launch over its algorithmic bytes, from an ncu
 # capture of one w4a16_decode_kernel launch at K=4096, N=22016, M=1 (47.237 MB read +
 # 0.016 MB written against 47.255 MB algorithmic; the weight stream is read exactly once,
@@ -332,7 +338,7 @@ def run_reference(args, world, rank):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total / len(times) * 1e3,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": "w4a16_decode sample: 16 calls on 1/8 of the columns"},
+            "config": dict(CONFIG),
             "cpu_baseline": {"value": value, "unit": "GB/s", "kind": "oracle", "cores": cb["cores"],
                              "sample": cb["sample"]},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
@@ -606,10 +612,7 @@ def main():
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "w4a16_decode: M in {1,4,16,32} x (K,N) in {(4096,12288),(4096,4096),"
-                                   "(4096,22016),(11008,4096)}, group-128 asym INT4, bf16 X/Y",
-                       "l2": "weights rotate over copies totalling >= 2x L2 per shape (no L2 reuse across calls)",
-                       "launch": "one CUDA graph per step (16 launches)"},
+            "config": dict(CONFIG),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "traffic": by * DECODE_TRAFFIC_RATIO,
                          "traffic_unit": "bytes per step", "peak_source": pk["source"],
