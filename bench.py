@@ -11,7 +11,11 @@ bf16 X + bf16 Y per call.  Weight buffers rotate over enough copies that every
 call reads its weights from HBM, not L2.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload w4a16_decode|w8a8|w4a16_prefill|w4a8|w4a16_tiny]
+                    [--no-cpu-baseline] [--skip-configs] [--profile]
+    python bench.py --single K,N,M [--op w4a16|w8a8|w4a8] [--reps R]   (one call shape)
+
+Besides the headline sweep, rank 0 times the other workloads (W4A16 tiny, W8A8, W4A16
+prefill, W4A8) and reports them under "configs".
 
 Under torchrun every rank runs the same workload on its own GPU (replicas, weak
 scaling); timing is the max over ranks of CUDA-event time; rank 0 prints one JSON line.
@@ -117,7 +121,9 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # distributed plumbing
 # ---------------------------------------------------------------------------
-def dist_setup(n_gpus):
+def dist_setup(n_gpus, backend="nccl"):
+    """One process per GPU (replicas): rank and world from the launcher's environment.
+    backend "gloo" (CPU, no device selection) serves the host-side tests."""
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -125,9 +131,10 @@ def dist_setup(n_gpus):
         import datetime
 
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
-    else:
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif backend == "nccl":
         torch.cuda.set_device(0)
     return world, rank, local
 
@@ -138,13 +145,19 @@ def barrier(world):
         dist.barrier()
 
 
-def max_over_ranks(x, world):
+def max_over_ranks(x, world, device="cuda"):
     if world == 1:
         return x
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_gbs(bytes_per_step, world, steps, ms_max):
+    """Whole-job throughput of the replicas: every rank processes one step's bytes per
+    step; the time is the slowest rank's (weak scaling)."""
+    return bytes_per_step * world * steps / (ms_max * 1e-3) / 1e9
 
 
 # ---------------------------------------------------------------------------
@@ -551,7 +564,6 @@ def main():
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="w4a16_decode")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--skip-configs", action="store_true", help="only the headline decode sweep")
     ap.add_argument("--single", default=None, help="K,N,M: time one decode call shape alone (profiling aid)")
@@ -586,7 +598,7 @@ def main():
     ms = max_over_ranks(ms, world)
     ms_step = ms / args.steps
     by = sweep.bytes_per_step()
-    value = by * world * args.steps / (ms * 1e-3) / 1e9
+    value = whole_job_gbs(by, world, args.steps, ms)
     achieved = by / (ms_step * 1e-3) / 1e9
 
     if args.profile:
@@ -594,7 +606,7 @@ def main():
             print(json.dumps({"profile_run": True, "ms_per_step": ms_step, "gbs": achieved}), flush=True)
         return
     e2e_ms, h2d, d2h = e2e_decode(sweep, args.steps, args.warmup, world)
-    e2e_val = by * world * args.steps / (e2e_ms * 1e-3) / 1e9
+    e2e_val = whole_job_gbs(by, world, args.steps, e2e_ms)
     calls = per_call_times(sweep) if rank == 0 else []
 
     cpu = None
