@@ -532,11 +532,11 @@ def run_single(spec, reps, workspace="auto", op="w4a16"):
             Wq = torch.empty(K, N, dtype=torch.int8, device="cuda")
             sw = torch.empty(N, dtype=torch.float32, device="cuda")
             q.qg_quantize_w8_channel(W, None, Wq, sw)
-            call = lambda: q.qg_gemm_w8a8(Xq, t, Wq, sw, Y)  # noqa: E731
+            call = lambda: q.qg_gemm_w8a8(Xq, t, Wq, sw, Y, workspace=workspace)  # noqa: E731
             by = K * N + 4 * N + M * K + 4 * M + 2 * M * N
         else:
             packed, sg, _ = gpu_quant_w4(q, W, None, sym=True)
-            call = lambda: q.qg_gemm_w4a8(Xq, t, packed, sg, Y)  # noqa: E731
+            call = lambda: q.qg_gemm_w4a8(Xq, t, packed, sg, Y, workspace=workspace)  # noqa: E731
             by = K * N // 2 + 4 * (K // 128) * N + M * K + 4 * M + 2 * M * N
     del W
     flush = torch.empty(2 * l2_bytes(), dtype=torch.uint8, device="cuda")

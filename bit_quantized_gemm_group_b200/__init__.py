@@ -177,11 +177,12 @@ def qg_gemm_w8a8(Xq, t, Wq, sw, Y, acc_dbg=None, workspace="auto", stream=None):
                              _stream(stream)), "qg_gemm_w8a8")
 
 
-def qg_gemm_w4a8(Xq, t, packed, sg, Y, part_dbg=None, group=128, stream=None):
+def qg_gemm_w4a8(Xq, t, packed, sg, Y, part_dbg=None, group=128, workspace="auto", stream=None):
     M, K = Xq.shape
     N = packed.shape[1]
-    _check(lib().qg_gemm_w4a8(_ptr(Xq), _ptr(t), M, K, _ptr(packed), _ptr(sg), N, group, _ptr(Y), _ptr(part_dbg), None,
-                             0, _stream(stream)), "qg_gemm_w4a8")
+    wp, wb = _ws(workspace, QG_OP_GEMM_W4A8, M, K, N, Xq.device)
+    _check(lib().qg_gemm_w4a8(_ptr(Xq), _ptr(t), M, K, _ptr(packed), _ptr(sg), N, group, _ptr(Y), _ptr(part_dbg), wp,
+                             wb, _stream(stream)), "qg_gemm_w4a8")
 
 
 def qg_smooth_scales(Xcal, W, alpha, s, inv_s, stream=None):

@@ -273,6 +273,17 @@ QG_DEV_INLINE void mma_i8_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, 
         : "memory");
 }
 
+// kind::i8 with A (M x K, int8) read from tensor memory: four consecutive k per 32-bit column
+QG_DEV_INLINE void mma_i8_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t accum)
+{
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accum)
+        : "memory");
+}
+
 // Arrive on `bar` once every tcgen05 operation issued so far by this thread has completed.
 QG_DEV_INLINE void mma_commit(uint64_t* bar)
 {
@@ -301,6 +312,25 @@ QG_DEV_INLINE void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16])
         : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
           "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
         : "r"(taddr));
+}
+
+// 4-byte global -> shared copy that bypasses registers (zero-filled when !valid)
+QG_DEV_INLINE void cp_async_4(void* dst_smem, const void* src, bool valid)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst_smem)), "l"(src),
+                 "r"(valid ? 4 : 0)
+                 : "memory");
+}
+QG_DEV_INLINE void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+QG_DEV_INLINE void cp_async_wait_group() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+// 32 lanes x 1 32-bit column -> 1 register per thread
+QG_DEV_INLINE uint32_t tmem_ld_32x32b_x1(uint32_t taddr)
+{
+    uint32_t r;
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr));
+    return r;
 }
 
 QG_DEV_INLINE void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }

@@ -18,6 +18,7 @@
 #include "w4a16_decode.cuh"
 #include "w4a16_tile.cuh"
 #include "int8_decode.cuh"
+#include "w4a8_decode.cuh"
 #include "w4a16_skinny.cuh"
 
 namespace {
@@ -466,6 +467,48 @@ qg_status launch_w8a8_decode(const int8_t* Xq, const float* t, int M, int K, con
     return launch_pdl(qg::w8a8_decode_fixup_kernel, dim3(d.nslabs), dim3(256), 0, stream, p, NT);
 }
 
+// W4A8 stream-K (17 <= M < 128; M <= 64 per launch, larger M in chunks of 64 tokens).
+// At 16 tokens and fewer the cluster split-K kernel is as fast or faster (measured at
+// K = N = 8192: 16.4 vs 25.6 us at M = 1, 24.6 vs 25.6 us at M = 16).
+constexpr int kW4A8DecodeMinM = 17;
+constexpr int kW4A8DecodeMaxM = 64;
+constexpr int kW4A8Issuers = 2;
+
+I8Plan w4a8_plan(int M, int K, int N)
+{
+    I8Plan d;
+    M = std::min(M, kW4A8DecodeMaxM);
+    d.NT = M <= 32 ? 32 : 64;
+    d.KB = K / 128;  // groups
+    d.nslabs = (N + 127) / 128;
+    d.units = d.KB * d.nslabs;
+    d.grid = std::min(std::min(num_sms(), d.units), 160);
+    d.partial_bytes = (size_t)d.grid * 2 * 128 * d.NT * sizeof(float);
+    return d;
+}
+
+template <int NT>
+qg_status launch_w4a8_decode(const int8_t* Xq, const float* t, int M, int K, const uint32_t* packed,
+                             const float* sg, int N, uint16_t* Y, int32_t* part_dbg, void* ws, qg_stream_t stream)
+{
+    using C = qg::W4A8DecCfg<NT, kW4A8Issuers>;
+    static_assert(C::TOTAL <= 227 * 1024, "W4A8 decode kernel shared memory");
+    auto kern = qg::w4a8_decode_kernel<NT, kW4A8Issuers>;
+    static KernelInfo info;
+    int occ = 1;
+    qg_status st = prepare_kernel(info, kern, C::THREADS, C::TOTAL, &occ);
+    if (st != QG_OK) return st;
+    const I8Plan d = w4a8_plan(M, K, N);
+    CUtensorMap tw, tx;
+    if ((st = make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, N, K / 8, 128, 16,
+                           CU_TENSOR_MAP_SWIZZLE_NONE)) ||
+        (st = make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Xq, K, M, 128, NT, CU_TENSOR_MAP_SWIZZLE_128B)))
+        return st;
+    qg::W4A8DecodeParams p{t, sg, Y, part_dbg, static_cast<float*>(ws), M, K, N, d.KB, d.nslabs, d.units, d.grid};
+    if ((st = launch_pdl(kern, dim3(d.grid), dim3(C::THREADS), C::TOTAL, stream, p, tw, tx)) != QG_OK) return st;
+    return launch_pdl(qg::w4a8_decode_fixup_kernel, dim3(d.nslabs), dim3(256), 0, stream, p, NT);
+}
+
 // ---------------------------------------------------------------------------
 // int8 skinny paths
 // ---------------------------------------------------------------------------
@@ -539,6 +582,10 @@ size_t qg_workspace_size(qg_op op, int M, int K, int N)
         case QG_OP_GEMM_W8A8: {
             if (M >= qg::kTcMinM || N % 16) return 0;
             return i8_plan(M, K, N).partial_bytes;
+        }
+        case QG_OP_GEMM_W4A8: {
+            if (M < kW4A8DecodeMinM || M >= qg::kTcMinMW4A8 || N % 16) return 0;
+            return w4a8_plan(M, K, N).partial_bytes;
         }
         default: return 0;
     }
@@ -654,19 +701,33 @@ qg_status qg_gemm_w4a8(const int8_t* Xq, const float* t, int M, int K, const uin
                        int N, int group, uint16_t* Y, int32_t* part_dbg, void* workspace, size_t ws_bytes,
                        qg_stream_t stream)
 {
-    (void)workspace;
-    (void)ws_bytes;
     if (M < 0 || K < 128 || N < 16 || K % 128 || N % 16 || group != 128) return QG_ERR_SHAPE;
     if (M == 0) return QG_OK;
     if (!Xq || !t || !packed || !sg || !Y) return QG_ERR_NULL;
     if (misaligned(Xq) || misaligned(t) || misaligned(packed) || misaligned(sg) || misaligned(Y) ||
-        misaligned(part_dbg))
+        misaligned(part_dbg) || misaligned(workspace))
         return QG_ERR_ALIGN;
     if (M >= qg::kTcMinMW4A8) {
         qg::TcInt8Args a{Xq, t, nullptr, nullptr, packed, sg, Y, part_dbg, M, K, N};
         return tc_w4a8(a, stream);
     }
     const int G = K / 128;
+    if (workspace && M >= kW4A8DecodeMinM) {
+        if (ws_bytes < qg_workspace_size(QG_OP_GEMM_W4A8, M, K, N)) return QG_ERR_WORKSPACE;
+        for (int m0 = 0; m0 < M; m0 += kW4A8DecodeMaxM) {
+            // chunks run in stream order; each reuses the workspace after the previous fixup
+            // (a ragged last chunk of 16 tokens or fewer runs on the 32-token tile)
+            const int mc = std::min(kW4A8DecodeMaxM, M - m0);
+            const int nt = w4a8_plan(mc, K, N).NT;
+            const int8_t* xc = Xq + (int64_t)m0 * K;
+            uint16_t* yc = Y + (int64_t)m0 * N;
+            int32_t* dc = part_dbg ? part_dbg + (int64_t)m0 * G * N : nullptr;
+            qg_status st = nt == 32 ? launch_w4a8_decode<32>(xc, t + m0, mc, K, packed, sg, N, yc, dc, workspace, stream)
+                                    : launch_w4a8_decode<64>(xc, t + m0, mc, K, packed, sg, N, yc, dc, workspace, stream);
+            if (st != QG_OK) return st;
+        }
+        return QG_OK;
+    }
     for (int m0 = 0; m0 < M; m0 += 32) {
         qg::Int8SkinnyParams p{Xq + (int64_t)m0 * K, t + m0, nullptr, nullptr, packed, sg, Y + (int64_t)m0 * N,
                                part_dbg ? part_dbg + (int64_t)m0 * G * N : nullptr, std::min(32, M - m0), K, N};

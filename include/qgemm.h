@@ -185,7 +185,15 @@ qg_status qg_gemm_w8a8(const int8_t* Xq, const float* t, int M, int K, const int
  * Xq int8 [M][K], t fp32 [M]; packed u32 [K/8][N] of symmetric codes (two's
  * complement nibbles in [-7,7]); sg fp32 [K/group][N]; Y bf16 [M][N].
  * part_dbg: NULL, or int32 [M][K/group][N] that also receives every P.
- * Rules: group == 128, K % 128 == 0, N % 16 == 0.  workspace unused (NULL, 0).
+ * Rules: group == 128, K % 128 == 0, N % 16 == 0.
+ * workspace: NULL, or (17 <= M < 128) a device buffer of at least
+ *   qg_workspace_size(QG_OP_GEMM_W4A8, M, K, N) bytes (contents irrelevant; it holds
+ *   the fp32 partial sums of column slabs split between CTAs; the size is 0, and any
+ *   workspace is ignored, for M <= 16 and M >= 128).  With it, 17 <= M < 128 runs the
+ *   stream-K tensor-core kernel on chunks of up to 64 tokens; without it (and always at
+ *   M <= 16), the cluster split-K kernel.  P is exact either way; Y may differ in the last bit
+ *   (fp32 summation order).  A workspace smaller than required -> QG_ERR_WORKSPACE
+ *   before any launch.  Calls that may run concurrently need workspaces of their own.
  * ------------------------------------------------------------------------ */
 qg_status qg_gemm_w4a8(const int8_t* Xq, const float* t, int M, int K, const uint32_t* packed,
                        const float* sg, int N, int group, uint16_t* Y, int32_t* part_dbg,

@@ -110,7 +110,9 @@ def test_workspace_size_and_too_small_workspace():
     assert L.qg_workspace_size(0, 1, 4096, 136) == 0       # N % 16 != 0: no workspace path
     assert L.qg_workspace_size(1, 16, 4096, 11008) > 0     # W8A8 below 128 tokens: stream-K partials
     assert L.qg_workspace_size(1, 128, 4096, 11008) == 0   # W8A8 tile kernel takes none
-    assert L.qg_workspace_size(2, 16, 4096, 11008) == 0    # W4A8 takes none
+    assert L.qg_workspace_size(2, 17, 4096, 11008) > 0     # W4A8 at 17..127 tokens: stream-K partials
+    assert L.qg_workspace_size(2, 16, 4096, 11008) == 0    # W4A8 at 16 tokens and fewer: split-K, none
+    assert L.qg_workspace_size(2, 128, 4096, 11008) == 0   # W4A8 tile kernel takes none
     assert L.qg_workspace_size(0, 0, 4096, 4096) == 0
     # a workspace smaller than required is refused before any launch
     assert L.qg_gemm_w4a16(A, 1, 32, 4096, 4096, A, A, A, 128, A, A, need - 1, None) == 10
@@ -118,3 +120,6 @@ def test_workspace_size_and_too_small_workspace():
     need8 = L.qg_workspace_size(1, 16, 4096, 11008)
     assert L.qg_gemm_w8a8(A, A, 16, 4096, A, A, 11008, A, None, A, need8 - 1, None) == 10
     assert L.qg_gemm_w8a8(A, A, 16, 4096, A, A, 11008, A, None, B, need8, None) == 3
+    need4 = L.qg_workspace_size(2, 32, 4096, 11008)
+    assert L.qg_gemm_w4a8(A, A, 32, 4096, A, A, 11008, 128, A, None, A, need4 - 1, None) == 10
+    assert L.qg_gemm_w4a8(A, A, 32, 4096, A, A, 11008, 128, A, None, B, need4, None) == 3

@@ -276,8 +276,11 @@ def w4a8_weights():
     return K, N, inv_o, oracle.pack_nibbles(c_o), sc_o
 
 
+@pytest.mark.parametrize("workspace", ["auto", None])
 @pytest.mark.parametrize("M", [1, 64, 1024, 3, 33])
-def test_gemm_w4a8(M, w4a8_weights):
+def test_gemm_w4a8(M, workspace, w4a8_weights):
+    """17..127 tokens: the stream-K kernel with a workspace, the cluster split-K kernel
+    without one; 16 tokens and fewer: split-K either way; 1024 tokens: the tile kernel."""
     K, N, inv_o, p_o, sc_o = w4a8_weights
     X, Xb = synth.workload_activations("w4a8", M, K)
     Xq_o, t_o, _ = oracle.smooth_quant_act_i8(X, inv_o)
@@ -286,7 +289,7 @@ def test_gemm_w4a8(M, w4a8_weights):
     want_part = M <= 64
     Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
     part = torch.empty(M, G, N, dtype=torch.int32, device="cuda") if want_part else None
-    q.qg_gemm_w4a8(cuda(Xq_o), cuda(t_o), cuda(p_o.view(np.int32)), cuda(sc_o), Y, part)
+    q.qg_gemm_w4a8(cuda(Xq_o), cuda(t_o), cuda(p_o.view(np.int32)), cuda(sc_o), Y, part, workspace=workspace)
     _status_ok()
     rows = sample_rows(M) if M > 64 else None
     part_o, yref, b = oracle.gemm_w4a8(Xq_o, t_o, p_o, sc_o, rows=rows, want_part=want_part)
@@ -296,6 +299,36 @@ def test_gemm_w4a8(M, w4a8_weights):
     if rows is not None:
         y = y[rows]
     assert_tol(y, yref, b)
+
+
+@pytest.mark.parametrize("K,N", [(512, 144), (1024, 272), (128, 16), (2048, 1296)])
+def test_gemm_w4a8_stream_k_edges(K, N):
+    """The W4A8 stream-K kernel (17..127 tokens) across its token tiles (32, 64 and chunks
+    of 64 with ragged last chunks), ragged column slabs, one-group K and slabs split
+    between CTAs, plus the split-K kernel the same call takes at 16 tokens and fewer; the
+    workspace starts with garbage (its contents must not matter)."""
+    rng = np.random.default_rng(3 * K + N)
+    q = qlib()
+    G = K // 128
+    ws = torch.full((q.qg_workspace_size(q.QG_OP_GEMM_W4A8, 127, K, N),), 0x5A, dtype=torch.uint8, device="cuda")
+    codes = rng.integers(-7, 8, (K, N)).astype(np.int8)
+    sg = rng.uniform(0.001, 0.01, (G, N)).astype(np.float32)
+    p_o = oracle.pack_nibbles(codes)
+    for M in [1, 2, 15, 16, 17, 31, 32, 33, 63, 64, 65, 100, 127]:
+        Xq = rng.integers(-127, 128, (M, K)).astype(np.int8)
+        t = rng.uniform(0.01, 1.0, M).astype(np.float32)
+        Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        part = torch.full((M, G, N), -1, dtype=torch.int32, device="cuda")
+        q.qg_gemm_w4a8(cuda(Xq), cuda(t), cuda(p_o.view(np.int32)), cuda(sg), Y, part, workspace=ws)
+        _status_ok()
+        part_o, yref, b = oracle.gemm_w4a8(Xq, t, p_o, sg)
+        np.testing.assert_array_equal(part.cpu().numpy(), part_o, err_msg=f"M={M}")
+        assert_tol(bf16_to_f32(u16(Y)), yref, b)
+        # without the debug output the same kernel path gives the same Y
+        Y2 = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        q.qg_gemm_w4a8(cuda(Xq), cuda(t), cuda(p_o.view(np.int32)), cuda(sg), Y2, None, workspace=ws)
+        _status_ok()
+        assert torch.equal(Y2.view(torch.int16), Y.view(torch.int16)), f"M={M}"
 
 
 # ---------------------------------------------------------------------------
