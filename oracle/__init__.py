@@ -86,6 +86,16 @@ def _declare(L):
     L.qgo_gemm_w4a8.restype = None
     L.qgo_gemm_f64.argtypes = [_p, _i64, _i64, _p, _i64, _p, _i64, _p]
     L.qgo_gemm_f64.restype = None
+    L.qgo_awq_act_mean.argtypes = [_p, _i64, _i64, _p]
+    L.qgo_awq_act_mean.restype = None
+    L.qgo_awq_scales.argtypes = [_p, _i64, ctypes.c_double, _p, _p]
+    L.qgo_awq_scales.restype = None
+    L.qgo_awq_alpha.argtypes = [_int, _int]
+    L.qgo_awq_alpha.restype = ctypes.c_double
+    L.qgo_awq_candidate_mse.argtypes = [_p, _i64, _i64, _p, _i64, _int, _p, _p, _p, _p]
+    L.qgo_awq_candidate_mse.restype = _int
+    L.qgo_awq_search.argtypes = [_p, _i64, _i64, _p, _i64, _int, _int, _p, _p, _p, _p]
+    L.qgo_awq_search.restype = _int
 
 
 def _c(a, dtype):
@@ -262,6 +272,62 @@ def gemm_f64(X, W, rows=None):
     y = np.zeros((nr, N), np.float64)
     lib().qgo_gemm_f64(_ptr(Xc), M, K, _ptr(Wc), N, _ptr(r), nr, _ptr(y))
     return y
+
+
+# --------------------------------------------------------------------------
+# AWQ scale search ("Quantization & Flash Attention -- LLM inference optimization (2)",
+# sec. 2.1-2.3): s_c = mean|X_c|^alpha, alpha on a grid in [0, 1], least output MSE
+# --------------------------------------------------------------------------
+def awq_act_mean(X):
+    """xm[c] = mean over tokens of |X[m][c]| (binary64 sum in token order, one rounding) -> f32 [K]."""
+    Xc = _c(X, np.float32)
+    M, K = Xc.shape
+    xm = np.zeros(K, np.float32)
+    lib().qgo_awq_act_mean(_ptr(Xc), M, K, _ptr(xm))
+    return xm
+
+
+def awq_alpha(i, n_grid):
+    """Grid point i of n_grid equally spaced points on [0, 1], both ends included."""
+    return lib().qgo_awq_alpha(int(i), int(n_grid))
+
+
+def awq_scales(xm, alpha):
+    """s = xm^alpha (binary64 pow, one rounding; xm == 0 -> 1) and inv_s = 1/s -> (s, inv_s) f32 [K]."""
+    x = _c(xm, np.float32)
+    s = np.zeros_like(x)
+    inv = np.zeros_like(x)
+    lib().qgo_awq_scales(_ptr(x), x.size, float(alpha), _ptr(s), _ptr(inv))
+    return s, inv
+
+
+def awq_candidate_mse(X, W, s, inv_s, group=128, yref=None):
+    """MSE over all outputs of X W - bf16(X inv_s) deq(Q(diag(s) W)) -> (mse, status)."""
+    Xc = _c(X, np.float32)
+    Wc = _c(W, np.float32)
+    M, K = Xc.shape
+    N = Wc.shape[1]
+    if yref is None:
+        yref = gemm_f64(Xc, Wc)
+    yref = _c(yref, np.float64)
+    out = np.zeros(1, np.float64)
+    st = lib().qgo_awq_candidate_mse(_ptr(Xc), M, K, _ptr(Wc), N, group, _ptr(_c(s, np.float32)),
+                                     _ptr(_c(inv_s, np.float32)), _ptr(yref), _ptr(out))
+    return float(out[0]), st
+
+
+def awq_search(X, W, n_grid=21, group=128):
+    """Grid search of alpha -> (mse f64 [n_grid], best index, s_best f32 [K], inv_s_best f32 [K], status)."""
+    Xc = _c(X, np.float32)
+    Wc = _c(W, np.float32)
+    M, K = Xc.shape
+    N = Wc.shape[1]
+    mse = np.zeros(n_grid, np.float64)
+    best = np.zeros(1, np.int32)
+    s = np.zeros(K, np.float32)
+    inv = np.zeros(K, np.float32)
+    st = lib().qgo_awq_search(_ptr(Xc), M, K, _ptr(Wc), N, group, n_grid, _ptr(mse), _ptr(best), _ptr(s), _ptr(inv))
+    return mse, int(best[0]), s, inv, st
 
 
 def within_tolerance(y, yref, bound, rel=1e-2, abs_=1e-3):

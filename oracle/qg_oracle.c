@@ -454,3 +454,130 @@ void qgo_gemm_f64(const float* X, int64_t M, int64_t K, const float* W, int64_t 
                 y[r * N + n] += (double)X[(rows ? rows[r] : r) * K + k] * w;
         }
 }
+
+/* ------------------------------------------------------------------------- */
+/* AWQ: activation-aware per-input-channel scales for the INT4 weights.        */
+/* "Quantization & Flash Attention -- LLM inference optimization (2)":          */
+/*   sec. 2.1  the statistic: the mean magnitude E[|X_c|] of each input channel */
+/*             over a small calibration batch;                                  */
+/*   sec. 2.2  the equivalent transform X W = (X / s)(s W), s per input channel;*/
+/*   sec. 2.3  s_c = mean(|X_c|)^alpha, alpha on a grid in [0, 1], chosen to    */
+/*             minimise the MSE between X W and the quantized layer's output.   */
+/* Readings (listed in the design notes):                                       */
+/*   K  the mean is a binary64 sum over the tokens in order, divided by the     */
+/*      token count in binary64 and rounded once to binary32;                   */
+/*   L  s_c = xm_c^alpha in binary64 (pow), rounded once to binary32; a channel */
+/*      whose statistic is 0 keeps s_c = 1; inv_s_c = 1/s_c in binary32;       */
+/*   M  the quantizer Q of sec. 2.3 acts on the scaled weight s W (the method   */
+/*      quantizes weights only): asymmetric INT4 groups of O1 applied to        */
+/*      diag(s) W, and the scaled activations X / s are stored in the layer's   */
+/*      activation dtype: X~ = bf16_rn(X * inv_s);                              */
+/*   N  the grid is alpha_i = i / (n_grid - 1), i = 0 .. n_grid - 1, both ends  */
+/*      included (n_grid == 1: alpha = 0 only); the MSE is the mean over all    */
+/*      M x N outputs of (X W - X~ deq(Q(s W)))^2 in binary64, both products    */
+/*      exact up to binary64 rounding; the first grid point with the least MSE  */
+/*      wins.                                                                   */
+/* ------------------------------------------------------------------------- */
+
+/* xm[c] = mean_m |X[m][c]| (reading K) */
+void qgo_awq_act_mean(const float* X, int64_t M, int64_t K, float* xm)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t c = 0; c < K; ++c) {
+        double sum = 0.0;
+        for (int64_t m = 0; m < M; ++m) sum += fabs((double)X[m * K + c]);
+        xm[c] = (float)(sum / (double)M);
+    }
+}
+
+/* s[c] = xm[c]^alpha, inv_s[c] = 1 / s[c] (reading L) */
+void qgo_awq_scales(const float* xm, int64_t K, double alpha, float* s, float* inv_s)
+{
+    for (int64_t c = 0; c < K; ++c) {
+        float sc = xm[c] == 0.0f ? 1.0f : (float)pow((double)xm[c], alpha);
+        s[c] = sc;
+        inv_s[c] = 1.0f / sc;
+    }
+}
+
+/* grid point i of n (reading N) */
+double qgo_awq_alpha(int i, int n_grid) { return n_grid > 1 ? (double)i / (double)(n_grid - 1) : 0.0; }
+
+/* yref[m][n] = sum_k X[m][k] W[k][n] in binary64 */
+static void awq_yref(const float* X, int64_t M, int64_t K, const float* W, int64_t N, double* yref)
+{
+    memset(yref, 0, sizeof(double) * M * N);
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k) {
+            double w = (double)W[k * N + n];
+            for (int64_t m = 0; m < M; ++m) yref[m * N + n] += (double)X[m * K + k] * w;
+        }
+}
+
+/* MSE of one candidate scale vector against yref (reading M, N).  Returns the
+ * quantizer's status; *mse is left unset unless that status is 0. */
+int qgo_awq_candidate_mse(const float* X, int64_t M, int64_t K, const float* W, int64_t N, int group,
+                          const float* s, const float* inv_s, const double* yref, double* mse)
+{
+    uint8_t* codes = (uint8_t*)malloc((size_t)K * N);
+    uint16_t* sc = (uint16_t*)malloc(sizeof(uint16_t) * (size_t)(K / group) * N);
+    uint8_t* z = (uint8_t*)malloc((size_t)(K / group) * N);
+    float* xs = (float*)malloc(sizeof(float) * (size_t)M * K);
+    double* yq = (double*)calloc((size_t)M * N, sizeof(double));
+    int status = qgo_quantize_w4_asym(W, s, K, N, group, codes, sc, z); /* Q(diag(s) W), O1 */
+    if (status == OR_OK) {
+        for (int64_t m = 0; m < M; ++m)
+            for (int64_t k = 0; k < K; ++k) /* X~ = bf16_rn(X * inv_s) */
+                xs[m * K + k] = qgo_bf16_to_f32(qgo_f32_to_bf16_rn(X[m * K + k] * inv_s[k]));
+#pragma omp parallel for schedule(static)
+        for (int64_t n = 0; n < N; ++n)
+            for (int64_t k = 0; k < K; ++k) {
+                int64_t g = k / group;
+                double w = (double)((int)codes[k * N + n] - (int)z[g * N + n]) * (double)qgo_f16_to_f32(sc[g * N + n]);
+                for (int64_t m = 0; m < M; ++m) yq[m * N + n] += (double)xs[m * K + k] * w;
+            }
+        double acc = 0.0;
+        for (int64_t i = 0; i < M * N; ++i) {
+            double d = yref[i] - yq[i];
+            acc += d * d;
+        }
+        *mse = acc / (double)(M * N);
+    }
+    free(codes);
+    free(sc);
+    free(z);
+    free(xs);
+    free(yq);
+    return status;
+}
+
+/* The grid search of sec. 2.3: mse[i] for every grid point, *best = the first
+ * index with the least MSE, and the scales at that point.  Returns the first
+ * non-zero quantizer status (mse and best are then unspecified). */
+int qgo_awq_search(const float* X, int64_t M, int64_t K, const float* W, int64_t N, int group, int n_grid,
+                   double* mse, int* best, float* s_best, float* inv_s_best)
+{
+    float* xm = (float*)malloc(sizeof(float) * (size_t)K);
+    float* s = (float*)malloc(sizeof(float) * (size_t)K);
+    float* inv_s = (float*)malloc(sizeof(float) * (size_t)K);
+    double* yref = (double*)malloc(sizeof(double) * (size_t)M * N);
+    int status = OR_OK;
+    qgo_awq_act_mean(X, M, K, xm);
+    awq_yref(X, M, K, W, N, yref);
+    int bi = 0;
+    for (int i = 0; i < n_grid && status == OR_OK; ++i) {
+        qgo_awq_scales(xm, K, qgo_awq_alpha(i, n_grid), s, inv_s);
+        status = qgo_awq_candidate_mse(X, M, K, W, N, group, s, inv_s, yref, &mse[i]);
+        if (status == OR_OK && mse[i] < mse[bi]) bi = i;
+    }
+    if (status == OR_OK) {
+        *best = bi;
+        qgo_awq_scales(xm, K, qgo_awq_alpha(bi, n_grid), s_best, inv_s_best);
+    }
+    free(xm);
+    free(s);
+    free(inv_s);
+    free(yref);
+    return status;
+}

@@ -4,6 +4,7 @@ then fail.  This shows the pins constrain the oracle's arithmetic, not just its 
 import pytest
 
 import oracle
+import test_oracle_awq_pins as awq
 import test_oracle_pins as pins
 
 MUTATIONS = [
@@ -23,6 +24,19 @@ MUTATIONS = [
     ("int qw = v >= 8 ? v - 16 : v;", "int qw = v;", [pins.test_w4a8_partials_and_reference]),
     ("float tm = a / 127.0f;", "float tm = a / 128.0f;", [pins.test_act_i8_closed_form_and_brute_force]),
     ("float s = amax / 7.0f;", "float s = amax / 8.0f;", [pins.test_w4_sym_absmax_bound_brute_force]),
+    # AWQ search
+    ("sum += fabs((double)X[m * K + c]);", "sum += (double)X[m * K + c];", [awq.test_act_mean_closed_form]),
+    ("(float)pow((double)xm[c], alpha);", "(float)pow((double)xm[c], 1.0 - alpha);",
+     [awq.test_scales_closed_forms, awq.test_alpha_one_is_exact_on_the_constructed_layer]),
+    ("qgo_f32_to_bf16_rn(X[m * K + k] * inv_s[k])", "qgo_f32_to_bf16_rn(X[m * K + k] * s[k])",
+     [awq.test_alpha_one_is_exact_on_the_constructed_layer]),
+    ("int status = qgo_quantize_w4_asym(W, s, K, N, group, codes, sc, z);",
+     "int status = qgo_quantize_w4_asym(W, inv_s, K, N, group, codes, sc, z);",
+     [awq.test_alpha_one_is_exact_on_the_constructed_layer]),
+    ("if (status == OR_OK && mse[i] < mse[bi]) bi = i;", "if (status == OR_OK && mse[i] <= mse[bi]) bi = i;",
+     [awq.test_zero_weights_tie_goes_to_the_first_point]),
+    ("(double)i / (double)(n_grid - 1)", "(double)i / (double)n_grid", [awq.test_grid_points]),
+    ("double d = yref[i] - yq[i];", "double d = yref[i] - 0.5 * yq[i];", [awq.test_alpha_zero_is_the_plain_int4_layer]),
 ]
 
 
