@@ -506,9 +506,45 @@ def bench_configs(q, pk, int8_peak):
             del X, Y
         del pw, sc, z
     out["w4a16_prefill"] = res
+    # --- AWQ scale search: 512 calibration tokens, the decode QKV weight, 21 grid points --
+    try:
+        out["awq_search"] = bench_awq(q, pk)
+    except Exception as e:  # reported in the line, not fatal to the headline
+        out["awq_search"] = {"error": repr(e)}
     out["int8_peak_tops_measured"] = int8_peak
     out["bf16_peak_tflops_measured"] = bf16_peak
     return out
+
+
+def bench_awq(q, pk):
+    cfg = synth.CONFIGS["awq"]
+    K, N = cfg["KN"][0]
+    Mc, ng = cfg["calib_tokens"], cfg["n_grid"]
+    W = torch.from_numpy(synth.workload_weights("awq", K, N)).cuda()
+    _, xcb = synth.calibration(K, cfg)
+    Xc = torch.from_numpy(xcb.view(np.int16)).cuda().view(torch.bfloat16)
+    mse = torch.empty(ng, dtype=torch.float64, device="cuda")
+    best = torch.empty(1, dtype=torch.int32, device="cuda")
+    s_b = torch.empty(K, dtype=torch.float32, device="cuda")
+    inv_b = torch.empty_like(s_b)
+    ms = time_calls(lambda i: q.qg_awq_search(Xc, W, ng, mse, best, s_b, inv_b), 1)
+    G = K // 128
+    # per grid point, algorithmic bytes of its kernels (run one after another):
+    # quantize diag(s) W (read W, s; write codes, fp16 scales, zeros), pack (read codes,
+    # write words), scale X, the W4A16 GEMM (words, scales, zeros, X/s, Y), the error (Yref, Y)
+    cand_bytes = (4 * K * N + 4 * K + K * N + 3 * G * N + K * N + K * N // 2 + 4 * Mc * K + 4 * K +
+                  K * N // 2 + 3 * G * N + 2 * Mc * K + 2 * Mc * N + 6 * Mc * N)
+    cand_flops = 2 * Mc * K * N
+    t_cand = cand_bytes / (pk["hbm_gbs"] * 1e9) + cand_flops / (pk["bf16_tflops"] * 1e12)
+    b_i = int(best.item())
+    m_np = mse.cpu().numpy()
+    assert q.qg_device_status() == q.QG_OK
+    return {"ms": ms, "ms_per_grid_point": ms / ng, "grid_points": ng, "calib_tokens": Mc, "K": K, "N": N,
+            "best_alpha": b_i / (ng - 1), "mse_plain_over_best": float(m_np[0] / m_np[b_i]),
+            "grid_point_bytes": cand_bytes, "grid_point_flops": cand_flops,
+            "roofline_frac": ng * t_cand / (ms * 1e-3),
+            "note": "roofline = per grid point HBM time of its passes + bf16 tensor time of its GEMM; "
+                    "the once-per-search fp32 reference GEMM is in the measured time only"}
 
 
 def run_single(spec, reps, workspace="auto", op="w4a16"):

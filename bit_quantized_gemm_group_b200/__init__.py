@@ -23,11 +23,12 @@ QG_OK, QG_ERR_NULL, QG_ERR_SHAPE, QG_ERR_ALIGN, QG_ERR_DTYPE = 0, 1, 2, 3, 4
 QG_ERR_NONFINITE, QG_ERR_RANGE, QG_ERR_TIMEOUT, QG_ERR_CUDA, QG_ERR_UNSUPPORTED = 5, 6, 7, 8, 9
 QG_ERR_WORKSPACE = 10
 QG_F16, QG_BF16 = 0, 1
-QG_OP_GEMM_W4A16, QG_OP_GEMM_W8A8, QG_OP_GEMM_W4A8 = 0, 1, 2
+QG_OP_GEMM_W4A16, QG_OP_GEMM_W8A8, QG_OP_GEMM_W4A8, QG_OP_AWQ_SEARCH = 0, 1, 2, 3
 
 EXPORTS = ["qg_quantize_w4_group", "qg_pack_nibbles", "qg_gemm_w4a16", "qg_smooth_quant_act_i8", "qg_gemm_w8a8",
            "qg_gemm_w4a8", "qg_smooth_scales", "qg_quantize_w8_channel", "qg_device_status", "qg_status_string",
-           "qg_last_error", "qg_selftest_bounded_wait", "qg_workspace_size", "qg_gemm_w4a16_noalloc"]
+           "qg_last_error", "qg_selftest_bounded_wait", "qg_workspace_size", "qg_gemm_w4a16_noalloc",
+           "qg_awq_act_mean", "qg_awq_scales", "qg_awq_scale_act", "qg_awq_search"]
 
 
 class QgError(RuntimeError):
@@ -50,6 +51,10 @@ _SIGS = {
     "qg_gemm_w4a8": [_P, _P, _I, _I, _P, _P, _I, _I, _P, _P, _P, _SZ, _P],
     "qg_smooth_scales": [_P, _I, _P, _I, _I, ctypes.c_float, _P, _P, _P],
     "qg_quantize_w8_channel": [_P, _P, _I, _I, _P, _P, _P],
+    "qg_awq_act_mean": [_P, _I, _I, _P, _P],
+    "qg_awq_scales": [_P, _I, ctypes.c_double, _P, _P, _P],
+    "qg_awq_scale_act": [_P, _I, _I, _P, _P, _P],
+    "qg_awq_search": [_P, _I, _I, _P, _I, _I, _I, _P, _P, _P, _P, _P, _SZ, _P],
     "qg_device_status": [_P],
     "qg_selftest_bounded_wait": [ctypes.c_uint64, _P],
 }
@@ -196,6 +201,29 @@ def qg_quantize_w8_channel(W, s, Wq, sw, stream=None):
     K, N = W.shape
     _check(lib().qg_quantize_w8_channel(_ptr(W), _ptr(s), K, N, _ptr(Wq), _ptr(sw), _stream(stream)),
            "qg_quantize_w8_channel")
+
+
+def qg_awq_act_mean(Xcal, xm, stream=None):
+    Mc, K = Xcal.shape
+    _check(lib().qg_awq_act_mean(_ptr(Xcal), Mc, K, _ptr(xm), _stream(stream)), "qg_awq_act_mean")
+
+
+def qg_awq_scales(xm, alpha, s, inv_s, stream=None):
+    _check(lib().qg_awq_scales(_ptr(xm), xm.numel(), float(alpha), _ptr(s), _ptr(inv_s), _stream(stream)),
+           "qg_awq_scales")
+
+
+def qg_awq_scale_act(X, inv_s, Xs, stream=None):
+    M, K = X.shape
+    _check(lib().qg_awq_scale_act(_ptr(X), M, K, _ptr(inv_s), _ptr(Xs), _stream(stream)), "qg_awq_scale_act")
+
+
+def qg_awq_search(Xcal, W, n_grid, mse, best, s, inv_s, group=128, workspace="auto", stream=None):
+    Mc, K = Xcal.shape
+    N = W.shape[1]
+    wp, wb = _ws(workspace, QG_OP_AWQ_SEARCH, Mc, K, N, Xcal.device)
+    _check(lib().qg_awq_search(_ptr(Xcal), Mc, K, _ptr(W), N, group, n_grid, _ptr(mse), _ptr(best), _ptr(s),
+                              _ptr(inv_s), wp, wb, _stream(stream)), "qg_awq_search")
 
 
 def qg_device_status(stream=None) -> int:

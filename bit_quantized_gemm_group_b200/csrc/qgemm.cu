@@ -11,6 +11,7 @@
 
 #include "../../include/qgemm.h"
 #include "act_quant.cuh"
+#include "awq.cuh"
 #include "common.cuh"
 #include "int8_skinny.cuh"
 #include "quantize.cuh"
@@ -509,6 +510,45 @@ qg_status launch_w4a8_decode(const int8_t* Xq, const float* t, int M, int K, con
     return launch_pdl(qg::w4a8_decode_fixup_kernel, dim3(d.nslabs), dim3(256), 0, stream, p, NT);
 }
 
+// AWQ search workspace: every buffer one candidate needs, 256-byte aligned pieces
+struct AwqWs {
+    float *xm, *sc, *inv;
+    uint16_t* xs;
+    uint8_t* codes;
+    uint16_t* scales;
+    uint8_t* zeros;
+    uint32_t* packed;
+    uint16_t* yq;
+    float* yref;
+    double* partials;
+    size_t bytes;
+};
+
+AwqWs awq_carve(void* base, int Mc, int K, int N)
+{
+    AwqWs w{};
+    size_t off = 0;
+    auto take = [&](size_t b) {
+        const size_t o = off;
+        off += (b + 255) & ~size_t(255);
+        return base ? static_cast<uint8_t*>(base) + o : nullptr;
+    };
+    const size_t G = (size_t)K / 128;
+    w.xm = reinterpret_cast<float*>(take(4 * (size_t)K));
+    w.sc = reinterpret_cast<float*>(take(4 * (size_t)K));
+    w.inv = reinterpret_cast<float*>(take(4 * (size_t)K));
+    w.xs = reinterpret_cast<uint16_t*>(take(2 * (size_t)Mc * K));
+    w.codes = take((size_t)K * N);
+    w.scales = reinterpret_cast<uint16_t*>(take(2 * G * N));
+    w.zeros = take(G * N);
+    w.packed = reinterpret_cast<uint32_t*>(take((size_t)K / 2 * N));
+    w.yq = reinterpret_cast<uint16_t*>(take(2 * (size_t)Mc * N));
+    w.yref = reinterpret_cast<float*>(take(4 * (size_t)Mc * N));
+    w.partials = reinterpret_cast<double*>(take(8 * (size_t)qg::kAwqErrBlocks));
+    w.bytes = off;
+    return w;
+}
+
 // ---------------------------------------------------------------------------
 // int8 skinny paths
 // ---------------------------------------------------------------------------
@@ -582,6 +622,10 @@ size_t qg_workspace_size(qg_op op, int M, int K, int N)
         case QG_OP_GEMM_W8A8: {
             if (M >= qg::kTcMinM || N % 16) return 0;
             return i8_plan(M, K, N).partial_bytes;
+        }
+        case QG_OP_AWQ_SEARCH: {
+            if (N % 8) return 0;
+            return awq_carve(nullptr, M, K, N).bytes;
         }
         case QG_OP_GEMM_W4A8: {
             if (M < kW4A8DecodeMinM || M >= qg::kTcMinMW4A8 || N % 16) return 0;
@@ -752,6 +796,86 @@ qg_status qg_smooth_scales(const uint16_t* Xcal, int Mc, const float* W, int K, 
     qg::row_absmax_f32_kernel<<<K, 256, 0, st>>>(W, K, N, inv_s);
     QG_CUDA(cudaGetLastError());
     qg::smooth_finalize_kernel<<<(K + 255) / 256, 256, 0, st>>>(s, inv_s, K, alpha);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+
+qg_status qg_awq_act_mean(const uint16_t* Xcal, int Mc, int K, float* xm, qg_stream_t stream)
+{
+    if (!Xcal || !xm) return QG_ERR_NULL;
+    if (Mc < 1 || K < 1) return QG_ERR_SHAPE;
+    if (misaligned(Xcal) || misaligned(xm)) return QG_ERR_ALIGN;
+    qg::awq_act_mean_kernel<<<(K + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(Xcal, Mc, K, xm);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+
+qg_status qg_awq_scales(const float* xm, int K, double alpha, float* s, float* inv_s, qg_stream_t stream)
+{
+    if (!xm || !s || !inv_s) return QG_ERR_NULL;
+    if (K < 1 || !(alpha >= 0.0 && alpha <= 1.0)) return QG_ERR_SHAPE;
+    if (misaligned(xm) || misaligned(s) || misaligned(inv_s)) return QG_ERR_ALIGN;
+    qg::awq_scales_kernel<<<(K + 255) / 256, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(xm, K, alpha, nullptr,
+                                                                                                  0, s, inv_s);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+
+qg_status qg_awq_scale_act(const uint16_t* X, int M, int K, const float* inv_s, uint16_t* Xs, qg_stream_t stream)
+{
+    if (M < 0 || K < 8 || K % 8) return QG_ERR_SHAPE;
+    if (M == 0) return QG_OK;
+    if (!X || !inv_s || !Xs) return QG_ERR_NULL;
+    if (misaligned(X) || misaligned(inv_s) || misaligned(Xs)) return QG_ERR_ALIGN;
+    const int64_t total8 = (int64_t)M * K / 8;
+    const int grid = (int)std::min<int64_t>((total8 + 255) / 256, 8 * num_sms());
+    qg::awq_scale_act_kernel<<<grid, 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(X, total8, K, inv_s, Xs);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+
+qg_status qg_awq_search(const uint16_t* Xcal, int Mc, int K, const float* W, int N, int group, int n_grid,
+                        double* mse, int32_t* best, float* s, float* inv_s, void* workspace, size_t ws_bytes,
+                        qg_stream_t stream)
+{
+    if (!Xcal || !W || !mse || !best || !s || !inv_s || !workspace) return QG_ERR_NULL;
+    if (Mc < 1 || K < 128 || K % 128 || N < 8 || N % 8 || group != 128 || n_grid < 1 || n_grid > 1024)
+        return QG_ERR_SHAPE;
+    if (misaligned(Xcal) || misaligned(W) || misaligned(mse) || misaligned(best) || misaligned(s) ||
+        misaligned(inv_s) || misaligned(workspace))
+        return QG_ERR_ALIGN;
+    if (ws_bytes < awq_carve(nullptr, Mc, K, N).bytes) return QG_ERR_WORKSPACE;
+    const AwqWs w = awq_carve(workspace, Mc, K, N);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int kgrid = (K + 255) / 256;
+    const int64_t outs = (int64_t)Mc * N;
+    qg_status r;
+    // statistic and reference output, once
+    qg::awq_act_mean_kernel<<<kgrid, 256, 0, st>>>(Xcal, Mc, K, w.xm);
+    QG_CUDA(cudaGetLastError());
+    qg::awq_ref_gemm_kernel<<<dim3((N + qg::kAwqRefBN - 1) / qg::kAwqRefBN, (Mc + qg::kAwqRefBM - 1) / qg::kAwqRefBM),
+                              256, 0, st>>>(Xcal, W, Mc, K, N, w.yref);
+    QG_CUDA(cudaGetLastError());
+    // one candidate per grid point: scales -> Q(diag(s) W) -> packed -> X / s -> W4A16 GEMM -> error
+    for (int i = 0; i < n_grid; ++i) {
+        const double alpha = n_grid > 1 ? (double)i / (double)(n_grid - 1) : 0.0;
+        qg::awq_scales_kernel<<<kgrid, 256, 0, st>>>(w.xm, K, alpha, nullptr, 0, w.sc, w.inv);
+        QG_CUDA(cudaGetLastError());
+        if ((r = qg_quantize_w4_group(W, w.sc, K, N, 128, 0, w.codes, w.scales, w.zeros, stream)) != QG_OK) return r;
+        if ((r = qg_pack_nibbles(w.codes, K, N, w.packed, stream)) != QG_OK) return r;
+        if ((r = qg_awq_scale_act(Xcal, Mc, K, w.inv, w.xs, stream)) != QG_OK) return r;
+        if ((r = qg_gemm_w4a16(w.xs, QG_BF16, Mc, K, N, w.packed, w.scales, w.zeros, 128, w.yq, nullptr, 0, stream)) !=
+            QG_OK)
+            return r;
+        qg::awq_sqerr_kernel<<<qg::kAwqErrBlocks, 256, 0, st>>>(w.yref, w.yq, outs, w.partials);
+        QG_CUDA(cudaGetLastError());
+        qg::awq_mse_finish_kernel<<<1, 32, 0, st>>>(w.partials, outs, mse + i);
+        QG_CUDA(cudaGetLastError());
+    }
+    // the winner and its scales
+    qg::awq_argmin_kernel<<<1, 32, 0, st>>>(mse, n_grid, best);
+    QG_CUDA(cudaGetLastError());
+    qg::awq_scales_kernel<<<kgrid, 256, 0, st>>>(w.xm, K, 0.0, best, n_grid, s, inv_s);
     QG_CUDA(cudaGetLastError());
     return QG_OK;
 }

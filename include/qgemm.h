@@ -12,6 +12,10 @@
  *        fused (Marlin-style) so that no dequantized copy of W is written.
  *   [G]  "LLM inference cost: W8A8/W4A8 ..." (0539edu.com), sec. 2.2: group-wise
  *        quantization with an independent scale and zero per group of 128; W4A8.
+ *   [A]  "Quantization & Flash Attention -- LLM inference optimization (2)"
+ *        (hustzhy.cn), sec. 2.1-2.3 (AWQ): per-input-channel scales
+ *        s_c = mean(|X_c|)^alpha, X W = (X / s)(s W), alpha chosen on a grid in
+ *        [0, 1] by the least MSE of the quantized layer's output.
  *
  * Readings taken where the pages are silent (the same ones the test oracle takes):
  *   asymmetric INT4 uses s = (max' - min')/15 over a range widened to contain 0,
@@ -65,7 +69,7 @@ typedef enum {
 } qg_status;
 
 /* Operations that may use a caller-provided workspace (qg_workspace_size). */
-typedef enum { QG_OP_GEMM_W4A16 = 0, QG_OP_GEMM_W8A8 = 1, QG_OP_GEMM_W4A8 = 2 } qg_op;
+typedef enum { QG_OP_GEMM_W4A16 = 0, QG_OP_GEMM_W8A8 = 1, QG_OP_GEMM_W4A8 = 2, QG_OP_AWQ_SEARCH = 3 } qg_op;
 
 typedef enum { QG_F16 = 0, QG_BF16 = 1 } qg_dtype;
 
@@ -225,8 +229,55 @@ qg_status qg_smooth_scales(const uint16_t* Xcal, int Mc, const float* W, int K, 
 qg_status qg_quantize_w8_channel(const float* W, const float* s, int K, int N, int8_t* Wq, float* sw,
                                  qg_stream_t stream);
 
+/* --------------------------------------------------------------------------
+ * AWQ: activation-aware per-input-channel scales for the INT4 weights.   [A]
+ *
+ * Statistic (sec. 2.1):
+ *   xm[c] = mean over the Mc calibration tokens of |Xcal[m][c]|: a binary64 sum
+ *   over the tokens in order, divided by Mc in binary64, rounded once to fp32
+ *   (the same bits on every run).
+ * Xcal bf16 [Mc][K]; xm fp32 [K].  Rules: Mc >= 1, K >= 1.
+ * ------------------------------------------------------------------------ */
+qg_status qg_awq_act_mean(const uint16_t* Xcal, int Mc, int K, float* xm, qg_stream_t stream);
+
+/* Scales for one exponent (sec. 2.3):
+ *   s[c] = xm[c]^alpha (binary64 pow, rounded once to fp32); xm[c] == 0 -> s[c] = 1;
+ *   inv_s[c] = 1 / s[c] (fp32, round to nearest).
+ * Rules: K >= 1, 0 <= alpha <= 1. */
+qg_status qg_awq_scales(const float* xm, int K, double alpha, float* s, float* inv_s,
+                        qg_stream_t stream);
+
+/* The scaled activations of the equivalent transform (sec. 2.2), in bf16:
+ *   Xs[m][k] = bf16_rn(X[m][k] * inv_s[k])   (one fp32 product, one rounding)
+ * X, Xs bf16 [M][K]; inv_s fp32 [K].  Rules: K % 8 == 0. */
+qg_status qg_awq_scale_act(const uint16_t* X, int M, int K, const float* inv_s, uint16_t* Xs,
+                           qg_stream_t stream);
+
+/* The grid search (sec. 2.3), on the device, asynchronous on `stream`:
+ *   alpha_i = i / (n_grid - 1), i = 0 .. n_grid-1 (alpha = 0 only when n_grid == 1);
+ *   for each: s = xm^alpha; codes, scales, zeros = asymmetric INT4 groups of
+ *   diag(s) W (qg_quantize_w4_group with s_smooth = s); Xs = qg_awq_scale_act(Xcal);
+ *   Yq = qg_gemm_w4a16(Xs, ...) (bf16);
+ *   mse[i] = mean over Mc x N of (Yref - Yq)^2 in binary64, where Yref = Xcal W
+ *   with fp32 accumulation;
+ *   best = the first i with the least mse[i]; s, inv_s = the scales at alpha_best.
+ * Xcal bf16 [Mc][K]; W fp32 [K][N]; mse fp64 [n_grid]; best int32 [1]; s, inv_s
+ * fp32 [K] (all device memory).  The winning weights are then
+ * qg_quantize_w4_group(W, s, ...), and the layer's activations are scaled by inv_s
+ * (qg_awq_scale_act, or folded into the producer of X).
+ * Rules: group == 128, K % 128 == 0, N % 8 == 0, Mc >= 1, 1 <= n_grid <= 1024.
+ * workspace (required): a device buffer of at least
+ *   qg_workspace_size(QG_OP_AWQ_SEARCH, Mc, K, N) bytes, contents irrelevant.
+ *   NULL -> QG_ERR_NULL; smaller -> QG_ERR_WORKSPACE, before any launch.
+ * Device errors: those of the quantizer (QG_ERR_NONFINITE, QG_ERR_RANGE).
+ * ------------------------------------------------------------------------ */
+qg_status qg_awq_search(const uint16_t* Xcal, int Mc, int K, const float* W, int N, int group,
+                        int n_grid, double* mse, int32_t* best, float* s, float* inv_s,
+                        void* workspace, size_t ws_bytes, qg_stream_t stream);
+
 /* Bytes of workspace the given operation and shape can use (0 = none).  The
- * value depends only on (op, M, K, N) and on the current device. */
+ * value depends only on (op, M, K, N) and on the current device.  For
+ * QG_OP_AWQ_SEARCH, M is the calibration token count Mc. */
 size_t qg_workspace_size(qg_op op, int M, int K, int N);
 
 /* --------------------------------------------------------------------------

@@ -90,6 +90,8 @@ def _declare(L):
     L.qgo_awq_act_mean.restype = None
     L.qgo_awq_scales.argtypes = [_p, _i64, ctypes.c_double, _p, _p]
     L.qgo_awq_scales.restype = None
+    L.qgo_awq_scale_act.argtypes = [_p, _i64, _i64, _p, _p]
+    L.qgo_awq_scale_act.restype = None
     L.qgo_awq_alpha.argtypes = [_int, _int]
     L.qgo_awq_alpha.restype = ctypes.c_double
     L.qgo_awq_candidate_mse.argtypes = [_p, _i64, _i64, _p, _i64, _int, _p, _p, _p, _p]
@@ -299,6 +301,15 @@ def awq_scales(xm, alpha):
     inv = np.zeros_like(x)
     lib().qgo_awq_scales(_ptr(x), x.size, float(alpha), _ptr(s), _ptr(inv))
     return s, inv
+
+
+def awq_scale_act(X, inv_s):
+    """X~ = bf16_rn(X * inv_s) -> bf16 bit patterns u16 [M][K]."""
+    Xc = _c(X, np.float32)
+    M, K = Xc.shape
+    out = np.zeros((M, K), np.uint16)
+    lib().qgo_awq_scale_act(_ptr(Xc), M, K, _ptr(_c(inv_s, np.float32)), _ptr(out))
+    return out
 
 
 def awq_candidate_mse(X, W, s, inv_s, group=128, yref=None):

@@ -500,6 +500,13 @@ void qgo_awq_scales(const float* xm, int64_t K, double alpha, float* s, float* i
     }
 }
 
+/* X~[m][k] = bf16_rn(X[m][k] * inv_s[k]) as bf16 bit patterns (reading M) */
+void qgo_awq_scale_act(const float* X, int64_t M, int64_t K, const float* inv_s, uint16_t* xs_bf16)
+{
+    for (int64_t m = 0; m < M; ++m)
+        for (int64_t k = 0; k < K; ++k) xs_bf16[m * K + k] = qgo_f32_to_bf16_rn(X[m * K + k] * inv_s[k]);
+}
+
 /* grid point i of n (reading N) */
 double qgo_awq_alpha(int i, int n_grid) { return n_grid > 1 ? (double)i / (double)(n_grid - 1) : 0.0; }
 
@@ -529,7 +536,7 @@ int qgo_awq_candidate_mse(const float* X, int64_t M, int64_t K, const float* W, 
     if (status == OR_OK) {
         for (int64_t m = 0; m < M; ++m)
             for (int64_t k = 0; k < K; ++k) /* X~ = bf16_rn(X * inv_s) */
-                xs[m * K + k] = qgo_bf16_to_f32(qgo_f32_to_bf16_rn(X[m * K + k] * inv_s[k]));
+                xs[m * K + k] = qgo_bf16_to_f32(qgo_f32_to_bf16_rn(X[m * K + k] * inv_s[k]));  /* = qgo_awq_scale_act */
 #pragma omp parallel for schedule(static)
         for (int64_t n = 0; n < N; ++n)
             for (int64_t k = 0; k < K; ++k) {

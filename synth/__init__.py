@@ -17,6 +17,9 @@ Workloads (shapes only; no model weights are involved):
                     bf16 X ~N(0,1); W ~N(0,0.015), 0.5% entries x8.
 * ``w4a8``          X [M x 8192] bf16 ~N(0,1) with 16 fixed channels x30, M in {1,64,1024};
                     W [8192 x 8192] ~N(0,0.02); smoothing alpha = 0.5.
+* ``awq``           AWQ scale search for the decode layers' INT4 weights: calibration X
+                    [512 x 4096] bf16 ~N(0,1) with 8 fixed channels x50; W [4096 x 12288]
+                    ~N(0,0.02), 1% entries x8 (the decode weights); 21 grid points.
 
 Random streams: every draw comes from ``numpy.random.Generator(PCG64)`` seeded by
 ``SeedSequence([seed, stream, *shape])`` with one stream id per tensor role, so a
@@ -41,6 +44,8 @@ CONFIGS = {
                           outlier_frac=0.005, outlier_mult=8.0, group=128),
     "w4a8": dict(M=[1, 64, 1024], KN=[(8192, 8192)], xdtype="bf16", w_std=0.02,
                  x_channels=16, x_mult=30.0, alpha=0.5, calib_tokens=512, group=128),
+    "awq": dict(M=[512], KN=[(4096, 12288)], xdtype="bf16", w_std=0.02, outlier_frac=0.01, outlier_mult=8.0,
+                x_channels=8, x_mult=50.0, calib_tokens=512, n_grid=21, group=128),
 }
 
 

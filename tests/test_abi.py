@@ -21,7 +21,7 @@ def test_header_declares_the_boundary():
     syms = declared_symbols()
     for name in ["qg_quantize_w4_group", "qg_pack_nibbles", "qg_gemm_w4a16", "qg_smooth_quant_act_i8",
                  "qg_gemm_w8a8", "qg_gemm_w4a8", "qg_smooth_scales", "qg_quantize_w8_channel", "qg_device_status",
-                 "qg_status_string"]:
+                 "qg_status_string", "qg_awq_act_mean", "qg_awq_scales", "qg_awq_scale_act", "qg_awq_search"]:
         assert name in syms
 
 
@@ -89,6 +89,25 @@ def test_gemm_w4a16_rejects(args, want):
     ("qg_pack_nibbles", (A, 12, 16, A, None), 2),
     ("qg_pack_nibbles", (None, 16, 16, A, None), 1),
     ("qg_quantize_w8_channel", (A, None, 0, 16, A, A, None), 2),
+    ("qg_awq_act_mean", (A, 0, 16, A, None), 2),
+    ("qg_awq_act_mean", (None, 4, 16, A, None), 1),
+    ("qg_awq_act_mean", (A, 4, 16, B, None), 3),
+    ("qg_awq_scales", (A, 16, 1.5, A, A, None), 2),                            # alpha outside [0, 1]
+    ("qg_awq_scales", (A, 16, -0.1, A, A, None), 2),
+    ("qg_awq_scales", (A, 16, float("nan"), A, A, None), 2),
+    ("qg_awq_scales", (A, 16, 0.5, None, A, None), 1),
+    ("qg_awq_scale_act", (A, 4, 12, A, A, None), 2),                           # K % 8
+    ("qg_awq_scale_act", (None, 0, 16, None, None, None), 0),
+    ("qg_awq_scale_act", (A, 4, 16, B, A, None), 3),
+    # awq_search(Xcal, Mc, K, W, N, group, n_grid, mse, best, s, inv_s, ws, ws_bytes, stream)
+    ("qg_awq_search", (A, 4, 256, A, 64, 64, 5, A, A, A, A, A, 1 << 30, None), 2),   # group != 128
+    ("qg_awq_search", (A, 4, 200, A, 64, 128, 5, A, A, A, A, A, 1 << 30, None), 2),  # K % 128
+    ("qg_awq_search", (A, 4, 256, A, 60, 128, 5, A, A, A, A, A, 1 << 30, None), 2),  # N % 8
+    ("qg_awq_search", (A, 4, 256, A, 64, 128, 0, A, A, A, A, A, 1 << 30, None), 2),  # empty grid
+    ("qg_awq_search", (A, 0, 256, A, 64, 128, 5, A, A, A, A, A, 1 << 30, None), 2),  # no tokens
+    ("qg_awq_search", (A, 4, 256, A, 64, 128, 5, A, A, A, A, None, 0, None), 1),     # workspace required
+    ("qg_awq_search", (A, 4, 256, A, 64, 128, 5, A, A, A, A, A, 100, None), 10),     # workspace too small
+    ("qg_awq_search", (A, 4, 256, A, 64, 128, 5, B, A, A, A, A, 1 << 30, None), 3),
 ])
 def test_other_calls_reject(fn, args, want):
     import bit_quantized_gemm_group_b200 as q
@@ -114,6 +133,10 @@ def test_workspace_size_and_too_small_workspace():
     assert L.qg_workspace_size(2, 16, 4096, 11008) == 0    # W4A8 at 16 tokens and fewer: split-K, none
     assert L.qg_workspace_size(2, 128, 4096, 11008) == 0   # W4A8 tile kernel takes none
     assert L.qg_workspace_size(0, 0, 4096, 4096) == 0
+    # AWQ search: every buffer of one candidate, so at least codes + packed + outputs
+    K, N, Mc = 4096, 12288, 512
+    assert L.qg_workspace_size(3, Mc, K, N) >= K * N * 3 // 2 + Mc * N * 6 + Mc * K * 2
+    assert L.qg_workspace_size(3, Mc, K, 12284) == 0
     # a workspace smaller than required is refused before any launch
     assert L.qg_gemm_w4a16(A, 1, 32, 4096, 4096, A, A, A, 128, A, A, need - 1, None) == 10
     assert L.qg_gemm_w4a16(A, 1, 32, 4096, 4096, A, A, A, 128, A, B, need, None) == 3

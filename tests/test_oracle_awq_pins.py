@@ -67,6 +67,19 @@ def test_grid_points():
     assert oracle.awq_alpha(0, 1) == 0.0
 
 
+def test_scale_act_rounds_once_to_bf16():
+    import torch
+    rng = np.random.default_rng(4)
+    X = _bf16_exact(rng.standard_normal((5, 64)) * 3)
+    inv = rng.uniform(0.01, 4.0, 64).astype(np.float32)
+    inv[:8] = [0.5, 2.0, 0.25, 1.0, 4.0, 0.125, 1.0, 0.5]  # powers of two: exact scaling
+    got = oracle.awq_scale_act(X, inv)
+    prod = torch.from_numpy(X) * torch.from_numpy(inv)[None, :]  # one fp32 product (torch)
+    want = prod.to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)  # torch's RNE conversion
+    np.testing.assert_array_equal(got, want)
+    np.testing.assert_array_equal((got[:, :8].astype(np.uint32) << 16).view(np.float32), X[:, :8] * inv[:8])
+
+
 def _exact_case(seed=0, M=8, K=256, N=16):
     """X[m][c] = +-2^e_c (so mean|X_c| = 2^e_c) and W[c][n] = q[c][n] 2^-e_c with every
     group of 128 rows of every column of q spanning exactly [-7, 8]."""

@@ -28,7 +28,7 @@ MUTATIONS = [
     ("sum += fabs((double)X[m * K + c]);", "sum += (double)X[m * K + c];", [awq.test_act_mean_closed_form]),
     ("(float)pow((double)xm[c], alpha);", "(float)pow((double)xm[c], 1.0 - alpha);",
      [awq.test_scales_closed_forms, awq.test_alpha_one_is_exact_on_the_constructed_layer]),
-    ("qgo_f32_to_bf16_rn(X[m * K + k] * inv_s[k])", "qgo_f32_to_bf16_rn(X[m * K + k] * s[k])",
+    ("qgo_bf16_to_f32(qgo_f32_to_bf16_rn(X[m * K + k] * inv_s[k]))", "qgo_bf16_to_f32(qgo_f32_to_bf16_rn(X[m * K + k] * s[k]))",
      [awq.test_alpha_one_is_exact_on_the_constructed_layer]),
     ("int status = qgo_quantize_w4_asym(W, s, K, N, group, codes, sc, z);",
      "int status = qgo_quantize_w4_asym(W, inv_s, K, N, group, codes, sc, z);",
@@ -36,6 +36,8 @@ MUTATIONS = [
     ("if (status == OR_OK && mse[i] < mse[bi]) bi = i;", "if (status == OR_OK && mse[i] <= mse[bi]) bi = i;",
      [awq.test_zero_weights_tie_goes_to_the_first_point]),
     ("(double)i / (double)(n_grid - 1)", "(double)i / (double)n_grid", [awq.test_grid_points]),
+    ("xs_bf16[m * K + k] = qgo_f32_to_bf16_rn(X[m * K + k] * inv_s[k]);",
+     "xs_bf16[m * K + k] = qgo_f32_to_bf16_rn(X[m * K + k] / inv_s[k]);", [awq.test_scale_act_rounds_once_to_bf16]),
     ("double d = yref[i] - yq[i];", "double d = yref[i] - 0.5 * yq[i];", [awq.test_alpha_zero_is_the_plain_int4_layer]),
 ]
 
