@@ -464,22 +464,22 @@ void qgo_gemm_f64(const float* X, int64_t M, int64_t K, const float* W, int64_t 
 /*   sec. 2.3  s_c = mean(|X_c|)^alpha, alpha on a grid in [0, 1], chosen to    */
 /*             minimise the MSE between X W and the quantized layer's output.   */
 /* Readings (listed in the design notes):                                       */
-/*   K  the mean is a binary64 sum over the tokens in order, divided by the     */
+/*   L  the mean is a binary64 sum over the tokens in order, divided by the     */
 /*      token count in binary64 and rounded once to binary32;                   */
-/*   L  s_c = xm_c^alpha in binary64 (pow), rounded once to binary32; a channel */
+/*   M  s_c = xm_c^alpha in binary64 (pow), rounded once to binary32; a channel */
 /*      whose statistic is 0 keeps s_c = 1; inv_s_c = 1/s_c in binary32;       */
-/*   M  the quantizer Q of sec. 2.3 acts on the scaled weight s W (the method   */
+/*   N  the quantizer Q of sec. 2.3 acts on the scaled weight s W (the method   */
 /*      quantizes weights only): asymmetric INT4 groups of O1 applied to        */
 /*      diag(s) W, and the scaled activations X / s are stored in the layer's   */
 /*      activation dtype: X~ = bf16_rn(X * inv_s);                              */
-/*   N  the grid is alpha_i = i / (n_grid - 1), i = 0 .. n_grid - 1, both ends  */
+/*   O  the grid is alpha_i = i / (n_grid - 1), i = 0 .. n_grid - 1, both ends  */
 /*      included (n_grid == 1: alpha = 0 only); the MSE is the mean over all    */
 /*      M x N outputs of (X W - X~ deq(Q(s W)))^2 in binary64, both products    */
 /*      exact up to binary64 rounding; the first grid point with the least MSE  */
 /*      wins.                                                                   */
 /* ------------------------------------------------------------------------- */
 
-/* xm[c] = mean_m |X[m][c]| (reading K) */
+/* xm[c] = mean_m |X[m][c]| (reading L) */
 void qgo_awq_act_mean(const float* X, int64_t M, int64_t K, float* xm)
 {
 #pragma omp parallel for schedule(static)
@@ -490,7 +490,7 @@ void qgo_awq_act_mean(const float* X, int64_t M, int64_t K, float* xm)
     }
 }
 
-/* s[c] = xm[c]^alpha, inv_s[c] = 1 / s[c] (reading L) */
+/* s[c] = xm[c]^alpha, inv_s[c] = 1 / s[c] (reading M) */
 void qgo_awq_scales(const float* xm, int64_t K, double alpha, float* s, float* inv_s)
 {
     for (int64_t c = 0; c < K; ++c) {
@@ -500,14 +500,14 @@ void qgo_awq_scales(const float* xm, int64_t K, double alpha, float* s, float* i
     }
 }
 
-/* X~[m][k] = bf16_rn(X[m][k] * inv_s[k]) as bf16 bit patterns (reading M) */
+/* X~[m][k] = bf16_rn(X[m][k] * inv_s[k]) as bf16 bit patterns (reading N) */
 void qgo_awq_scale_act(const float* X, int64_t M, int64_t K, const float* inv_s, uint16_t* xs_bf16)
 {
     for (int64_t m = 0; m < M; ++m)
         for (int64_t k = 0; k < K; ++k) xs_bf16[m * K + k] = qgo_f32_to_bf16_rn(X[m * K + k] * inv_s[k]);
 }
 
-/* grid point i of n (reading N) */
+/* grid point i of n (reading O) */
 double qgo_awq_alpha(int i, int n_grid) { return n_grid > 1 ? (double)i / (double)(n_grid - 1) : 0.0; }
 
 /* yref[m][n] = sum_k X[m][k] W[k][n] in binary64 */
@@ -522,7 +522,7 @@ static void awq_yref(const float* X, int64_t M, int64_t K, const float* W, int64
         }
 }
 
-/* MSE of one candidate scale vector against yref (reading M, N).  Returns the
+/* MSE of one candidate scale vector against yref (readings N, O).  Returns the
  * quantizer's status; *mse is left unset unless that status is 0. */
 int qgo_awq_candidate_mse(const float* X, int64_t M, int64_t K, const float* W, int64_t N, int group,
                           const float* s, const float* inv_s, const double* yref, double* mse)
