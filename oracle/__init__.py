@@ -86,6 +86,13 @@ def _declare(L):
     L.qgo_gemm_w4a8.restype = None
     L.qgo_gemm_f64.argtypes = [_p, _i64, _i64, _p, _i64, _p, _i64, _p]
     L.qgo_gemm_f64.restype = None
+    L.qgo_outlier_count.argtypes = [_int]
+    L.qgo_outlier_count.restype = _int
+    L.qgo_outlier_split.argtypes = [_p, _p, _i64, _i64, _int, _int, _p, _p, _p, _p]
+    L.qgo_outlier_split.restype = _int
+    L.qgo_gemm_w4a16_outlier_ref.argtypes = [_p, _i64, _i64, _i64, _p, _p, _p, _int, _int, _p, _p, _p, _p, _i64,
+                                             _p, _p]
+    L.qgo_gemm_w4a16_outlier_ref.restype = None
     L.qgo_awq_act_mean.argtypes = [_p, _i64, _i64, _p]
     L.qgo_awq_act_mean.restype = None
     L.qgo_awq_scales.argtypes = [_p, _i64, ctypes.c_double, _p, _p]
@@ -274,6 +281,47 @@ def gemm_f64(X, W, rows=None):
     y = np.zeros((nr, N), np.float64)
     lib().qgo_gemm_f64(_ptr(Xc), M, K, _ptr(Wc), N, _ptr(r), nr, _ptr(y))
     return y
+
+
+# --------------------------------------------------------------------------
+# INT8 outlier side path ("LLM inference cost: W8A8/W4A8 ...", sec. 2.2, second
+# technique): the top 2% |w| of each group kept in INT8 beside the INT4 tile
+# --------------------------------------------------------------------------
+def outlier_count(group=128):
+    """Outliers per group: ceil(2% of the group size) (3 of 128)."""
+    return lib().qgo_outlier_count(int(group))
+
+
+def outlier_split(W, group=128, count=None, s_smooth=None):
+    """-> (idx u8 [G][count][N], codes8 i8 [G][count][N], s8 f32 [G][N], W_dense f32 [K][N], status)."""
+    Wc = _c(W, np.float32)
+    K, N = Wc.shape
+    count = outlier_count(group) if count is None else int(count)
+    G = K // group
+    idx = np.zeros((G, count, N), np.uint8)
+    c8 = np.zeros((G, count, N), np.int8)
+    s8 = np.zeros((G, N), np.float32)
+    dense = np.zeros((K, N), np.float32)
+    ss = None if s_smooth is None else _c(s_smooth, np.float32)
+    st = lib().qgo_outlier_split(_ptr(Wc), _ptr(ss), K, N, group, count, _ptr(idx), _ptr(c8), _ptr(s8), _ptr(dense))
+    return idx, c8, s8, dense, st
+
+
+def gemm_w4a16_outlier_ref(X, packed, scales, zeros, idx, codes8, s8, group=128, rows=None):
+    """fp64 y = X deq4 + X deq8(outliers) and its |X||W| bound for the selected rows."""
+    Xc = _c(X, np.float32)
+    M, K = Xc.shape
+    p = _c(packed, np.uint32)
+    N = p.shape[1]
+    count = idx.shape[1]
+    r, nr = _rows(rows)
+    nr = M if r is None else nr
+    y = np.zeros((nr, N), np.float64)
+    b = np.zeros((nr, N), np.float64)
+    lib().qgo_gemm_w4a16_outlier_ref(_ptr(Xc), M, K, N, _ptr(p), _ptr(_c(scales, np.uint16)), _ptr(_c(zeros, np.uint8)),
+                                     group, count, _ptr(_c(idx, np.uint8)), _ptr(_c(codes8, np.int8)),
+                                     _ptr(_c(s8, np.float32)), _ptr(r), nr, _ptr(y), _ptr(b))
+    return y, b
 
 
 # --------------------------------------------------------------------------

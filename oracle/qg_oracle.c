@@ -48,7 +48,7 @@
  * Layouts: row-major everywhere.  X[M][K], W[K][N], Y[M][N]; groups run along K.
  *
  * Status codes returned here are the oracle's own: 0 ok, 1 non-finite input,
- * 2 a scale that does not fit fp16.
+ * 2 a scale that does not fit fp16, 3 an argument out of range.
  */
 #include <math.h>
 #include <stdint.h>
@@ -58,6 +58,7 @@
 #define OR_OK 0
 #define OR_NONFINITE 1
 #define OR_RANGE 2
+#define OR_ARGS 3
 
 /* ------------------------------------------------------------------------- */
 /* binary16 and bfloat16, decoded and encoded from the IEEE 754 definitions. */
@@ -587,4 +588,97 @@ int qgo_awq_search(const float* X, int64_t M, int64_t K, const float* W, int64_t
     free(inv_s);
     free(yref);
     return status;
+}
+
+/* ------------------------------------------------------------------------- */
+/* INT8 outlier side path beside the INT4 groups.                              */
+/* "LLM inference cost: W8A8/W4A8 ...", sec. 2.2, second technique: during     */
+/* calibration the largest-magnitude 2% of each group's weights are found,      */
+/* kept in INT8 apart from the INT4 tile, and multiplied on a side path whose   */
+/* result is added to the INT4 product.                                         */
+/* Readings (listed in the design notes):                                       */
+/*   P  per (group g, column n) the outliers are the count = ceil(2% of the     */
+/*      group size) weights (3 of 128) of largest |w|, ranked by |w|            */
+/*      descending, equal |w| by smaller k; slot r holds rank r;                */
+/*   Q  they are stored as symmetric INT8 with one fp32 scale per (g, n):       */
+/*      s8 = max|outlier| / 127, code = clamp(round(w / s8), -127, 127) (ties   */
+/*      to even; s8 == 0 -> codes 0), with the k offset inside the group (u8);  */
+/*   R  the INT4 part is the asymmetric INT4 group quantization (O1) of W with   */
+/*      the outliers replaced by 0;                                             */
+/*   S  Y = X deq4(dense) + X deq8(outliers); the reference runs in binary64.   */
+/* Layouts: idx u8 [G][count][N], codes8 i8 [G][count][N], s8 fp32 [G][N].      */
+/* ------------------------------------------------------------------------- */
+
+/* count of outliers per group (reading P): ceil(0.02 * group) */
+int qgo_outlier_count(int group) { return (2 * group + 99) / 100; }
+
+/* Splits W~ (= diag(s) W, or W) into the outliers (idx, codes8, s8) and the dense
+ * remainder W_dense (fp32 [K][N], outliers set to 0).  Returns 1 on a non-finite
+ * element (that group's outputs are then unspecified). */
+int qgo_outlier_split(const float* W, const float* s_smooth, int64_t K, int64_t N, int group, int count,
+                      uint8_t* idx, int8_t* codes8, float* s8, float* W_dense)
+{
+    int64_t G = K / group;
+    int status = OR_OK;
+    if (count < 0 || count > 64 || count > group) return OR_ARGS;
+#pragma omp parallel for schedule(static) reduction(max : status)
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t g = 0; g < G; ++g) {
+            int pick[64];
+            for (int i = 0; i < group; ++i) {
+                float v = smoothed(W, s_smooth, N, g * group + i, n);
+                if (!isfinite(v)) status = OR_NONFINITE;
+                W_dense[(g * group + i) * N + n] = v;
+            }
+            /* reading P: repeated selection of the largest remaining |w|, first k on ties */
+            for (int r = 0; r < count; ++r) {
+                int best = -1;
+                float bm = -1.0f;
+                for (int i = 0; i < group; ++i) {
+                    int taken = 0;
+                    for (int j = 0; j < r; ++j) taken |= pick[j] == i;
+                    if (taken) continue;
+                    float a = fabsf(smoothed(W, s_smooth, N, g * group + i, n));
+                    if (a > bm) { bm = a; best = i; }
+                }
+                pick[r] = best;
+            }
+            /* reading Q: symmetric INT8 over the outliers of this group */
+            float amax = count > 0 ? fabsf(smoothed(W, s_smooth, N, g * group + pick[0], n)) : 0.0f;
+            float sc = amax / 127.0f;
+            s8[g * N + n] = sc;
+            for (int r = 0; r < count; ++r) {
+                float v = smoothed(W, s_smooth, N, g * group + pick[r], n);
+                int q = sc != 0.0f ? clampi((int)nearbyintf(v / sc), -127, 127) : 0;
+                idx[(g * count + r) * N + n] = (uint8_t)pick[r];
+                codes8[(g * count + r) * N + n] = (int8_t)q;
+                W_dense[(g * group + pick[r]) * N + n] = 0.0f; /* reading R */
+            }
+        }
+    }
+    return status;
+}
+
+/* y = X deq4 + X deq8 (reading S) in binary64, and bound = |X| |deq4| + |X| |deq8|,
+ * for the selected rows. */
+void qgo_gemm_w4a16_outlier_ref(const float* X, int64_t M, int64_t K, int64_t N, const uint32_t* packed,
+                                const uint16_t* scales, const uint8_t* zeros, int group, int count,
+                                const uint8_t* idx, const int8_t* codes8, const float* s8,
+                                const int64_t* rows, int64_t nrows, double* y, double* bound)
+{
+    qgo_gemm_w4a16_ref(X, M, K, N, packed, scales, zeros, group, rows, nrows, y, bound);
+    if (!rows) nrows = M;
+    int64_t G = K / group;
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t g = 0; g < G; ++g)
+            for (int r = 0; r < count; ++r) {
+                int64_t k = g * group + idx[(g * count + r) * N + n];
+                double w = (double)codes8[(g * count + r) * N + n] * (double)s8[g * N + n];
+                for (int64_t i = 0; i < nrows; ++i) {
+                    double x = (double)X[(rows ? rows[i] : i) * K + k];
+                    y[i * N + n] += x * w;
+                    bound[i * N + n] += fabs(x) * fabs(w);
+                }
+            }
 }

@@ -5,6 +5,7 @@ import pytest
 
 import oracle
 import test_oracle_awq_pins as awq
+import test_oracle_outlier_pins as outl
 import test_oracle_pins as pins
 
 MUTATIONS = [
@@ -38,6 +39,13 @@ MUTATIONS = [
     ("(double)i / (double)(n_grid - 1)", "(double)i / (double)n_grid", [awq.test_grid_points]),
     ("xs_bf16[m * K + k] = qgo_f32_to_bf16_rn(X[m * K + k] * inv_s[k]);",
      "xs_bf16[m * K + k] = qgo_f32_to_bf16_rn(X[m * K + k] / inv_s[k]);", [awq.test_scale_act_rounds_once_to_bf16]),
+    # INT8 outlier side path
+    ("if (a > bm) { bm = a; best = i; }", "if (a >= bm) { bm = a; best = i; }", [outl.test_selection_matches_a_stable_sort]),
+    ("float sc = amax / 127.0f;", "float sc = amax / 128.0f;", [outl.test_int8_codes_closed_form]),
+    ("W_dense[(g * group + pick[r]) * N + n] = 0.0f; /* reading R */", "/* outlier left in the dense part */",
+     [outl.test_dense_remainder]),
+    ("int64_t k = g * group + idx[(g * count + r) * N + n];", "int64_t k = idx[(g * count + r) * N + n];",
+     [outl.test_side_path_product_against_numpy]),
     ("double d = yref[i] - yq[i];", "double d = yref[i] - 0.5 * yq[i];", [awq.test_alpha_zero_is_the_plain_int4_layer]),
 ]
 
