@@ -511,9 +511,46 @@ def bench_configs(q, pk, int8_peak):
         out["awq_search"] = bench_awq(q, pk)
     except Exception as e:  # reported in the line, not fatal to the headline
         out["awq_search"] = {"error": repr(e)}
+    # --- INT4 + INT8 outlier side path on the decode QKV weight -----------------------
+    try:
+        out["w4a16_outlier"] = bench_outlier(q, pk, L2)
+    except Exception as e:
+        out["w4a16_outlier"] = {"error": repr(e)}
     out["int8_peak_tops_measured"] = int8_peak
     out["bf16_peak_tflops_measured"] = bf16_peak
     return out
+
+
+def bench_outlier(q, pk, L2):
+    """The decode layer 4096 x 12288 with the top 3 |w| of every group of 128 kept in INT8
+    beside the INT4 tile: the layer call (W4A16 GEMM + side path) against the plain
+    W4A16 call on the same dense part, weights rotated over copies > 2 x L2."""
+    K, N = synth.CONFIGS["w4a16_decode"]["KN"][0]
+    G, count = K // 128, 3
+    W = torch.from_numpy(synth.workload_weights("w4a16_decode", K, N)).cuda()
+    idx = torch.empty(G, count, N, dtype=torch.uint8, device="cuda")
+    c8 = torch.empty(G, count, N, dtype=torch.int8, device="cuda")
+    s8 = torch.empty(G, N, dtype=torch.float32, device="cuda")
+    dense = torch.empty_like(W)
+    q.qg_outlier_split_w4(W, None, 128, count, idx, c8, s8, dense)
+    del W
+    pw, sc, z = gpu_quant_w4(q, dense)
+    del dense
+    side_b = 2 * count * G * N + 4 * G * N
+    wb = w4_bytes(K, N) + side_b
+    rot = max(1, math.ceil(2 * L2 / wb))
+    sets = [(pw, sc, z, idx, c8, s8)] + [tuple(t.clone() for t in (pw, sc, z, idx, c8, s8)) for _ in range(rot - 1)]
+    res = {}
+    for M in (1, 16):
+        X = x_bf16("w4a16_decode", M, K)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        ms_o = time_calls(lambda i: q.qg_gemm_w4a16_outlier(X, *sets[i][:3], *sets[i][3:], Y), 16, rot)
+        ms_p = time_calls(lambda i: q.qg_gemm_w4a16(X, *sets[i][:3], Y), 16, rot)
+        by = wb + 2 * M * K + 2 * M * N + 4 * M * N  # + the side path's read-modify-write of Y
+        res[f"M={M}"] = {"us": ms_o * 1e3, "us_plain_w4a16": ms_p * 1e3, "gbs": by / (ms_o * 1e-3) / 1e9,
+                         "side_path_bytes": side_b, "roofline_frac": by / (pk["hbm_gbs"] * 1e9) / (ms_o * 1e-3)}
+    assert q.qg_device_status() == q.QG_OK
+    return res
 
 
 def bench_awq(q, pk):

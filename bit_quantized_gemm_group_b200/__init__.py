@@ -28,7 +28,8 @@ QG_OP_GEMM_W4A16, QG_OP_GEMM_W8A8, QG_OP_GEMM_W4A8, QG_OP_AWQ_SEARCH = 0, 1, 2, 
 EXPORTS = ["qg_quantize_w4_group", "qg_pack_nibbles", "qg_gemm_w4a16", "qg_smooth_quant_act_i8", "qg_gemm_w8a8",
            "qg_gemm_w4a8", "qg_smooth_scales", "qg_quantize_w8_channel", "qg_device_status", "qg_status_string",
            "qg_last_error", "qg_selftest_bounded_wait", "qg_workspace_size", "qg_gemm_w4a16_noalloc",
-           "qg_awq_act_mean", "qg_awq_scales", "qg_awq_scale_act", "qg_awq_search"]
+           "qg_awq_act_mean", "qg_awq_scales", "qg_awq_scale_act", "qg_awq_search", "qg_outlier_split_w4",
+           "qg_outlier_side_add", "qg_gemm_w4a16_outlier"]
 
 
 class QgError(RuntimeError):
@@ -51,6 +52,9 @@ _SIGS = {
     "qg_gemm_w4a8": [_P, _P, _I, _I, _P, _P, _I, _I, _P, _P, _P, _SZ, _P],
     "qg_smooth_scales": [_P, _I, _P, _I, _I, ctypes.c_float, _P, _P, _P],
     "qg_quantize_w8_channel": [_P, _P, _I, _I, _P, _P, _P],
+    "qg_outlier_split_w4": [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P],
+    "qg_outlier_side_add": [_P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P],
+    "qg_gemm_w4a16_outlier": [_P, _I, _I, _I, _I, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _SZ, _P],
     "qg_awq_act_mean": [_P, _I, _I, _P, _P],
     "qg_awq_scales": [_P, _I, ctypes.c_double, _P, _P, _P],
     "qg_awq_scale_act": [_P, _I, _I, _P, _P, _P],
@@ -201,6 +205,34 @@ def qg_quantize_w8_channel(W, s, Wq, sw, stream=None):
     K, N = W.shape
     _check(lib().qg_quantize_w8_channel(_ptr(W), _ptr(s), K, N, _ptr(Wq), _ptr(sw), _stream(stream)),
            "qg_quantize_w8_channel")
+
+
+def _xdt(X):
+    return QG_BF16 if X.dtype == torch.bfloat16 else QG_F16 if X.dtype == torch.float16 else -1
+
+
+def qg_outlier_split_w4(W, s_smooth, group, count, idx, codes8, s8, W_dense, stream=None):
+    K, N = W.shape
+    _check(lib().qg_outlier_split_w4(_ptr(W), _ptr(s_smooth), K, N, group, count, _ptr(idx), _ptr(codes8), _ptr(s8),
+                                    _ptr(W_dense), _stream(stream)), "qg_outlier_split_w4")
+
+
+def qg_outlier_side_add(X, idx, codes8, s8, Y, group=128, stream=None):
+    M, K = X.shape
+    N = Y.shape[1]
+    count = idx.shape[1]
+    _check(lib().qg_outlier_side_add(_ptr(X), _xdt(X), M, K, N, group, count, _ptr(idx), _ptr(codes8), _ptr(s8),
+                                    _ptr(Y), _stream(stream)), "qg_outlier_side_add")
+
+
+def qg_gemm_w4a16_outlier(X, packed, scales, zeros, idx, codes8, s8, Y, group=128, workspace="auto", stream=None):
+    M, K = X.shape
+    N = packed.shape[1]
+    count = idx.shape[1]
+    wp, wb = _ws(workspace, QG_OP_GEMM_W4A16, M, K, N, X.device)
+    _check(lib().qg_gemm_w4a16_outlier(_ptr(X), _xdt(X), M, K, N, _ptr(packed), _ptr(scales), _ptr(zeros), group,
+                                      count, _ptr(idx), _ptr(codes8), _ptr(s8), _ptr(Y), wp, wb, _stream(stream)),
+           "qg_gemm_w4a16_outlier")
 
 
 def qg_awq_act_mean(Xcal, xm, stream=None):

@@ -14,6 +14,7 @@
 #include "awq.cuh"
 #include "common.cuh"
 #include "int8_skinny.cuh"
+#include "outlier.cuh"
 #include "quantize.cuh"
 #include "tc_gemm.cuh"
 #include "w4a16_decode.cuh"
@@ -798,6 +799,74 @@ qg_status qg_smooth_scales(const uint16_t* Xcal, int Mc, const float* W, int K, 
     qg::smooth_finalize_kernel<<<(K + 255) / 256, 256, 0, st>>>(s, inv_s, K, alpha);
     QG_CUDA(cudaGetLastError());
     return QG_OK;
+}
+
+qg_status qg_outlier_split_w4(const float* W, const float* s_smooth, int K, int N, int group, int count,
+                              uint8_t* idx, int8_t* codes8, float* s8, float* W_dense, qg_stream_t stream)
+{
+    if (!W || !s8 || !W_dense || (count > 0 && (!idx || !codes8))) return QG_ERR_NULL;
+    if (K < 1 || N < 1 || group < 8 || group > 256 || group % 8 || K % group || count < 0 ||
+        count > qg::kMaxOutliers || count > group)
+        return QG_ERR_SHAPE;
+    if (misaligned(W) || misaligned(s_smooth) || misaligned(idx) || misaligned(codes8) || misaligned(s8) ||
+        misaligned(W_dense))
+        return QG_ERR_ALIGN;
+    const dim3 grid((N + 255) / 256, K / group), block(256);
+    qg::outlier_split_kernel<<<grid, block, 0, reinterpret_cast<cudaStream_t>(stream)>>>(W, s_smooth, K, N, group, count,
+                                                                                          idx, codes8, s8, W_dense);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+
+namespace {
+qg_status outlier_side_args(const void* X, qg_dtype xdt, int M, int K, int N, int group, int count,
+                            const uint8_t* idx, const int8_t* codes8, const float* s8, const void* Y)
+{
+    if (xdt != QG_F16 && xdt != QG_BF16) return QG_ERR_DTYPE;
+    if (M < 0 || K < 1 || N < 1 || group < 8 || group > 256 || group % 8 || K % group || count < 0 ||
+        count > qg::kMaxOutliers || count > group)
+        return QG_ERR_SHAPE;
+    if (M > 0 && count > 0 && (!X || !idx || !codes8 || !s8 || !Y)) return QG_ERR_NULL;
+    if (misaligned(X) || misaligned(idx) || misaligned(codes8) || misaligned(s8) || misaligned(Y)) return QG_ERR_ALIGN;
+    return QG_OK;
+}
+
+qg_status outlier_side_launch(const void* X, qg_dtype xdt, int M, int K, int N, int group, int count,
+                              const uint8_t* idx, const int8_t* codes8, const float* s8, void* Y, qg_stream_t stream)
+{
+    if (M == 0 || count == 0) return QG_OK;
+    constexpr int MT = 8;
+    const dim3 grid((N + 127) / 128, (M + MT - 1) / MT), block(128);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const uint16_t* x = static_cast<const uint16_t*>(X);
+    uint16_t* y = static_cast<uint16_t*>(Y);
+    if (xdt == QG_BF16)
+        qg::outlier_side_add_kernel<MT, true><<<grid, block, 0, st>>>(x, M, K, N, group, count, idx, codes8, s8, y);
+    else
+        qg::outlier_side_add_kernel<MT, false><<<grid, block, 0, st>>>(x, M, K, N, group, count, idx, codes8, s8, y);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+}  // namespace
+
+qg_status qg_outlier_side_add(const void* X, qg_dtype xdt, int M, int K, int N, int group, int count,
+                              const uint8_t* idx, const int8_t* codes8, const float* s8, void* Y, qg_stream_t stream)
+{
+    qg_status st = outlier_side_args(X, xdt, M, K, N, group, count, idx, codes8, s8, Y);
+    if (st != QG_OK) return st;
+    return outlier_side_launch(X, xdt, M, K, N, group, count, idx, codes8, s8, Y, stream);
+}
+
+qg_status qg_gemm_w4a16_outlier(const void* X, qg_dtype xdt, int M, int K, int N, const uint32_t* packed,
+                                const uint16_t* scales, const uint8_t* zeros, int group, int count,
+                                const uint8_t* idx, const int8_t* codes8, const float* s8, void* Y, void* workspace,
+                                size_t ws_bytes, qg_stream_t stream)
+{
+    qg_status st = outlier_side_args(X, xdt, M, K, N, group, count, idx, codes8, s8, Y);
+    if (st != QG_OK) return st;
+    if ((st = qg_gemm_w4a16(X, xdt, M, K, N, packed, scales, zeros, group, Y, workspace, ws_bytes, stream)) != QG_OK)
+        return st;
+    return outlier_side_launch(X, xdt, M, K, N, group, count, idx, codes8, s8, Y, stream);
 }
 
 qg_status qg_awq_act_mean(const uint16_t* Xcal, int Mc, int K, float* xm, qg_stream_t stream)

@@ -230,6 +230,43 @@ qg_status qg_quantize_w8_channel(const float* W, const float* s, int K, int N, i
                                  qg_stream_t stream);
 
 /* --------------------------------------------------------------------------
+ * INT8 outlier side path beside the INT4 groups.   [G] sec. 2.2 (second technique)
+ *
+ * Split (offline), per group g of `group` rows along K and column n of
+ * W~ = diag(s_smooth) W (or W):
+ *   the `count` elements of largest |w| (ties: smaller k first), slot r = rank r:
+ *     idx[g][r][n]    = their k offset inside the group (u8)
+ *     s8[g][n]        = max |outlier| / 127 (fp32)
+ *     codes8[g][r][n] = clamp(round(w / s8), -127, 127) (ties to even; s8 == 0 -> 0)
+ *   W_dense = W~ with those elements set to 0 (fp32 [K][N]); it then goes through
+ *   qg_quantize_w4_group (asymmetric) and qg_pack_nibbles as usual.
+ * The pages keep the top 2% of each group: count = ceil(0.02 * group) = 3 for 128.
+ * Rules: group % 8 == 0, 8 <= group <= 256, K % group == 0, 0 <= count <= 8
+ * (count == 0: idx and codes8 may be NULL; s8 is set to 0 and W_dense = W~).
+ * Device error: QG_ERR_NONFINITE (that group's outputs are then unspecified).
+ * ------------------------------------------------------------------------ */
+qg_status qg_outlier_split_w4(const float* W, const float* s_smooth, int K, int N, int group,
+                              int count, uint8_t* idx, int8_t* codes8, float* s8, float* W_dense,
+                              qg_stream_t stream);
+
+/* Side path (run time): Y[m][n] = rn(Y[m][n] + sum_{g,r} X[m][g*group + idx] * codes8 * s8),
+ * the sum in fp32 and one rounding back to the output dtype (= xdt, as for
+ * qg_gemm_w4a16).  Same rules as the split; M == 0 or count == 0 launches nothing.
+ * Device error: QG_ERR_RANGE when an idx entry is not below `group` (that entry is
+ * skipped, never read past X). */
+qg_status qg_outlier_side_add(const void* X, qg_dtype xdt, int M, int K, int N, int group,
+                              int count, const uint8_t* idx, const int8_t* codes8,
+                              const float* s8, void* Y, qg_stream_t stream);
+
+/* The layer with the side path: qg_gemm_w4a16 on the dense INT4 part, then
+ * qg_outlier_side_add.  Every argument of both is validated before either launches. */
+qg_status qg_gemm_w4a16_outlier(const void* X, qg_dtype xdt, int M, int K, int N,
+                                const uint32_t* packed, const uint16_t* scales,
+                                const uint8_t* zeros, int group, int count, const uint8_t* idx,
+                                const int8_t* codes8, const float* s8, void* Y, void* workspace,
+                                size_t ws_bytes, qg_stream_t stream);
+
+/* --------------------------------------------------------------------------
  * AWQ: activation-aware per-input-channel scales for the INT4 weights.   [A]
  *
  * Statistic (sec. 2.1):

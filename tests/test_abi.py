@@ -21,7 +21,8 @@ def test_header_declares_the_boundary():
     syms = declared_symbols()
     for name in ["qg_quantize_w4_group", "qg_pack_nibbles", "qg_gemm_w4a16", "qg_smooth_quant_act_i8",
                  "qg_gemm_w8a8", "qg_gemm_w4a8", "qg_smooth_scales", "qg_quantize_w8_channel", "qg_device_status",
-                 "qg_status_string", "qg_awq_act_mean", "qg_awq_scales", "qg_awq_scale_act", "qg_awq_search"]:
+                 "qg_status_string", "qg_awq_act_mean", "qg_awq_scales", "qg_awq_scale_act", "qg_awq_search",
+                 "qg_outlier_split_w4", "qg_outlier_side_add", "qg_gemm_w4a16_outlier"]:
         assert name in syms
 
 
@@ -89,6 +90,22 @@ def test_gemm_w4a16_rejects(args, want):
     ("qg_pack_nibbles", (A, 12, 16, A, None), 2),
     ("qg_pack_nibbles", (None, 16, 16, A, None), 1),
     ("qg_quantize_w8_channel", (A, None, 0, 16, A, A, None), 2),
+    # outlier_split_w4(W, s, K, N, group, count, idx, codes8, s8, W_dense, stream)
+    ("qg_outlier_split_w4", (A, None, 256, 64, 128, 9, A, A, A, A, None), 2),   # count above 8
+    ("qg_outlier_split_w4", (A, None, 256, 64, 128, -1, A, A, A, A, None), 2),
+    ("qg_outlier_split_w4", (A, None, 512, 64, 512, 3, A, A, A, A, None), 2),   # offsets must fit u8
+    ("qg_outlier_split_w4", (A, None, 200, 64, 128, 3, A, A, A, A, None), 2),   # K % group
+    ("qg_outlier_split_w4", (A, None, 256, 64, 128, 3, None, A, A, A, None), 1),
+    ("qg_outlier_split_w4", (A, B, 256, 64, 128, 3, A, A, A, A, None), 3),
+    # outlier_side_add(X, xdt, M, K, N, group, count, idx, codes8, s8, Y, stream)
+    ("qg_outlier_side_add", (A, 7, 4, 256, 64, 128, 3, A, A, A, A, None), 4),
+    ("qg_outlier_side_add", (A, 1, 4, 256, 64, 128, 3, A, A, None, A, None), 1),
+    ("qg_outlier_side_add", (None, 1, 0, 256, 64, 128, 3, None, None, None, None, None), 0),
+    ("qg_outlier_side_add", (A, 1, 4, 256, 64, 128, 3, A, A, A, B, None), 3),
+    # gemm_w4a16_outlier: the side-path arguments are checked before the GEMM launches
+    ("qg_gemm_w4a16_outlier", (A, 1, 4, 256, 64, A, A, A, 128, 9, A, A, A, A, None, 0, None), 2),
+    ("qg_gemm_w4a16_outlier", (A, 1, 4, 256, 64, A, A, A, 128, 3, A, A, None, A, None, 0, None), 1),
+    ("qg_gemm_w4a16_outlier", (A, 1, 4, 256, 60, A, A, A, 128, 3, A, A, A, A, None, 0, None), 2),   # GEMM's N % 8
     ("qg_awq_act_mean", (A, 0, 16, A, None), 2),
     ("qg_awq_act_mean", (None, 4, 16, A, None), 1),
     ("qg_awq_act_mean", (A, 4, 16, B, None), 3),
