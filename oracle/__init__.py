@@ -93,6 +93,10 @@ def _declare(L):
     L.qgo_gemm_w4a16_outlier_ref.argtypes = [_p, _i64, _i64, _i64, _p, _p, _p, _int, _int, _p, _p, _p, _p, _i64,
                                              _p, _p]
     L.qgo_gemm_w4a16_outlier_ref.restype = None
+    L.qgo_gptq_hessian.argtypes = [_p, _i64, _i64, ctypes.c_double, _p]
+    L.qgo_gptq_hessian.restype = None
+    L.qgo_gptq.argtypes = [_p, _i64, _i64, _p, _i64, _int, ctypes.c_double, _p, _p, _p]
+    L.qgo_gptq.restype = _int
     L.qgo_awq_act_mean.argtypes = [_p, _i64, _i64, _p]
     L.qgo_awq_act_mean.restype = None
     L.qgo_awq_scales.argtypes = [_p, _i64, ctypes.c_double, _p, _p]
@@ -322,6 +326,33 @@ def gemm_w4a16_outlier_ref(X, packed, scales, zeros, idx, codes8, s8, group=128,
                                      group, count, _ptr(_c(idx, np.uint8)), _ptr(_c(codes8, np.int8)),
                                      _ptr(_c(s8, np.float32)), _ptr(r), nr, _ptr(y), _ptr(b))
     return y, b
+
+
+# --------------------------------------------------------------------------
+# GPTQ ("Quantization & Flash Attention -- LLM inference optimization (2)", sec. 3.1-3.3):
+# rows rounded one after another, each error spread over the later rows through the
+# inverse Hessian (sequential OBS steps), stored in the asymmetric INT4 group format
+# --------------------------------------------------------------------------
+def gptq_hessian(X, damp=0.01):
+    """H = (2/n) X^T X + lambda I, lambda = damp * mean diag -> f64 [K][K]."""
+    Xc = _c(X, np.float32)
+    M, K = Xc.shape
+    H = np.zeros((K, K), np.float64)
+    lib().qgo_gptq_hessian(_ptr(Xc), M, K, float(damp), _ptr(H))
+    return H
+
+
+def gptq(X, W, group=128, damp=0.01):
+    """-> (codes u8 [K][N], scales fp16 bits [K/g][N], zeros u8 [K/g][N], status)."""
+    Xc = _c(X, np.float32)
+    Wc = _c(W, np.float32)
+    M, K = Xc.shape
+    N = Wc.shape[1]
+    codes = np.zeros((K, N), np.uint8)
+    scales = np.zeros((K // group, N), np.uint16)
+    zeros = np.zeros((K // group, N), np.uint8)
+    st = lib().qgo_gptq(_ptr(Xc), M, K, _ptr(Wc), N, group, float(damp), _ptr(codes), _ptr(scales), _ptr(zeros))
+    return codes, scales, zeros, st
 
 
 # --------------------------------------------------------------------------

@@ -682,3 +682,155 @@ void qgo_gemm_w4a16_outlier_ref(const float* X, int64_t M, int64_t K, int64_t N,
                 }
             }
 }
+
+/* ------------------------------------------------------------------------- */
+/* GPTQ: INT4 weights with Hessian-weighted error compensation.                */
+/* "Quantization & Flash Attention -- LLM inference optimization (2)",          */
+/*   sec. 3.1  the Optimal Brain Surgeon idea: when one weight is rounded, move */
+/*             the weights not yet rounded to compensate;                       */
+/*   sec. 3.2  H = (2/n) X^T X + lambda I over n calibration samples; the       */
+/*             dimensions are rounded one after another and the error of each  */
+/*             is spread over the later ones through the inverse Hessian;       */
+/*   sec. 3.3  blocks of 128 and a Cholesky factor make it fast and stable.     */
+/* Readings (listed in the design notes):                                       */
+/*   T  H is formed in binary64 with lambda = damp * mean(diag((2/n) X^T X)),   */
+/*      damp = 0.01 (the page: a small ridge); an all-zero diagonal gives       */
+/*      lambda = damp;                                                          */
+/*   U  the dimensions the page's loop walks are the input channels, i.e. the   */
+/*      rows k = 0 .. K-1 of W[K][N]; every output column n is rounded on its   */
+/*      own, with the same compensation coefficients;                           */
+/*   V  the grid is the stored INT4 format: asymmetric groups of `group` rows   */
+/*      (O1's rules); a group's scale and zero come from its compensated        */
+/*      weights, rounded to binary32, when the loop reaches the group's first   */
+/*      row, and each row's code is O1's code of its compensated binary32 value;*/
+/*   W  the update is the sequential OBS step in binary64: with Hinv the        */
+/*      inverse Hessian over the rows not yet rounded,                          */
+/*        e = (w_k - deq(q_k)) / Hinv[k][k];  w_j -= e * Hinv[k][j]  (j > k),   */
+/*      then row and column k are eliminated from Hinv.  The Cholesky form of   */
+/*      sec. 3.3 carries the same ratios Hinv[k][j] / Hinv[k][k] row by row.     */
+/* ------------------------------------------------------------------------- */
+
+/* Gauss-Jordan inverse with partial pivoting, binary64, in place on a copy.
+ * Returns 0, or 3 when the matrix is singular. */
+static int invert_f64(const double* A, int64_t n, double* inv)
+{
+    double* a = (double*)malloc(sizeof(double) * (size_t)n * n);
+    memcpy(a, A, sizeof(double) * (size_t)n * n);
+    for (int64_t i = 0; i < n; ++i)
+        for (int64_t j = 0; j < n; ++j) inv[i * n + j] = i == j ? 1.0 : 0.0;
+    int status = OR_OK;
+    for (int64_t c = 0; c < n && status == OR_OK; ++c) {
+        int64_t p = c;
+        for (int64_t r = c + 1; r < n; ++r)
+            if (fabs(a[r * n + c]) > fabs(a[p * n + c])) p = r;
+        if (a[p * n + c] == 0.0) { status = OR_ARGS; break; }
+        if (p != c)
+            for (int64_t j = 0; j < n; ++j) {
+                double t = a[c * n + j]; a[c * n + j] = a[p * n + j]; a[p * n + j] = t;
+                t = inv[c * n + j]; inv[c * n + j] = inv[p * n + j]; inv[p * n + j] = t;
+            }
+        double d = a[c * n + c];
+        for (int64_t j = 0; j < n; ++j) { a[c * n + j] /= d; inv[c * n + j] /= d; }
+        for (int64_t r = 0; r < n; ++r) {
+            if (r == c) continue;
+            double f = a[r * n + c];
+            if (f == 0.0) continue;
+            for (int64_t j = 0; j < n; ++j) { a[r * n + j] -= f * a[c * n + j]; inv[r * n + j] -= f * inv[c * n + j]; }
+        }
+    }
+    free(a);
+    return status;
+}
+
+/* H = (2/Mc) X^T X + lambda I (reading T), binary64, K x K. */
+void qgo_gptq_hessian(const float* X, int64_t Mc, int64_t K, double damp, double* H)
+{
+#pragma omp parallel for schedule(static)
+    for (int64_t a = 0; a < K; ++a)
+        for (int64_t b = 0; b < K; ++b) {
+            double s = 0.0;
+            for (int64_t m = 0; m < Mc; ++m) s += (double)X[m * K + a] * (double)X[m * K + b];
+            H[a * K + b] = 2.0 * s / (double)Mc;
+        }
+    double tr = 0.0;
+    for (int64_t a = 0; a < K; ++a) tr += H[a * K + a];
+    double lambda = tr > 0.0 ? damp * tr / (double)K : damp;
+    for (int64_t a = 0; a < K; ++a) H[a * K + a] += lambda;
+}
+
+/* O1's scale and zero of one group of binary32 values (readings A-C, J).
+ * Returns OR_RANGE when the scale does not fit fp16. */
+static int asym_scale_zero(const float* v, int group, uint16_t* s16_out, float* s_out, int* z_out)
+{
+    float mn = 0.0f, mx = 0.0f;
+    for (int i = 0; i < group; ++i) {
+        if (v[i] < mn) mn = v[i];
+        if (v[i] > mx) mx = v[i];
+    }
+    float r = mx - mn;
+    float s32 = r / 15.0f;
+    uint16_t s16 = qgo_f32_to_f16_ru(s32);
+    float s = qgo_f16_to_f32(s16);
+    int z = 0;
+    if (r == 0.0f) { s16 = 0; s = 0.0f; }
+    else z = clampi((int)nearbyintf(-mn / s), 0, 15);
+    *s16_out = s16;
+    *s_out = s;
+    *z_out = z;
+    return s32 > 65504.0f ? OR_RANGE : OR_OK;
+}
+
+/* GPTQ of W[K][N] against calibration X[Mc][K] -> O1-format codes, fp16 scales, zeros.
+ * Returns 0, 1 on a non-finite weight, 2 on a scale above fp16, 3 on a singular H. */
+int qgo_gptq(const float* X, int64_t Mc, int64_t K, const float* W, int64_t N, int group, double damp,
+             uint8_t* codes, uint16_t* scales, uint8_t* zeros)
+{
+    int64_t G = K / group;
+    double* H = (double*)malloc(sizeof(double) * (size_t)K * K);
+    double* Hinv = (double*)malloc(sizeof(double) * (size_t)K * K);
+    double* Wc = (double*)malloc(sizeof(double) * (size_t)K * N);
+    float* gv = (float*)malloc(sizeof(float) * (size_t)group);
+    float* sN = (float*)malloc(sizeof(float) * (size_t)N);
+    int* zN = (int*)malloc(sizeof(int) * (size_t)N);
+    int status = OR_OK;
+    for (int64_t i = 0; i < K * N; ++i) {
+        if (!isfinite(W[i])) status = OR_NONFINITE;
+        Wc[i] = (double)W[i];
+    }
+    qgo_gptq_hessian(X, Mc, K, damp, H);
+    if (status == OR_OK) status = invert_f64(H, K, Hinv);
+    for (int64_t k = 0; k < K && status == OR_OK; ++k) {
+        if (k % group == 0) { /* reading V: the group's scale and zero, from its compensated weights */
+            int64_t g = k / group;
+            for (int64_t n = 0; n < N; ++n) {
+                for (int i = 0; i < group; ++i) gv[i] = (float)Wc[(k + i) * N + n];
+                uint16_t s16;
+                if (asym_scale_zero(gv, group, &s16, &sN[n], &zN[n]) != OR_OK) status = OR_RANGE;
+                scales[g * N + n] = s16;
+                zeros[g * N + n] = (uint8_t)zN[n];
+            }
+        }
+        double d = Hinv[k * K + k];
+        for (int64_t n = 0; n < N; ++n) {
+            float w = (float)Wc[k * N + n];
+            float s = sN[n];
+            int z = zN[n];
+            int q = s != 0.0f ? clampi((int)nearbyintf(w / s) + z, 0, 15) : 0;
+            codes[k * N + n] = (uint8_t)q;
+            double e = (Wc[k * N + n] - (double)(q - z) * (double)s) / d; /* reading W */
+            for (int64_t j = k + 1; j < K; ++j) Wc[j * N + n] -= e * Hinv[k * K + j];
+        }
+        /* eliminate row and column k from the inverse Hessian of the remaining rows */
+        for (int64_t a = k + 1; a < K; ++a) {
+            double f = Hinv[a * K + k] / d;
+            for (int64_t b = k + 1; b < K; ++b) Hinv[a * K + b] -= f * Hinv[k * K + b];
+        }
+    }
+    free(H);
+    free(Hinv);
+    free(Wc);
+    free(gv);
+    free(sN);
+    free(zN);
+    return status;
+}

@@ -5,6 +5,7 @@ import pytest
 
 import oracle
 import test_oracle_awq_pins as awq
+import test_oracle_gptq_pins as gptq
 import test_oracle_outlier_pins as outl
 import test_oracle_pins as pins
 
@@ -46,6 +47,18 @@ MUTATIONS = [
      [outl.test_dense_remainder]),
     ("int64_t k = g * group + idx[(g * count + r) * N + n];", "int64_t k = idx[(g * count + r) * N + n];",
      [outl.test_side_path_product_against_numpy]),
+    # GPTQ
+    ("for (int64_t j = k + 1; j < K; ++j) Wc[j * N + n] -= e * Hinv[k * K + j];",
+     "for (int64_t j = k + 1; j < K; ++j) Wc[j * N + n] += e * Hinv[k * K + j];",
+     [gptq.test_cholesky_form_agrees, gptq.test_lower_layer_error_than_round_to_nearest]),
+    ("for (int64_t b = k + 1; b < K; ++b) Hinv[a * K + b] -= f * Hinv[k * K + b];",
+     "for (int64_t b = k + 1; b < K; ++b) Hinv[a * K + b] -= 0.0 * f * Hinv[k * K + b];",
+     [gptq.test_cholesky_form_agrees]),
+    ("double lambda = tr > 0.0 ? damp * tr / (double)K : damp;", "double lambda = tr > 0.0 ? damp * tr : damp;",
+     [gptq.test_hessian_hand_case]),
+    ("H[a * K + b] = 2.0 * s / (double)Mc;", "H[a * K + b] = s / (double)Mc;", [gptq.test_hessian_hand_case]),
+    ("for (int i = 0; i < group; ++i) gv[i] = (float)Wc[(k + i) * N + n];",
+     "for (int i = 0; i < group; ++i) gv[i] = W[(k + i) * N + n];", [gptq.test_cholesky_form_agrees]),
     ("double d = yref[i] - yq[i];", "double d = yref[i] - 0.5 * yq[i];", [awq.test_alpha_zero_is_the_plain_int4_layer]),
 ]
 
