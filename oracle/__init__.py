@@ -97,6 +97,8 @@ def _declare(L):
     L.qgo_gptq_hessian.restype = None
     L.qgo_gptq.argtypes = [_p, _i64, _i64, _p, _i64, _int, ctypes.c_double, _p, _p, _p]
     L.qgo_gptq.restype = _int
+    L.qgo_gptq_replay.argtypes = [_p, _i64, _i64, _p, _i64, _int, ctypes.c_double, _p, _p, _p, _int, _p, _p, _p]
+    L.qgo_gptq_replay.restype = _int
     L.qgo_awq_act_mean.argtypes = [_p, _i64, _i64, _p]
     L.qgo_awq_act_mean.restype = None
     L.qgo_awq_scales.argtypes = [_p, _i64, ctypes.c_double, _p, _p]
@@ -353,6 +355,21 @@ def gptq(X, W, group=128, damp=0.01):
     zeros = np.zeros((K // group, N), np.uint8)
     st = lib().qgo_gptq(_ptr(Xc), M, K, _ptr(Wc), N, group, float(damp), _ptr(codes), _ptr(scales), _ptr(zeros))
     return codes, scales, zeros, st
+
+
+def gptq_replay(X, W, codes, scales, zeros, group=128, damp=0.01, scale_ulps=1):
+    """Teacher-forced replay of a given GPTQ result -> (code_slack, scale_miss, zero_miss, status)."""
+    Xc = _c(X, np.float32)
+    Wc = _c(W, np.float32)
+    M, K = Xc.shape
+    N = Wc.shape[1]
+    slack = np.zeros(1, np.float64)
+    sm = np.zeros(1, np.int64)
+    zm = np.zeros(1, np.int64)
+    st = lib().qgo_gptq_replay(_ptr(Xc), M, K, _ptr(Wc), N, group, float(damp), _ptr(_c(codes, np.uint8)),
+                               _ptr(_c(scales, np.uint16)), _ptr(_c(zeros, np.uint8)), int(scale_ulps), _ptr(slack),
+                               _ptr(sm), _ptr(zm))
+    return float(slack[0]), int(sm[0]), int(zm[0]), st
 
 
 # --------------------------------------------------------------------------

@@ -834,3 +834,73 @@ int qgo_gptq(const float* X, int64_t Mc, int64_t K, const float* W, int64_t N, i
     free(zN);
     return status;
 }
+
+/* Replays a given GPTQ result (codes, fp16 scales, zeros; e.g. one made on the GPU)
+ * through the compensation of readings T-W, taking every decision from the arguments
+ * (teacher forcing), so that one rounding difference does not change the rest of the
+ * trajectory.  Reports:
+ *   *code_slack   the largest distance, in grid steps, by which a given code lies
+ *                 outside the rounding cell of its replayed value (0 when every code
+ *                 is O1's code of its replayed binary32 value);
+ *   *scale_miss   groups whose given scale differs from O1's scale of the replayed
+ *                 group by more than `scale_ulps` fp16 units in the last place;
+ *   *zero_miss    groups whose given zero differs from O1's zero by more than 1.
+ * Returns the status of qgo_gptq's Hessian step (3 on a singular H). */
+int qgo_gptq_replay(const float* X, int64_t Mc, int64_t K, const float* W, int64_t N, int group, double damp,
+                    const uint8_t* codes, const uint16_t* scales, const uint8_t* zeros, int scale_ulps,
+                    double* code_slack, int64_t* scale_miss, int64_t* zero_miss)
+{
+    double* H = (double*)malloc(sizeof(double) * (size_t)K * K);
+    double* Hinv = (double*)malloc(sizeof(double) * (size_t)K * K);
+    double* Wc = (double*)malloc(sizeof(double) * (size_t)K * N);
+    float* gv = (float*)malloc(sizeof(float) * (size_t)group);
+    for (int64_t i = 0; i < K * N; ++i) Wc[i] = (double)W[i];
+    qgo_gptq_hessian(X, Mc, K, damp, H);
+    int status = invert_f64(H, K, Hinv);
+    double slack = 0.0;
+    int64_t smiss = 0, zmiss = 0;
+    for (int64_t k = 0; k < K && status == OR_OK; ++k) {
+        int64_t g = k / group;
+        if (k % group == 0)
+            for (int64_t n = 0; n < N; ++n) {
+                for (int i = 0; i < group; ++i) gv[i] = (float)Wc[(k + i) * N + n];
+                uint16_t s16;
+                float s_ref;
+                int z_ref;
+                asym_scale_zero(gv, group, &s16, &s_ref, &z_ref);
+                if (abs((int)s16 - (int)scales[g * N + n]) > scale_ulps) ++smiss;
+                if (abs(z_ref - (int)zeros[g * N + n]) > 1) ++zmiss;
+            }
+        double d = Hinv[k * K + k];
+        for (int64_t n = 0; n < N; ++n) {
+            float s = qgo_f16_to_f32(scales[g * N + n]);
+            int z = zeros[g * N + n];
+            int q = codes[k * N + n];
+            float w = (float)Wc[k * N + n];
+            int q_ref = s != 0.0f ? clampi((int)nearbyintf(w / s) + z, 0, 15) : 0;
+            if (q != q_ref && s != 0.0f) {
+                double t = (double)w / (double)s + (double)z; /* the replayed value in grid steps */
+                double lo = q == 0 ? -INFINITY : (double)q - 0.5, hi = q == 15 ? INFINITY : (double)q + 0.5;
+                double miss = t < lo ? lo - t : (t > hi ? t - hi : 0.0);
+                if (miss > slack) slack = miss;
+                if (miss == 0.0 && slack == 0.0) slack = 1e-300; /* a tie decided the other way */
+            } else if (q != q_ref) {
+                slack = INFINITY; /* a nonzero code in an all-zero group */
+            }
+            double e = (Wc[k * N + n] - (double)(q - z) * (double)s) / d;
+            for (int64_t j = k + 1; j < K; ++j) Wc[j * N + n] -= e * Hinv[k * K + j];
+        }
+        for (int64_t a = k + 1; a < K; ++a) {
+            double f = Hinv[a * K + k] / d;
+            for (int64_t b = k + 1; b < K; ++b) Hinv[a * K + b] -= f * Hinv[k * K + b];
+        }
+    }
+    *code_slack = slack;
+    *scale_miss = smiss;
+    *zero_miss = zmiss;
+    free(H);
+    free(Hinv);
+    free(Wc);
+    free(gv);
+    return status;
+}

@@ -11,7 +11,10 @@ The page prints no worked example.  The pins:
 * the Cholesky form of sec. 3.3 (numpy: upper factor of H^-1, row ratios U[k][j]/U[k][k])
   reaching the same codes, scales and zeros as the oracle's explicit eliminations;
 * output columns rounded independently;
-* the method's claim: a lower layer error ||X (W - W_hat)||^2 than round-to-nearest.
+* the method's claim: a lower layer error ||X (W - W_hat)||^2 than round-to-nearest;
+* the teacher-forced replay (the checker for results made elsewhere, e.g. on a GPU)
+  accepts the oracle's own result and flags a code moved by one step or a scale moved by
+  more than the allowed ulps.
 They run on the CPU only.
 """
 import numpy as np
@@ -127,3 +130,19 @@ def test_lower_layer_error_than_round_to_nearest():
     e_gptq = np.sum((Xd @ (W - _deq(codes, scales, zeros, g))) ** 2)
     e_rtn = np.sum((Xd @ (W - _deq(c0, s0, z0, g))) ** 2)
     assert e_gptq < 0.7 * e_rtn
+
+
+def test_replay_accepts_its_own_result_and_flags_a_changed_code():
+    K, N, g = 256, 10, 128
+    X = _correlated(300, K, 6)
+    W = (np.random.default_rng(6).standard_normal((K, N)) * 0.02).astype(np.float32)
+    codes, scales, zeros, st = oracle.gptq(X, W, g)
+    assert oracle.gptq_replay(X, W, codes, scales, zeros, g, scale_ulps=0) == (0.0, 0, 0, 0)
+    bad = codes.copy()
+    k, n = 200, 3
+    bad[k, n] = bad[k, n] + 1 if bad[k, n] < 15 else bad[k, n] - 1  # one step off: half a step outside
+    slack, sm, zm, _ = oracle.gptq_replay(X, W, bad, scales, zeros, g, scale_ulps=0)
+    assert slack >= 0.5 - 1e-9 and sm == 0 and zm == 0
+    bad_s = scales.copy()
+    bad_s[1, 4] += 3
+    assert oracle.gptq_replay(X, W, codes, bad_s, zeros, g, scale_ulps=1)[1] >= 1
