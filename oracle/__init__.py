@@ -93,6 +93,12 @@ def _declare(L):
     L.qgo_gemm_w4a16_outlier_ref.argtypes = [_p, _i64, _i64, _i64, _p, _p, _p, _int, _int, _p, _p, _p, _p, _i64,
                                              _p, _p]
     L.qgo_gemm_w4a16_outlier_ref.restype = None
+    L.qgo_prune24.argtypes = [_p, _i64, _i64, _p, _p]
+    L.qgo_prune24.restype = None
+    L.qgo_pack24_vals.argtypes = [_p, _p, _i64, _i64, _p]
+    L.qgo_pack24_vals.restype = None
+    L.qgo_gemm_w4a16_24_ref.argtypes = [_p, _i64, _i64, _i64, _p, _p, _p, _p, _int, _p, _i64, _p, _p]
+    L.qgo_gemm_w4a16_24_ref.restype = None
     L.qgo_gptq_hessian.argtypes = [_p, _i64, _i64, ctypes.c_double, _p]
     L.qgo_gptq_hessian.restype = None
     L.qgo_gptq.argtypes = [_p, _i64, _i64, _p, _i64, _int, ctypes.c_double, _p, _p, _p]
@@ -327,6 +333,44 @@ def gemm_w4a16_outlier_ref(X, packed, scales, zeros, idx, codes8, s8, group=128,
     lib().qgo_gemm_w4a16_outlier_ref(_ptr(Xc), M, K, N, _ptr(p), _ptr(_c(scales, np.uint16)), _ptr(_c(zeros, np.uint8)),
                                      group, count, _ptr(_c(idx, np.uint8)), _ptr(_c(codes8, np.int8)),
                                      _ptr(_c(s8, np.float32)), _ptr(r), nr, _ptr(y), _ptr(b))
+    return y, b
+
+
+# --------------------------------------------------------------------------
+# 2:4 structured sparsity + INT4 ("LLM inference cost: W8A8/W4A8 ...", sec. 3.2):
+# the 2 largest |w| of every 4 along K kept, then INT4 groups of 128
+# --------------------------------------------------------------------------
+def prune24(W):
+    """-> (Wp f32 [K][N] with 2 of every 4 along K zeroed, meta u32 [K/32][N])."""
+    Wc = _c(W, np.float32)
+    K, N = Wc.shape
+    Wp = np.zeros_like(Wc)
+    meta = np.zeros((K // 32, N), np.uint32)
+    lib().qgo_prune24(_ptr(Wc), K, N, _ptr(Wp), _ptr(meta))
+    return Wp, meta
+
+
+def pack24_vals(codes, meta):
+    """Kept codes in k order, 8 per uint32 along K -> u32 [K/16][N]."""
+    c = _c(codes, np.uint8)
+    K, N = c.shape
+    vals = np.zeros((K // 16, N), np.uint32)
+    lib().qgo_pack24_vals(_ptr(c), _ptr(_c(meta, np.uint32)), K, N, _ptr(vals))
+    return vals
+
+
+def gemm_w4a16_24_ref(X, vals, meta, scales, zeros, group=128, rows=None):
+    """fp64 y = X deq(2:4 sparse INT4 W) and its |X||W| bound for the selected rows."""
+    Xc = _c(X, np.float32)
+    M, K = Xc.shape
+    v = _c(vals, np.uint32)
+    N = v.shape[1]
+    r, nr = _rows(rows)
+    nr = M if r is None else nr
+    y = np.zeros((nr, N), np.float64)
+    b = np.zeros((nr, N), np.float64)
+    lib().qgo_gemm_w4a16_24_ref(_ptr(Xc), M, K, N, _ptr(v), _ptr(_c(meta, np.uint32)), _ptr(_c(scales, np.uint16)),
+                                _ptr(_c(zeros, np.uint8)), group, _ptr(r), nr, _ptr(y), _ptr(b))
     return y, b
 
 

@@ -904,3 +904,91 @@ int qgo_gptq_replay(const float* X, int64_t Mc, int64_t K, const float* W, int64
     free(gv);
     return status;
 }
+
+/* ------------------------------------------------------------------------- */
+/* 2:4 structured sparsity + INT4.                                              */
+/* "LLM inference cost: W8A8/W4A8 ...", sec. 3.2: in every 4 weights the 2      */
+/* largest are kept (2:4, the pattern the tensor cores accelerate), then the    */
+/* kept weights are quantized to INT4 in groups of 128 with a zero point.       */
+/* Readings (listed in the design notes):                                       */
+/*   X  the 4-blocks run along K (the reduction dimension, as the hardware's    */
+/*      2:4 pattern does), k = 4b .. 4b+3 of one column; "largest" is by |w|;   */
+/*      ties go to the smaller k;                                               */
+/*   Y  the INT4 step is O1 on the pruned matrix (groups of 128 along K; with   */
+/*      reading A the pruned zeros do not change a group's range), and pruned   */
+/*      positions dequantize to exactly 0 (they are not stored);                */
+/*   Z  storage: the kept codes in k order, 8 per uint32 along K (vals          */
+/*      [K/16][N], two per 4-block); the kept positions i0 < i1 of block b as   */
+/*      the nibble (i1 << 2) | i0 at bits 4(b mod 8) of meta[b / 8][n]          */
+/*      ([K/32][N]); fp16 scales and u8 zeros as O1.                            */
+/* ------------------------------------------------------------------------- */
+
+/* Wp = W with the 2 smaller |w| of every 4-block along K set to 0; meta as reading Z.
+ * Requires K % 32 == 0. */
+void qgo_prune24(const float* W, int64_t K, int64_t N, float* Wp, uint32_t* meta)
+{
+    memset(meta, 0, sizeof(uint32_t) * (size_t)(K / 32) * N);
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t b = 0; b < K / 4; ++b) {
+            /* the two largest |w| of the block, first k on ties */
+            int keep[2] = {-1, -1};
+            for (int r = 0; r < 2; ++r) {
+                float best = -1.0f;
+                for (int i = 0; i < 4; ++i) {
+                    if (i == keep[0]) continue;
+                    float a = fabsf(W[(4 * b + i) * N + n]);
+                    if (a > best) { best = a; keep[r] = i; }
+                }
+            }
+            int i0 = keep[0] < keep[1] ? keep[0] : keep[1];
+            int i1 = keep[0] < keep[1] ? keep[1] : keep[0];
+            for (int i = 0; i < 4; ++i) {
+                float v = W[(4 * b + i) * N + n];
+                Wp[(4 * b + i) * N + n] = (i == i0 || i == i1) ? v : 0.0f;
+            }
+            meta[(b / 8) * N + n] |= (uint32_t)((i1 << 2) | i0) << (4 * (b % 8));
+        }
+}
+
+/* vals[kv/8][n] nibble kv%8 = the kv-th kept code of column n in k order (reading Z). */
+void qgo_pack24_vals(const uint8_t* codes, const uint32_t* meta, int64_t K, int64_t N, uint32_t* vals)
+{
+    memset(vals, 0, sizeof(uint32_t) * (size_t)(K / 16) * N);
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t b = 0; b < K / 4; ++b) {
+            uint32_t nib = (meta[(b / 8) * N + n] >> (4 * (b % 8))) & 0xF;
+            int pos[2] = {(int)(nib & 3), (int)(nib >> 2)};
+            for (int j = 0; j < 2; ++j) {
+                int64_t kv = 2 * b + j;
+                uint32_t c = codes[(4 * b + pos[j]) * N + n] & 0xF;
+                vals[(kv / 8) * N + n] |= c << (4 * (kv % 8));
+            }
+        }
+}
+
+/* y = X * deq(sparse W) in binary64 and its |X||W| bound, for the selected rows. */
+void qgo_gemm_w4a16_24_ref(const float* X, int64_t M, int64_t K, int64_t N, const uint32_t* vals,
+                           const uint32_t* meta, const uint16_t* scales, const uint8_t* zeros, int group,
+                           const int64_t* rows, int64_t nrows, double* y, double* bound)
+{
+    if (!rows) nrows = M;
+    memset(y, 0, sizeof(double) * nrows * N);
+    memset(bound, 0, sizeof(double) * nrows * N);
+#pragma omp parallel for schedule(static)
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t b = 0; b < K / 4; ++b) {
+            uint32_t nib = (meta[(b / 8) * N + n] >> (4 * (b % 8))) & 0xF;
+            int pos[2] = {(int)(nib & 3), (int)(nib >> 2)};
+            for (int j = 0; j < 2; ++j) {
+                int64_t k = 4 * b + pos[j], kv = 2 * b + j, g = k / group;
+                int q = (int)((vals[(kv / 8) * N + n] >> (4 * (kv % 8))) & 0xF);
+                double w = (double)(q - (int)zeros[g * N + n]) * (double)qgo_f16_to_f32(scales[g * N + n]);
+                for (int64_t r = 0; r < nrows; ++r) {
+                    double x = (double)X[(rows ? rows[r] : r) * K + k];
+                    y[r * N + n] += x * w;
+                    bound[r * N + n] += fabs(x) * fabs(w);
+                }
+            }
+        }
+}

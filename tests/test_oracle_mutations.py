@@ -8,6 +8,7 @@ import test_oracle_awq_pins as awq
 import test_oracle_gptq_pins as gptq
 import test_oracle_outlier_pins as outl
 import test_oracle_pins as pins
+import test_oracle_sparse24_pins as sp24
 
 MUTATIONS = [
     # (original text, mutated text, pins that must fail)
@@ -47,6 +48,13 @@ MUTATIONS = [
      [outl.test_dense_remainder]),
     ("int64_t k = g * group + idx[(g * count + r) * N + n];", "int64_t k = idx[(g * count + r) * N + n];",
      [outl.test_side_path_product_against_numpy]),
+    # 2:4 sparsity
+    ("if (a > best) { best = a; keep[r] = i; }", "if (a >= best) { best = a; keep[r] = i; }",
+     [sp24.test_hand_column, sp24.test_selection_matches_a_stable_sort]),
+    ("meta[(b / 8) * N + n] |= (uint32_t)((i1 << 2) | i0) << (4 * (b % 8));",
+     "meta[(b / 8) * N + n] |= (uint32_t)((i0 << 2) | i1) << (4 * (b % 8));", [sp24.test_hand_column]),
+    ("int64_t k = 4 * b + pos[j], kv = 2 * b + j, g = k / group;", "int64_t k = 4 * b + j, kv = 2 * b + j, g = k / group;",
+     [sp24.test_reference_product_against_numpy]),
     # GPTQ
     ("for (int64_t j = k + 1; j < K; ++j) Wc[j * N + n] -= e * Hinv[k * K + j];",
      "for (int64_t j = k + 1; j < K; ++j) Wc[j * N + n] += e * Hinv[k * K + j];",
