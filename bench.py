@@ -516,6 +516,11 @@ def bench_configs(q, pk, int8_peak):
         out["w4a16_outlier"] = bench_outlier(q, pk, L2)
     except Exception as e:
         out["w4a16_outlier"] = {"error": repr(e)}
+    # --- 2:4 sparse INT4 on the decode QKV weight ----------------------------------------
+    try:
+        out["w4a16_sparse24"] = bench_sparse24(q, pk, L2)
+    except Exception as e:
+        out["w4a16_sparse24"] = {"error": repr(e)}
     out["int8_peak_tops_measured"] = int8_peak
     out["bf16_peak_tflops_measured"] = bf16_peak
     return out
@@ -549,6 +554,41 @@ def bench_outlier(q, pk, L2):
         by = wb + 2 * M * K + 2 * M * N + 4 * M * N  # + the side path's read-modify-write of Y
         res[f"M={M}"] = {"us": ms_o * 1e3, "us_plain_w4a16": ms_p * 1e3, "gbs": by / (ms_o * 1e-3) / 1e9,
                          "side_path_bytes": side_b, "roofline_frac": by / (pk["hbm_gbs"] * 1e9) / (ms_o * 1e-3)}
+    assert q.qg_device_status() == q.QG_OK
+    return res
+
+
+def bench_sparse24(q, pk, L2):
+    """The decode layer 4096 x 12288 pruned 2:4 and quantized to INT4 (0.375 bytes per
+    weight with positions): the SIMT sparse GEMM at M = 1 and 16, beside the dense W4A16
+    call on the same pruned matrix, weights rotated over copies > 2 x L2."""
+    K, N = synth.CONFIGS["w4a16_decode"]["KN"][0]
+    W = torch.from_numpy(synth.workload_weights("w4a16_decode", K, N)).cuda()
+    Wp = torch.empty_like(W)
+    meta = torch.empty(K // 32, N, dtype=torch.int32, device="cuda")
+    q.qg_prune24(W, Wp, meta)
+    del W
+    codes = torch.empty(K, N, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(K // 128, N, dtype=torch.int16, device="cuda")
+    z = torch.empty(K // 128, N, dtype=torch.uint8, device="cuda")
+    q.qg_quantize_w4_group(Wp, None, 128, False, codes, sc, z)
+    vals = torch.empty(K // 16, N, dtype=torch.int32, device="cuda")
+    q.qg_pack24_vals(codes, meta, vals)
+    pw = torch.empty(K // 8, N, dtype=torch.int32, device="cuda")
+    q.qg_pack_nibbles(codes, pw)
+    del Wp, codes
+    wb = K * N * 3 // 8 + 3 * (K // 128) * N
+    rot = max(1, math.ceil(2 * L2 / wb))
+    sets = [(vals, meta, sc, z, pw)] + [tuple(t.clone() for t in (vals, meta, sc, z, pw)) for _ in range(rot - 1)]
+    res = {}
+    for M in (1, 16):
+        X = x_bf16("w4a16_decode", M, K)
+        Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        ms_s = time_calls(lambda i: q.qg_gemm_w4a16_24(X, *sets[i][:4], Y), 16, rot)
+        ms_d = time_calls(lambda i: q.qg_gemm_w4a16(X, sets[i][4], sets[i][2], sets[i][3], Y), 16, rot)
+        by = wb + 2 * M * K + 2 * M * N
+        res[f"M={M}"] = {"us": ms_s * 1e3, "us_dense_w4a16": ms_d * 1e3, "gbs": by / (ms_s * 1e-3) / 1e9,
+                         "bytes": by, "roofline_frac": by / (pk["hbm_gbs"] * 1e9) / (ms_s * 1e-3)}
     assert q.qg_device_status() == q.QG_OK
     return res
 

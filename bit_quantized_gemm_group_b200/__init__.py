@@ -29,7 +29,7 @@ EXPORTS = ["qg_quantize_w4_group", "qg_pack_nibbles", "qg_gemm_w4a16", "qg_smoot
            "qg_gemm_w4a8", "qg_smooth_scales", "qg_quantize_w8_channel", "qg_device_status", "qg_status_string",
            "qg_last_error", "qg_selftest_bounded_wait", "qg_workspace_size", "qg_gemm_w4a16_noalloc",
            "qg_awq_act_mean", "qg_awq_scales", "qg_awq_scale_act", "qg_awq_search", "qg_outlier_split_w4",
-           "qg_outlier_side_add", "qg_gemm_w4a16_outlier"]
+           "qg_outlier_side_add", "qg_gemm_w4a16_outlier", "qg_prune24", "qg_pack24_vals", "qg_gemm_w4a16_24"]
 
 
 class QgError(RuntimeError):
@@ -55,6 +55,9 @@ _SIGS = {
     "qg_outlier_split_w4": [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P],
     "qg_outlier_side_add": [_P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P],
     "qg_gemm_w4a16_outlier": [_P, _I, _I, _I, _I, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _SZ, _P],
+    "qg_prune24": [_P, _I, _I, _P, _P, _P],
+    "qg_pack24_vals": [_P, _P, _I, _I, _P, _P],
+    "qg_gemm_w4a16_24": [_P, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P, _P],
     "qg_awq_act_mean": [_P, _I, _I, _P, _P],
     "qg_awq_scales": [_P, _I, ctypes.c_double, _P, _P, _P],
     "qg_awq_scale_act": [_P, _I, _I, _P, _P, _P],
@@ -233,6 +236,23 @@ def qg_gemm_w4a16_outlier(X, packed, scales, zeros, idx, codes8, s8, Y, group=12
     _check(lib().qg_gemm_w4a16_outlier(_ptr(X), _xdt(X), M, K, N, _ptr(packed), _ptr(scales), _ptr(zeros), group,
                                       count, _ptr(idx), _ptr(codes8), _ptr(s8), _ptr(Y), wp, wb, _stream(stream)),
            "qg_gemm_w4a16_outlier")
+
+
+def qg_prune24(W, Wp, meta, stream=None):
+    K, N = W.shape
+    _check(lib().qg_prune24(_ptr(W), K, N, _ptr(Wp), _ptr(meta), _stream(stream)), "qg_prune24")
+
+
+def qg_pack24_vals(codes, meta, vals, stream=None):
+    K, N = codes.shape
+    _check(lib().qg_pack24_vals(_ptr(codes), _ptr(meta), K, N, _ptr(vals), _stream(stream)), "qg_pack24_vals")
+
+
+def qg_gemm_w4a16_24(X, vals, meta, scales, zeros, Y, group=128, stream=None):
+    M, K = X.shape
+    N = vals.shape[1]
+    _check(lib().qg_gemm_w4a16_24(_ptr(X), _xdt(X), M, K, N, _ptr(vals), _ptr(meta), _ptr(scales), _ptr(zeros), group,
+                                 _ptr(Y), _stream(stream)), "qg_gemm_w4a16_24")
 
 
 def qg_awq_act_mean(Xcal, xm, stream=None):

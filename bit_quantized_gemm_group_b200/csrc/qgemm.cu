@@ -16,6 +16,7 @@
 #include "int8_skinny.cuh"
 #include "outlier.cuh"
 #include "quantize.cuh"
+#include "sparse24.cuh"
 #include "tc_gemm.cuh"
 #include "w4a16_decode.cuh"
 #include "w4a16_tile.cuh"
@@ -867,6 +868,52 @@ qg_status qg_gemm_w4a16_outlier(const void* X, qg_dtype xdt, int M, int K, int N
     if ((st = qg_gemm_w4a16(X, xdt, M, K, N, packed, scales, zeros, group, Y, workspace, ws_bytes, stream)) != QG_OK)
         return st;
     return outlier_side_launch(X, xdt, M, K, N, group, count, idx, codes8, s8, Y, stream);
+}
+
+qg_status qg_prune24(const float* W, int K, int N, float* Wp, uint32_t* meta, qg_stream_t stream)
+{
+    if (!W || !Wp || !meta) return QG_ERR_NULL;
+    if (K < 32 || K % 32 || N < 1) return QG_ERR_SHAPE;
+    if (misaligned(W) || misaligned(Wp) || misaligned(meta)) return QG_ERR_ALIGN;
+    qg::prune24_kernel<<<dim3((N + 255) / 256, K / 32), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(W, K, N, Wp,
+                                                                                                          meta);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+
+qg_status qg_pack24_vals(const uint8_t* codes, const uint32_t* meta, int K, int N, uint32_t* vals, qg_stream_t stream)
+{
+    if (!codes || !meta || !vals) return QG_ERR_NULL;
+    if (K < 32 || K % 32 || N < 1) return QG_ERR_SHAPE;
+    if (misaligned(codes) || misaligned(meta) || misaligned(vals)) return QG_ERR_ALIGN;
+    qg::pack24_kernel<<<dim3((N + 255) / 256, K / 16), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(codes, meta, K,
+                                                                                                         N, vals);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+
+qg_status qg_gemm_w4a16_24(const void* X, qg_dtype xdt, int M, int K, int N, const uint32_t* vals,
+                           const uint32_t* meta, const uint16_t* scales, const uint8_t* zeros, int group, void* Y,
+                           qg_stream_t stream)
+{
+    if (xdt != QG_F16 && xdt != QG_BF16) return QG_ERR_DTYPE;
+    if (M < 0 || K < 128 || K % 128 || N < 1 || group != 128) return QG_ERR_SHAPE;
+    if (M == 0) return QG_OK;
+    if (!X || !vals || !meta || !scales || !zeros || !Y) return QG_ERR_NULL;
+    if (misaligned(X) || misaligned(vals) || misaligned(meta) || misaligned(scales) || misaligned(zeros) ||
+        misaligned(Y))
+        return QG_ERR_ALIGN;
+    constexpr int MT = 8;
+    const dim3 grid((N + 127) / 128, (M + MT - 1) / MT), block(128);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const uint16_t* x = static_cast<const uint16_t*>(X);
+    uint16_t* y = static_cast<uint16_t*>(Y);
+    if (xdt == QG_BF16)
+        qg::gemm_w4a16_24_kernel<MT, true><<<grid, block, 0, st>>>(x, M, K, N, vals, meta, scales, zeros, y);
+    else
+        qg::gemm_w4a16_24_kernel<MT, false><<<grid, block, 0, st>>>(x, M, K, N, vals, meta, scales, zeros, y);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
 }
 
 qg_status qg_awq_act_mean(const uint16_t* Xcal, int Mc, int K, float* xm, qg_stream_t stream)

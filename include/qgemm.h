@@ -267,6 +267,28 @@ qg_status qg_gemm_w4a16_outlier(const void* X, qg_dtype xdt, int M, int K, int N
                                 size_t ws_bytes, qg_stream_t stream);
 
 /* --------------------------------------------------------------------------
+ * 2:4 structured sparsity + INT4.   [G] sec. 3.2
+ *
+ * Prune: in every 4 consecutive rows k = 4b .. 4b+3 of a column the 2 elements of
+ *   largest |w| are kept (ties: smaller k) and the other 2 set to 0 in Wp (fp32
+ *   [K][N]); their positions i0 < i1 go to meta[b/8][n] as the nibble (i1 << 2) | i0
+ *   at bits 4 (b mod 8) (u32 [K/32][N]).  Rules: K % 32 == 0.
+ * Then: qg_quantize_w4_group(Wp, ..., symmetric = 0) as usual (the pruned zeros do
+ *   not change a group's range), and the kept codes are packed with qg_pack24_vals:
+ *   vals[kv/8][n] holds the kv-th kept code of column n (k order) at bits 4 (kv mod 8)
+ *   (u32 [K/16][N]).  Rules: K % 32 == 0.
+ * GEMM: Y = X * deq(W), pruned positions contributing exactly 0; fp32 accumulation,
+ *   Y in the activation dtype.  Rules: group == 128, K % 128 == 0.  A SIMT kernel for
+ *   few tokens (it reads 0.375 bytes per weight, positions included).
+ * ------------------------------------------------------------------------ */
+qg_status qg_prune24(const float* W, int K, int N, float* Wp, uint32_t* meta, qg_stream_t stream);
+qg_status qg_pack24_vals(const uint8_t* codes, const uint32_t* meta, int K, int N, uint32_t* vals,
+                         qg_stream_t stream);
+qg_status qg_gemm_w4a16_24(const void* X, qg_dtype xdt, int M, int K, int N, const uint32_t* vals,
+                           const uint32_t* meta, const uint16_t* scales, const uint8_t* zeros,
+                           int group, void* Y, qg_stream_t stream);
+
+/* --------------------------------------------------------------------------
  * AWQ: activation-aware per-input-channel scales for the INT4 weights.   [A]
  *
  * Statistic (sec. 2.1):

@@ -22,7 +22,8 @@ def test_header_declares_the_boundary():
     for name in ["qg_quantize_w4_group", "qg_pack_nibbles", "qg_gemm_w4a16", "qg_smooth_quant_act_i8",
                  "qg_gemm_w8a8", "qg_gemm_w4a8", "qg_smooth_scales", "qg_quantize_w8_channel", "qg_device_status",
                  "qg_status_string", "qg_awq_act_mean", "qg_awq_scales", "qg_awq_scale_act", "qg_awq_search",
-                 "qg_outlier_split_w4", "qg_outlier_side_add", "qg_gemm_w4a16_outlier"]:
+                 "qg_outlier_split_w4", "qg_outlier_side_add", "qg_gemm_w4a16_outlier", "qg_prune24",
+                 "qg_pack24_vals", "qg_gemm_w4a16_24"]:
         assert name in syms
 
 
@@ -106,6 +107,18 @@ def test_gemm_w4a16_rejects(args, want):
     ("qg_gemm_w4a16_outlier", (A, 1, 4, 256, 64, A, A, A, 128, 9, A, A, A, A, None, 0, None), 2),
     ("qg_gemm_w4a16_outlier", (A, 1, 4, 256, 64, A, A, A, 128, 3, A, A, None, A, None, 0, None), 1),
     ("qg_gemm_w4a16_outlier", (A, 1, 4, 256, 60, A, A, A, 128, 3, A, A, A, A, None, 0, None), 2),   # GEMM's N % 8
+    ("qg_prune24", (A, 48, 16, A, A, None), 2),                                # K % 32
+    ("qg_prune24", (A, 64, 16, None, A, None), 1),
+    ("qg_prune24", (A, 64, 16, A, B, None), 3),
+    ("qg_pack24_vals", (A, A, 40, 16, A, None), 2),
+    ("qg_pack24_vals", (A, None, 64, 16, A, None), 1),
+    # gemm_w4a16_24(X, xdt, M, K, N, vals, meta, scales, zeros, group, Y, stream)
+    ("qg_gemm_w4a16_24", (A, 9, 1, 256, 16, A, A, A, A, 128, A, None), 4),
+    ("qg_gemm_w4a16_24", (A, 1, 1, 192, 16, A, A, A, A, 128, A, None), 2),   # K % 128
+    ("qg_gemm_w4a16_24", (A, 1, 1, 256, 16, A, A, A, A, 64, A, None), 2),
+    ("qg_gemm_w4a16_24", (None, 1, 0, 256, 16, None, None, None, None, 128, None, None), 0),
+    ("qg_gemm_w4a16_24", (A, 1, 1, 256, 16, A, None, A, A, 128, A, None), 1),
+    ("qg_gemm_w4a16_24", (A, 1, 1, 256, 16, A, A, A, A, 128, B, None), 3),
     ("qg_awq_act_mean", (A, 0, 16, A, None), 2),
     ("qg_awq_act_mean", (None, 4, 16, A, None), 1),
     ("qg_awq_act_mean", (A, 4, 16, B, None), 3),
