@@ -710,35 +710,34 @@ void qgo_gemm_w4a16_outlier_ref(const float* X, int64_t M, int64_t K, int64_t N,
 /*      sec. 3.3 carries the same ratios Hinv[k][j] / Hinv[k][k] row by row.     */
 /* ------------------------------------------------------------------------- */
 
-/* Gauss-Jordan inverse with partial pivoting, binary64, in place on a copy.
- * Returns 0, or 3 when the matrix is singular. */
+/* Gauss-Jordan inverse in binary64.  H is symmetric positive definite (a Gram matrix
+ * plus a positive ridge), so the elimination needs no pivoting: column c is scaled by
+ * its pivot, then every other row r subtracts a[r][c] times row c (a[r][c] read before
+ * the row changes).  Each product and difference is rounded on its own.  Returns 0, or 3
+ * on a zero pivot. */
 static int invert_f64(const double* A, int64_t n, double* inv)
 {
     double* a = (double*)malloc(sizeof(double) * (size_t)n * n);
+    double* f = (double*)malloc(sizeof(double) * (size_t)n);
     memcpy(a, A, sizeof(double) * (size_t)n * n);
     for (int64_t i = 0; i < n; ++i)
         for (int64_t j = 0; j < n; ++j) inv[i * n + j] = i == j ? 1.0 : 0.0;
     int status = OR_OK;
     for (int64_t c = 0; c < n && status == OR_OK; ++c) {
-        int64_t p = c;
-        for (int64_t r = c + 1; r < n; ++r)
-            if (fabs(a[r * n + c]) > fabs(a[p * n + c])) p = r;
-        if (a[p * n + c] == 0.0) { status = OR_ARGS; break; }
-        if (p != c)
-            for (int64_t j = 0; j < n; ++j) {
-                double t = a[c * n + j]; a[c * n + j] = a[p * n + j]; a[p * n + j] = t;
-                t = inv[c * n + j]; inv[c * n + j] = inv[p * n + j]; inv[p * n + j] = t;
-            }
         double d = a[c * n + c];
+        if (d == 0.0) { status = OR_ARGS; break; }
         for (int64_t j = 0; j < n; ++j) { a[c * n + j] /= d; inv[c * n + j] /= d; }
+        for (int64_t r = 0; r < n; ++r) f[r] = a[r * n + c];
         for (int64_t r = 0; r < n; ++r) {
             if (r == c) continue;
-            double f = a[r * n + c];
-            if (f == 0.0) continue;
-            for (int64_t j = 0; j < n; ++j) { a[r * n + j] -= f * a[c * n + j]; inv[r * n + j] -= f * inv[c * n + j]; }
+            for (int64_t j = 0; j < n; ++j) {
+                a[r * n + j] -= f[r] * a[c * n + j];
+                inv[r * n + j] -= f[r] * inv[c * n + j];
+            }
         }
     }
     free(a);
+    free(f);
     return status;
 }
 
