@@ -521,6 +521,11 @@ def bench_configs(q, pk, int8_peak):
         out["w4a16_sparse24"] = bench_sparse24(q, pk, L2)
     except Exception as e:
         out["w4a16_sparse24"] = {"error": repr(e)}
+    # --- GPTQ of the decode 4096 x 4096 weight on 512 calibration tokens ------------------
+    try:
+        out["gptq"] = bench_gptq(q, pk)
+    except Exception as e:
+        out["gptq"] = {"error": repr(e)}
     out["int8_peak_tops_measured"] = int8_peak
     out["bf16_peak_tflops_measured"] = bf16_peak
     return out
@@ -591,6 +596,34 @@ def bench_sparse24(q, pk, L2):
                          "bytes": by, "roofline_frac": by / (pk["hbm_gbs"] * 1e9) / (ms_s * 1e-3)}
     assert q.qg_device_status() == q.QG_OK
     return res
+
+
+def bench_gptq(q, pk):
+    """One GPTQ call (an offline step) on the 4096 x 4096 decode weight with 512
+    calibration tokens, timed with CUDA events after one untimed call.  The roofline is
+    the HBM time of the binary64 passes it makes: the Gauss-Jordan inverse (K steps over
+    two K x K matrices) and, per row, the update of the rows below it and the elimination
+    of the inverse Hessian."""
+    K, N = 4096, 4096
+    Mc = synth.CONFIGS["awq"]["calib_tokens"]
+    W = torch.from_numpy(synth.workload_weights("w4a16_decode", K, N)).cuda()
+    _, xcb = synth.calibration(K, synth.CONFIGS["awq"])
+    Xc = torch.from_numpy(xcb.view(np.int16)).cuda().view(torch.bfloat16)
+    codes = torch.empty(K, N, dtype=torch.uint8, device="cuda")
+    sc = torch.empty(K // 128, N, dtype=torch.int16, device="cuda")
+    z = torch.empty(K // 128, N, dtype=torch.uint8, device="cuda")
+    q.qg_gptq(Xc, W, codes, sc, z)
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    q.qg_gptq(Xc, W, codes, sc, z)
+    b.record()
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    assert q.qg_device_status() == q.QG_OK
+    by = K * 2 * K * K * 16 + sum((K - k - 1) * N * 16 + (K - k - 1) ** 2 * 16 for k in range(K))
+    return {"ms": ms, "K": K, "N": N, "calib_tokens": Mc, "binary64_bytes": by,
+            "roofline_frac": by / (pk["hbm_gbs"] * 1e9) / (ms * 1e-3)}
 
 
 def bench_awq(q, pk):

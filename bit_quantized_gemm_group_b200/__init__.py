@@ -23,13 +23,14 @@ QG_OK, QG_ERR_NULL, QG_ERR_SHAPE, QG_ERR_ALIGN, QG_ERR_DTYPE = 0, 1, 2, 3, 4
 QG_ERR_NONFINITE, QG_ERR_RANGE, QG_ERR_TIMEOUT, QG_ERR_CUDA, QG_ERR_UNSUPPORTED = 5, 6, 7, 8, 9
 QG_ERR_WORKSPACE = 10
 QG_F16, QG_BF16 = 0, 1
-QG_OP_GEMM_W4A16, QG_OP_GEMM_W8A8, QG_OP_GEMM_W4A8, QG_OP_AWQ_SEARCH = 0, 1, 2, 3
+QG_OP_GEMM_W4A16, QG_OP_GEMM_W8A8, QG_OP_GEMM_W4A8, QG_OP_AWQ_SEARCH, QG_OP_GPTQ = 0, 1, 2, 3, 4
 
 EXPORTS = ["qg_quantize_w4_group", "qg_pack_nibbles", "qg_gemm_w4a16", "qg_smooth_quant_act_i8", "qg_gemm_w8a8",
            "qg_gemm_w4a8", "qg_smooth_scales", "qg_quantize_w8_channel", "qg_device_status", "qg_status_string",
            "qg_last_error", "qg_selftest_bounded_wait", "qg_workspace_size", "qg_gemm_w4a16_noalloc",
            "qg_awq_act_mean", "qg_awq_scales", "qg_awq_scale_act", "qg_awq_search", "qg_outlier_split_w4",
-           "qg_outlier_side_add", "qg_gemm_w4a16_outlier", "qg_prune24", "qg_pack24_vals", "qg_gemm_w4a16_24"]
+           "qg_outlier_side_add", "qg_gemm_w4a16_outlier", "qg_prune24", "qg_pack24_vals", "qg_gemm_w4a16_24",
+           "qg_gptq"]
 
 
 class QgError(RuntimeError):
@@ -55,6 +56,7 @@ _SIGS = {
     "qg_outlier_split_w4": [_P, _P, _I, _I, _I, _I, _P, _P, _P, _P, _P],
     "qg_outlier_side_add": [_P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P],
     "qg_gemm_w4a16_outlier": [_P, _I, _I, _I, _I, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _SZ, _P],
+    "qg_gptq": [_P, _I, _I, _P, _I, _I, ctypes.c_double, _P, _P, _P, _P, _SZ, _P],
     "qg_prune24": [_P, _I, _I, _P, _P, _P],
     "qg_pack24_vals": [_P, _P, _I, _I, _P, _P],
     "qg_gemm_w4a16_24": [_P, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P, _P],
@@ -236,6 +238,14 @@ def qg_gemm_w4a16_outlier(X, packed, scales, zeros, idx, codes8, s8, Y, group=12
     _check(lib().qg_gemm_w4a16_outlier(_ptr(X), _xdt(X), M, K, N, _ptr(packed), _ptr(scales), _ptr(zeros), group,
                                       count, _ptr(idx), _ptr(codes8), _ptr(s8), _ptr(Y), wp, wb, _stream(stream)),
            "qg_gemm_w4a16_outlier")
+
+
+def qg_gptq(Xcal, W, codes, scales, zeros, group=128, damp=0.01, workspace="auto", stream=None):
+    Mc, K = Xcal.shape
+    N = W.shape[1]
+    wp, wb = _ws(workspace, QG_OP_GPTQ, Mc, K, N, Xcal.device)
+    _check(lib().qg_gptq(_ptr(Xcal), Mc, K, _ptr(W), N, group, float(damp), _ptr(codes), _ptr(scales), _ptr(zeros), wp,
+                        wb, _stream(stream)), "qg_gptq")
 
 
 def qg_prune24(W, Wp, meta, stream=None):

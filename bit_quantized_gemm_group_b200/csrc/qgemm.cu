@@ -12,6 +12,7 @@
 #include "../../include/qgemm.h"
 #include "act_quant.cuh"
 #include "awq.cuh"
+#include "gptq.cuh"
 #include "common.cuh"
 #include "int8_skinny.cuh"
 #include "outlier.cuh"
@@ -551,6 +552,35 @@ AwqWs awq_carve(void* base, int Mc, int K, int N)
     return w;
 }
 
+// GPTQ workspace: the Gauss-Jordan matrix, the inverse Hessian, the pivot column, the
+// compensated weights (binary64) and the per-column row state
+struct GptqWs {
+    double *a, *inv, *f, *wc, *e;
+    float* s_col;
+    int* z_col;
+    size_t bytes;
+};
+
+GptqWs gptq_carve(void* base, int K, int N)
+{
+    GptqWs w{};
+    size_t off = 0;
+    auto take = [&](size_t b) {
+        const size_t o = off;
+        off += (b + 255) & ~size_t(255);
+        return base ? static_cast<uint8_t*>(base) + o : nullptr;
+    };
+    w.a = reinterpret_cast<double*>(take(8 * (size_t)K * K));
+    w.inv = reinterpret_cast<double*>(take(8 * (size_t)K * K));
+    w.f = reinterpret_cast<double*>(take(8 * (size_t)K));
+    w.wc = reinterpret_cast<double*>(take(8 * (size_t)K * N));
+    w.e = reinterpret_cast<double*>(take(8 * (size_t)N));
+    w.s_col = reinterpret_cast<float*>(take(4 * (size_t)N));
+    w.z_col = reinterpret_cast<int*>(take(4 * (size_t)N));
+    w.bytes = off;
+    return w;
+}
+
 // ---------------------------------------------------------------------------
 // int8 skinny paths
 // ---------------------------------------------------------------------------
@@ -624,6 +654,10 @@ size_t qg_workspace_size(qg_op op, int M, int K, int N)
         case QG_OP_GEMM_W8A8: {
             if (M >= qg::kTcMinM || N % 16) return 0;
             return i8_plan(M, K, N).partial_bytes;
+        }
+        case QG_OP_GPTQ: {
+            if (K > 16384) return 0;
+            return gptq_carve(nullptr, K, N).bytes;
         }
         case QG_OP_AWQ_SEARCH: {
             if (N % 8) return 0;
@@ -912,6 +946,52 @@ qg_status qg_gemm_w4a16_24(const void* X, qg_dtype xdt, int M, int K, int N, con
         qg::gemm_w4a16_24_kernel<MT, true><<<grid, block, 0, st>>>(x, M, K, N, vals, meta, scales, zeros, y);
     else
         qg::gemm_w4a16_24_kernel<MT, false><<<grid, block, 0, st>>>(x, M, K, N, vals, meta, scales, zeros, y);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+
+qg_status qg_gptq(const uint16_t* Xcal, int Mc, int K, const float* W, int N, int group, double damp,
+                  uint8_t* codes, uint16_t* scales, uint8_t* zeros, void* workspace, size_t ws_bytes,
+                  qg_stream_t stream)
+{
+    if (!Xcal || !W || !codes || !scales || !zeros || !workspace) return QG_ERR_NULL;
+    if (Mc < 1 || K < 8 || K > 16384 || N < 1 || group < 8 || group > 1024 || group % 8 || K % group ||
+        !(damp > 0.0 && damp < 1e30))
+        return QG_ERR_SHAPE;
+    if (misaligned(Xcal) || misaligned(W) || misaligned(codes) || misaligned(scales) || misaligned(zeros) ||
+        misaligned(workspace))
+        return QG_ERR_ALIGN;
+    if (ws_bytes < gptq_carve(nullptr, K, N).bytes) return QG_ERR_WORKSPACE;
+    const GptqWs w = gptq_carve(workspace, K, N);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    const int kb = (K + 255) / 256, nb = (N + 255) / 256;
+    // H, then its inverse by Gauss-Jordan (w.a is destroyed, w.inv receives H^-1)
+    qg::gptq_hessian_kernel<<<dim3(kb, K), 256, 0, st>>>(Xcal, Mc, K, w.a);
+    QG_CUDA(cudaGetLastError());
+    qg::gptq_ridge_kernel<<<1, 32, 0, st>>>(w.a, K, damp);
+    QG_CUDA(cudaGetLastError());
+    qg::gptq_identity_kernel<<<dim3(kb, K), 256, 0, st>>>(w.inv, K);
+    QG_CUDA(cudaGetLastError());
+    for (int c = 0; c < K; ++c) {
+        qg::gj_column_kernel<<<kb, 256, 0, st>>>(w.a, K, c, w.f);
+        qg::gj_scale_kernel<<<kb, 256, 0, st>>>(w.a, w.inv, K, c, w.f);
+        qg::gj_eliminate_kernel<<<dim3(kb, K), 256, 0, st>>>(w.a, w.inv, K, c, w.f);
+    }
+    QG_CUDA(cudaGetLastError());
+    // the rows, in order
+    const int64_t total = (int64_t)K * N;
+    qg::gptq_load_kernel<<<(int)std::min<int64_t>((total + 255) / 256, 8 * num_sms()), 256, 0, st>>>(W, total, w.wc);
+    QG_CUDA(cudaGetLastError());
+    for (int k = 0; k < K; ++k) {
+        if (k % group == 0)
+            qg::gptq_group_kernel<<<nb, 256, 0, st>>>(w.wc, N, k, group, scales, zeros, w.s_col, w.z_col);
+        qg::gptq_row_kernel<<<nb, 256, 0, st>>>(w.wc, K, N, k, w.inv, w.s_col, w.z_col, codes, w.e);
+        const int rest = K - k - 1;
+        if (rest > 0) {
+            qg::gptq_update_kernel<<<dim3(nb, rest), 256, 0, st>>>(w.wc, K, N, k, w.inv, w.e);
+            qg::gptq_eliminate_kernel<<<dim3((rest + 255) / 256, rest), 256, 0, st>>>(w.inv, K, k);
+        }
+    }
     QG_CUDA(cudaGetLastError());
     return QG_OK;
 }

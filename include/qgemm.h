@@ -69,7 +69,13 @@ typedef enum {
 } qg_status;
 
 /* Operations that may use a caller-provided workspace (qg_workspace_size). */
-typedef enum { QG_OP_GEMM_W4A16 = 0, QG_OP_GEMM_W8A8 = 1, QG_OP_GEMM_W4A8 = 2, QG_OP_AWQ_SEARCH = 3 } qg_op;
+typedef enum {
+    QG_OP_GEMM_W4A16 = 0,
+    QG_OP_GEMM_W8A8 = 1,
+    QG_OP_GEMM_W4A8 = 2,
+    QG_OP_AWQ_SEARCH = 3,
+    QG_OP_GPTQ = 4
+} qg_op;
 
 typedef enum { QG_F16 = 0, QG_BF16 = 1 } qg_dtype;
 
@@ -287,6 +293,31 @@ qg_status qg_pack24_vals(const uint8_t* codes, const uint32_t* meta, int K, int 
 qg_status qg_gemm_w4a16_24(const void* X, qg_dtype xdt, int M, int K, int N, const uint32_t* vals,
                            const uint32_t* meta, const uint16_t* scales, const uint8_t* zeros,
                            int group, void* Y, qg_stream_t stream);
+
+/* --------------------------------------------------------------------------
+ * GPTQ: INT4 weights with Hessian-weighted error compensation.   [A] sec. 3.1-3.3
+ *
+ *   H = (2/Mc) Xcal^T Xcal + lambda I, lambda = damp * trace / K (damp if the trace
+ *   is 0), in binary64; H^-1 by Gauss-Jordan (no pivoting: H is positive definite).
+ *   Rows k = 0 .. K-1 of W in order: at a group's first row the group's scale and
+ *   zero (the asymmetric rules of qg_quantize_w4_group) from its compensated weights
+ *   rounded to fp32; codes[k][n] = clamp(round(w / s) + z, 0, 15) on the compensated
+ *   fp32 value; e = (w - (q - z) s) / H^-1[k][k]; w_j -= e H^-1[k][j] for j > k; then
+ *   row and column k are eliminated from H^-1.  Every operation is one IEEE rounding
+ *   in that order, so the results are reproducible bit for bit.
+ * Xcal bf16 [Mc][K]; W fp32 [K][N]; codes u8 [K][N]; scales fp16 bits [K/group][N];
+ * zeros u8 [K/group][N] (then qg_pack_nibbles and qg_gemm_w4a16 as usual).
+ * Rules: Mc >= 1, 8 <= group <= 1024, group % 8 == 0, K % group == 0, K <= 16384,
+ *   0 < damp (0.01 is the usual ridge).
+ * workspace (required): at least qg_workspace_size(QG_OP_GPTQ, Mc, K, N) bytes
+ *   (2 K^2 + K N doubles and a few vectors), contents irrelevant.
+ * Device errors: QG_ERR_NONFINITE (a non-finite weight), QG_ERR_RANGE (a scale above
+ *   fp16, or a zero pivot).  An offline step: about 7 K kernel launches and
+ *   O(K^3 + K^2 N) binary64 operations.
+ * ------------------------------------------------------------------------ */
+qg_status qg_gptq(const uint16_t* Xcal, int Mc, int K, const float* W, int N, int group,
+                  double damp, uint8_t* codes, uint16_t* scales, uint8_t* zeros, void* workspace,
+                  size_t ws_bytes, qg_stream_t stream);
 
 /* --------------------------------------------------------------------------
  * AWQ: activation-aware per-input-channel scales for the INT4 weights.   [A]

@@ -23,7 +23,7 @@ def test_header_declares_the_boundary():
                  "qg_gemm_w8a8", "qg_gemm_w4a8", "qg_smooth_scales", "qg_quantize_w8_channel", "qg_device_status",
                  "qg_status_string", "qg_awq_act_mean", "qg_awq_scales", "qg_awq_scale_act", "qg_awq_search",
                  "qg_outlier_split_w4", "qg_outlier_side_add", "qg_gemm_w4a16_outlier", "qg_prune24",
-                 "qg_pack24_vals", "qg_gemm_w4a16_24"]:
+                 "qg_pack24_vals", "qg_gemm_w4a16_24", "qg_gptq"]:
         assert name in syms
 
 
@@ -107,6 +107,14 @@ def test_gemm_w4a16_rejects(args, want):
     ("qg_gemm_w4a16_outlier", (A, 1, 4, 256, 64, A, A, A, 128, 9, A, A, A, A, None, 0, None), 2),
     ("qg_gemm_w4a16_outlier", (A, 1, 4, 256, 64, A, A, A, 128, 3, A, A, None, A, None, 0, None), 1),
     ("qg_gemm_w4a16_outlier", (A, 1, 4, 256, 60, A, A, A, 128, 3, A, A, A, A, None, 0, None), 2),   # GEMM's N % 8
+    # gptq(Xcal, Mc, K, W, N, group, damp, codes, scales, zeros, ws, ws_bytes, stream)
+    ("qg_gptq", (A, 16, 256, A, 64, 100, 0.01, A, A, A, A, 1 << 40, None), 2),    # group % 8
+    ("qg_gptq", (A, 16, 200, A, 64, 128, 0.01, A, A, A, A, 1 << 40, None), 2),    # K % group
+    ("qg_gptq", (A, 16, 256, A, 64, 128, 0.0, A, A, A, A, 1 << 40, None), 2),     # damp must be > 0
+    ("qg_gptq", (A, 0, 256, A, 64, 128, 0.01, A, A, A, A, 1 << 40, None), 2),
+    ("qg_gptq", (A, 16, 256, A, 64, 128, 0.01, A, A, A, None, 0, None), 1),       # workspace required
+    ("qg_gptq", (A, 16, 256, A, 64, 128, 0.01, A, A, A, A, 1000, None), 10),      # too small
+    ("qg_gptq", (A, 16, 256, A, 64, 128, 0.01, A, B, A, A, 1 << 40, None), 3),
     ("qg_prune24", (A, 48, 16, A, A, None), 2),                                # K % 32
     ("qg_prune24", (A, 64, 16, None, A, None), 1),
     ("qg_prune24", (A, 64, 16, A, B, None), 3),
