@@ -645,6 +645,10 @@ const char* qg_last_error(void) { return g_last_error; }
 
 size_t qg_workspace_size(qg_op op, int M, int K, int N)
 {
+    if (op == QG_OP_GPTQ) {  // any K that a group size divides (K % 8 == 0), any N
+        if (M < 1 || K < 8 || K % 8 || K > 16384 || N < 1) return 0;
+        return gptq_carve(nullptr, K, N).bytes;
+    }
     if (M < 1 || K < 128 || N < 8 || K % 128) return 0;
     switch (op) {
         case QG_OP_GEMM_W4A16: {
@@ -654,10 +658,6 @@ size_t qg_workspace_size(qg_op op, int M, int K, int N)
         case QG_OP_GEMM_W8A8: {
             if (M >= qg::kTcMinM || N % 16) return 0;
             return i8_plan(M, K, N).partial_bytes;
-        }
-        case QG_OP_GPTQ: {
-            if (K > 16384) return 0;
-            return gptq_carve(nullptr, K, N).bytes;
         }
         case QG_OP_AWQ_SEARCH: {
             if (N % 8) return 0;

@@ -175,6 +175,10 @@ def test_workspace_size_and_too_small_workspace():
     K, N, Mc = 4096, 12288, 512
     assert L.qg_workspace_size(3, Mc, K, N) >= K * N * 3 // 2 + Mc * N * 6 + Mc * K * 2
     assert L.qg_workspace_size(3, Mc, K, 12284) == 0
+    # GPTQ: two K x K binary64 matrices and the binary64 weights, for any K a group divides
+    assert L.qg_workspace_size(4, 16, 96, 5) >= 8 * (2 * 96 * 96 + 96 * 5)
+    assert L.qg_workspace_size(4, 16, 100, 5) == 0
+    assert L.qg_workspace_size(4, 16, 32768, 5) == 0
     # a workspace smaller than required is refused before any launch
     assert L.qg_gemm_w4a16(A, 1, 32, 4096, 4096, A, A, A, 128, A, A, need - 1, None) == 10
     assert L.qg_gemm_w4a16(A, 1, 32, 4096, 4096, A, A, A, 128, A, B, need, None) == 3
