@@ -739,7 +739,9 @@ def main():
 
     clocks = ClockSampler(local)
     clocks.start()
+    torch.cuda.nvtx.range_push("decode sweep: timed steps")  # NVTX range for profilers (ncu --nvtx)
     ms = time_graphs(graphs, args.steps, args.warmup, world)
+    torch.cuda.nvtx.range_pop()
     ck = clocks.stop()
     ms = max_over_ranks(ms, world)
     ms_step = ms / args.steps
@@ -751,7 +753,9 @@ def main():
         if rank == 0:
             print(json.dumps({"profile_run": True, "ms_per_step": ms_step, "gbs": achieved}), flush=True)
         return
+    torch.cuda.nvtx.range_push("decode sweep: end to end")
     e2e_ms, h2d, d2h = e2e_decode(sweep, args.steps, args.warmup, world)
+    torch.cuda.nvtx.range_pop()
     e2e_val = whole_job_gbs(by, world, args.steps, e2e_ms)
     calls = per_call_times(sweep) if rank == 0 else []
 
@@ -762,7 +766,9 @@ def main():
     if rank == 0 and not args.skip_configs:
         cs = ClockSampler(local)
         cs.start()
+        torch.cuda.nvtx.range_push("other workloads")
         configs = bench_configs(q, pk, measure_int8_peak())
+        torch.cuda.nvtx.range_pop()
         configs["clocks"] = cs.stop()
 
     if rank == 0:
