@@ -506,6 +506,11 @@ def bench_configs(q, pk, int8_peak):
             del X, Y
         del pw, sc, z
     out["w4a16_prefill"] = res
+    # --- offline single-pass kernels: quantizers, packing, smoothing -------------------
+    try:
+        out["offline"] = bench_offline(q, pk)
+    except Exception as e:
+        out["offline"] = {"error": repr(e)}
     # --- AWQ scale search: 512 calibration tokens, the decode QKV weight, 21 grid points --
     try:
         out["awq_search"] = bench_awq(q, pk)
@@ -529,6 +534,45 @@ def bench_configs(q, pk, int8_peak):
     out["int8_peak_tops_measured"] = int8_peak
     out["bf16_peak_tflops_measured"] = bf16_peak
     return out
+
+
+def bench_offline(q, pk):
+    """The single-pass offline kernels on the decode QKV weight (4096 x 12288, fp32):
+    asymmetric and symmetric INT4 group quantization, nibble packing, SmoothQuant factors
+    (512 calibration tokens) and per-channel INT8 quantization, each against the HBM time
+    of its algorithmic bytes (its input read once, its outputs written once)."""
+    K, N = synth.CONFIGS["w4a16_decode"]["KN"][0]
+    G = K // 128
+    W = torch.from_numpy(synth.workload_weights("w4a16_decode", K, N)).cuda()
+    _, xcb = synth.calibration(K, synth.CONFIGS["w8a8"])
+    Xc = torch.from_numpy(xcb.view(np.int16)).cuda().view(torch.bfloat16)
+    Mc = Xc.shape[0]
+    codes = torch.empty(K, N, dtype=torch.uint8, device="cuda")
+    sc16 = torch.empty(G, N, dtype=torch.int16, device="cuda")
+    zeros = torch.empty(G, N, dtype=torch.uint8, device="cuda")
+    sc32 = torch.empty(G, N, dtype=torch.float32, device="cuda")
+    packed = torch.empty(K // 8, N, dtype=torch.int32, device="cuda")
+    s = torch.empty(K, dtype=torch.float32, device="cuda")
+    inv = torch.empty_like(s)
+    Wq = torch.empty(K, N, dtype=torch.int8, device="cuda")
+    sw = torch.empty(N, dtype=torch.float32, device="cuda")
+    runs = {
+        "quantize_w4_asym": (lambda i: q.qg_quantize_w4_group(W, None, 128, False, codes, sc16, zeros),
+                             4 * K * N + K * N + 3 * G * N),
+        "quantize_w4_sym": (lambda i: q.qg_quantize_w4_group(W, None, 128, True, codes, sc32, None),
+                            4 * K * N + K * N + 4 * G * N),
+        "pack_nibbles": (lambda i: q.qg_pack_nibbles(codes, packed), K * N + K * N // 2),
+        "smooth_scales": (lambda i: q.qg_smooth_scales(Xc, W, 0.5, s, inv), 2 * Mc * K + 4 * K * N + 8 * K),
+        "quantize_w8_channel": (lambda i: q.qg_quantize_w8_channel(W, s, Wq, sw), 4 * K * N + 4 * K + K * N + 4 * N),
+    }
+    res = {}
+    for name, (fn, by) in runs.items():
+        ms = time_calls(fn, 4)
+        res[name] = {"us": ms * 1e3, "gbs": by / (ms * 1e-3) / 1e9, "bytes": by,
+                     "roofline_frac": by / (pk["hbm_gbs"] * 1e9) / (ms * 1e-3)}
+    assert q.qg_device_status() == q.QG_OK
+    res["shape"] = {"K": K, "N": N, "calib_tokens": Mc}
+    return res
 
 
 def bench_outlier(q, pk, L2):
