@@ -334,6 +334,52 @@ def cpu_baseline_decode(min_seconds=10.0, col_frac=1, max_reps=20):
                        f"({by / 1e6:.1f} MB algorithmic), fp64 reference GEMM with OpenMP, {dt:.2f} s"), dt
 
 
+def cpu_oracle_rows():
+    """The oracle, as it stands, timed beside each of the other workloads on a bounded
+    sample (the unit of each sample is stated; the GPU figures are in the same `configs`)."""
+    import oracle
+    cores = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
+
+    def timed(fn):
+        t0 = time.perf_counter()
+        fn()
+        return time.perf_counter() - t0
+
+    out = {"cores": cores, "kind": "oracle"}
+    rng = np.random.default_rng(0)
+    # W8A8 GEMM, 16 tokens of the 4096 x 11008 layer
+    Xq = rng.integers(-127, 128, (16, 4096)).astype(np.int8)
+    Wq = rng.integers(-127, 128, (4096, 11008)).astype(np.int8)
+    dt = timed(lambda: oracle.gemm_w8a8(Xq, np.ones(16, np.float32), Wq, np.ones(11008, np.float32)))
+    out["w8a8_m16"] = {"s": dt, "tops": 2 * 16 * 4096 * 11008 / dt / 1e12}
+    # W4A8 GEMM, 1 token of the 8192 x 8192 layer
+    p = oracle.pack_nibbles(rng.integers(-7, 8, (8192, 8192)).astype(np.int8))
+    sg = np.full((64, 8192), 0.01, np.float32)
+    dt = timed(lambda: oracle.gemm_w4a8(rng.integers(-127, 128, (1, 8192)).astype(np.int8), np.ones(1, np.float32),
+                                        p, sg))
+    out["w4a8_m1"] = {"s": dt, "gbs": (8192 * 8192 // 2 + 4 * 64 * 8192) / dt / 1e9}
+    # W4A16 prefill: 2 tokens x K = 8192 x 4096 columns, weights drawn like the prefill layer's
+    Wp = synth.weights(8192, 4096, 0.015, 0.005, 8.0)
+    c, sc, z, _ = oracle.quantize_w4_asym(Wp)
+    pk_ = oracle.pack_nibbles(c)
+    X2, _ = synth.activations(2, 8192, "bf16")
+    dt = timed(lambda: oracle.gemm_w4a16_ref(X2, pk_, sc, z))
+    out["w4a16_prefill_2tok_4096col"] = {"s": dt, "tflops": 2 * 2 * 8192 * 4096 / dt / 1e12}
+    # the INT4 quantizer on the 4096 x 12288 decode weight
+    Wd = synth.workload_weights("w4a16_decode", 4096, 12288)
+    dt = timed(lambda: oracle.quantize_w4_asym(Wd))
+    out["quantize_w4_asym"] = {"s": dt, "gbs": (5 * 4096 * 12288) / dt / 1e9}
+    # AWQ: 8 calibration tokens, 3 grid points, the 4096 x 12288 layer
+    Xc, _ = synth.calibration(4096, synth.CONFIGS["awq"])
+    dt = timed(lambda: oracle.awq_search(Xc[:8].copy(), Wd, 3))
+    out["awq_search_8tok_3pts"] = {"s": dt}
+    # GPTQ of a 512 x 512 weight on 256 tokens
+    Xg, _ = synth.activations(256, 512, "bf16")
+    dt = timed(lambda: oracle.gptq(Xg, Wd[:512, :512].copy()))
+    out["gptq_512x512"] = {"s": dt}
+    return out
+
+
 def run_reference(args, world, rank):
     """--impl reference: the CPU oracle timed on a bounded sample of the workload."""
     if rank != 0:
@@ -806,6 +852,10 @@ def main():
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu, _ = cpu_baseline_decode()
+        try:
+            cpu["other_workloads"] = cpu_oracle_rows()
+        except Exception as e:  # reported, not fatal
+            cpu["other_workloads"] = {"error": repr(e)}
     configs = None
     if rank == 0 and not args.skip_configs:
         cs = ClockSampler(local)
