@@ -61,7 +61,9 @@ typedef enum {
     QG_ERR_ALIGN = 3,       /* a base pointer is not 16-byte aligned */
     QG_ERR_DTYPE = 4,       /* unknown dtype enumerator */
     QG_ERR_NONFINITE = 5,   /* (device) an input that must be finite was NaN or Inf */
-    QG_ERR_RANGE = 6,       /* (device) an fp16 scale would overflow */
+    QG_ERR_RANGE = 6,       /* (device) a value outside its allowed range: an fp16 scale
+                               that would overflow, an outlier offset outside its group,
+                               a zero pivot in the GPTQ inverse */
     QG_ERR_TIMEOUT = 7,     /* (device) a bounded wait inside a kernel gave up */
     QG_ERR_CUDA = 8,        /* the CUDA runtime reported an error; see qg_last_error() */
     QG_ERR_UNSUPPORTED = 9, /* the device is not sm_100 or a feature is missing */
