@@ -188,3 +188,20 @@ def test_workspace_size_and_too_small_workspace():
     need4 = L.qg_workspace_size(2, 32, 4096, 11008)
     assert L.qg_gemm_w4a8(A, A, 32, 4096, A, A, 11008, 128, A, None, A, need4 - 1, None) == 10
     assert L.qg_gemm_w4a8(A, A, 32, 4096, A, A, 11008, 128, A, None, B, need4, None) == 3
+
+
+@pytest.mark.skipif(__import__("torch").cuda.is_available(),
+                    reason="needs a host without a usable GPU: the call below launches with fake pointers")
+def test_host_side_cuda_failure_is_reported():
+    """A CUDA runtime failure on the host (here: no usable device) comes back as
+    QG_ERR_CUDA with the failing call and the runtime's message, and the binding's
+    exception carries that text."""
+    import bit_quantized_gemm_group_b200 as q
+    L = q.lib()
+    assert L.qg_pack_nibbles(A, 16, 16, A, None) == q.QG_ERR_CUDA
+    msg = L.qg_last_error().decode()
+    assert "cudaGetLastError" in msg and len(msg) > len("cudaGetLastError(): ")
+    assert L.qg_device_status(None) == q.QG_ERR_CUDA
+    assert "cudaStreamSynchronize" in L.qg_last_error().decode()
+    err = q.QgError(q.QG_ERR_CUDA, "qg_device_status")
+    assert "QG_ERR_CUDA" in str(err) and "cudaStreamSynchronize" in str(err)
