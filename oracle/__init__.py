@@ -82,7 +82,7 @@ def _declare(L):
     L.qgo_quantize_w8_channel.restype = _int
     L.qgo_gemm_w8a8.argtypes = [_p, _p, _i64, _i64, _p, _p, _i64, _p, _i64, _p, _p, _p, _p]
     L.qgo_gemm_w8a8.restype = None
-    L.qgo_gemm_w4a8.argtypes = [_p, _p, _i64, _i64, _p, _p, _i64, _int, _p, _i64, _p, _p, _p]
+    L.qgo_gemm_w4a8.argtypes = [_p, _p, _i64, _i64, _p, _p, _i64, _int, _p, _i64, _p, _p, _p, _p]
     L.qgo_gemm_w4a8.restype = None
     L.qgo_gemm_f64.argtypes = [_p, _i64, _i64, _p, _i64, _p, _i64, _p]
     L.qgo_gemm_f64.restype = None
@@ -267,8 +267,10 @@ def gemm_w8a8(Xq, t, Wq, sw, rows=None):
     return acc, y, yref, b
 
 
-def gemm_w4a8(Xq, t, packed, sg, group=128, rows=None, want_part=True):
-    """-> (part i32 [rows][K/g][N] or None, yref f64, bound f64) for the selected rows."""
+def gemm_w4a8(Xq, t, packed, sg, group=128, rows=None, want_part=True, want_y=False):
+    """-> (part i32 [rows][K/g][N] or None, yref f64, bound f64) for the selected rows;
+    with want_y also the output bf16 bits as the workload defines it (binary32 group
+    products summed in ascending group order, times t, rounded once)."""
     Xq = _c(Xq, np.int8)
     M, K = Xq.shape
     p = _c(packed, np.uint32)
@@ -278,8 +280,11 @@ def gemm_w4a8(Xq, t, packed, sg, group=128, rows=None, want_part=True):
     part = np.zeros((nr, K // group, N), np.int32) if want_part else None
     yref = np.zeros((nr, N), np.float64)
     b = np.zeros((nr, N), np.float64)
+    y = np.zeros((nr, N), np.uint16) if want_y else None
     lib().qgo_gemm_w4a8(_ptr(Xq), _ptr(_c(t, np.float32)), M, K, _ptr(p), _ptr(_c(sg, np.float32)), N, group,
-                        _ptr(r), nr, _ptr(part), _ptr(yref), _ptr(b))
+                        _ptr(r), nr, _ptr(part), _ptr(yref), _ptr(b), _ptr(y))
+    if want_y:
+        return part, yref, b, y
     return part, yref, b
 
 

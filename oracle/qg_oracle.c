@@ -23,7 +23,7 @@
  *   W4A8                  4-bit weights, 8-bit activations, group-wise
  *       "LLM inference cost: W8A8/W4A8 ...", sec. 2.2
  *
- * Readings where the pages are silent (each one is listed in the design notes):
+ * Readings where the pages are silent, each taken as stated here:
  *   A  the asymmetric range is widened to include 0: mn' = min(min V, 0),
  *      mx' = max(max V, 0), so that z lies in [0,15] and 0 is exact;
  *   B  the 4-bit asymmetric scale divides by 15 = 2^4 - 1 (the page's 255 is 2^8 - 1);
@@ -409,10 +409,15 @@ void qgo_gemm_w8a8(const int8_t* Xq, const float* t, int64_t M, int64_t K, const
 /* two's-complement nibbles); Y = t_m * sum_g P * s_gn.  The reference is the  */
 /* fp64 dot of (qx*t_m)(qw4*s_gn) and its absolute-value bound.                */
 /* part is [nrows][K/group][N] or NULL.                                        */
+/* y_bf16 (nullable) is the output as the workload defines it ("int32 per-     */
+/* group partial sums scaled by the group scale in fp32; bf16 out", "LLM       */
+/* inference cost: W8A8/W4A8 ...", sec. 2.2): in binary32, each partial       */
+/* converted and multiplied by its group scale, the products summed over g in  */
+/* ascending order, the sum multiplied by t_m, then rounded once to bf16.      */
 /* ------------------------------------------------------------------------- */
 void qgo_gemm_w4a8(const int8_t* Xq, const float* t, int64_t M, int64_t K, const uint32_t* packed,
                    const float* sg, int64_t N, int group, const int64_t* rows, int64_t nrows,
-                   int32_t* part, double* yref, double* bound)
+                   int32_t* part, double* yref, double* bound, uint16_t* y_bf16)
 {
     if (!rows) nrows = M;
     int64_t G = K / group;
@@ -421,6 +426,7 @@ void qgo_gemm_w4a8(const int8_t* Xq, const float* t, int64_t M, int64_t K, const
         for (int64_t r = 0; r < nrows; ++r) {
             int64_t m = rows ? rows[r] : r;
             double y = 0.0, b = 0.0;
+            float acc = 0.0f;
             for (int64_t g = 0; g < G; ++g) {
                 int64_t p = 0;
                 for (int i = 0; i < group; ++i) {
@@ -434,7 +440,12 @@ void qgo_gemm_w4a8(const int8_t* Xq, const float* t, int64_t M, int64_t K, const
                     b += fabs(xd) * fabs(wd);
                 }
                 if (part) part[(r * G + g) * N + n] = (int32_t)p;
+                {
+                    volatile float prod = (float)p * sg[g * N + n]; /* one binary32 rounding */
+                    acc = acc + prod;
+                }
             }
+            if (y_bf16) y_bf16[r * N + n] = qgo_f32_to_bf16_rn(acc * t[m]);
             yref[r * N + n] = y;
             bound[r * N + n] = b;
         }
@@ -464,7 +475,7 @@ void qgo_gemm_f64(const float* X, int64_t M, int64_t K, const float* W, int64_t 
 /*   sec. 2.2  the equivalent transform X W = (X / s)(s W), s per input channel;*/
 /*   sec. 2.3  s_c = mean(|X_c|)^alpha, alpha on a grid in [0, 1], chosen to    */
 /*             minimise the MSE between X W and the quantized layer's output.   */
-/* Readings (listed in the design notes):                                       */
+/* Readings where the page is silent, each taken as stated here:              */
 /*   L  the mean is a binary64 sum over the tokens in order, divided by the     */
 /*      token count in binary64 and rounded once to binary32;                   */
 /*   M  s_c = xm_c^alpha in binary64 (pow), rounded once to binary32; a channel */
@@ -596,7 +607,7 @@ int qgo_awq_search(const float* X, int64_t M, int64_t K, const float* W, int64_t
 /* calibration the largest-magnitude 2% of each group's weights are found,      */
 /* kept in INT8 apart from the INT4 tile, and multiplied on a side path whose   */
 /* result is added to the INT4 product.                                         */
-/* Readings (listed in the design notes):                                       */
+/* Readings where the page is silent, each taken as stated here:              */
 /*   P  per (group g, column n) the outliers are the count = ceil(2% of the     */
 /*      group size) weights (3 of 128) of largest |w|, ranked by |w|            */
 /*      descending, equal |w| by smaller k; slot r holds rank r;                */
@@ -692,7 +703,7 @@ void qgo_gemm_w4a16_outlier_ref(const float* X, int64_t M, int64_t K, int64_t N,
 /*             dimensions are rounded one after another and the error of each  */
 /*             is spread over the later ones through the inverse Hessian;       */
 /*   sec. 3.3  blocks of 128 and a Cholesky factor make it fast and stable.     */
-/* Readings (listed in the design notes):                                       */
+/* Readings where the page is silent, each taken as stated here:              */
 /*   T  H is formed in binary64 with lambda = damp * mean(diag((2/n) X^T X)),   */
 /*      damp = 0.01 (the page: a small ridge); an all-zero diagonal gives       */
 /*      lambda = damp;                                                          */
@@ -909,7 +920,7 @@ int qgo_gptq_replay(const float* X, int64_t Mc, int64_t K, const float* W, int64
 /* "LLM inference cost: W8A8/W4A8 ...", sec. 3.2: in every 4 weights the 2      */
 /* largest are kept (2:4, the pattern the tensor cores accelerate), then the    */
 /* kept weights are quantized to INT4 in groups of 128 with a zero point.       */
-/* Readings (listed in the design notes):                                       */
+/* Readings where the page is silent, each taken as stated here:              */
 /*   X  the 4-blocks run along K (the reduction dimension, as the hardware's    */
 /*      2:4 pattern does), k = 4b .. 4b+3 of one column; "largest" is by |w|;   */
 /*      ties go to the smaller k;                                               */

@@ -25,6 +25,11 @@ MUTATIONS = [
      [pins.test_w4a16_ref_reduces_to_integer_matmul]),
     ("sj = sqrtf(ax) / sqrtf(aw);", "sj = sqrtf(aw) / sqrtf(ax);", [pins.test_smooth_half_alpha_equalises_ranges]),
     ("int qw = v >= 8 ? v - 16 : v;", "int qw = v;", [pins.test_w4a8_partials_and_reference]),
+    # W4A8 output: binary64 accumulation instead of binary32, and t applied twice
+    ("float acc = 0.0f;", "double acc = 0.0;",
+     [pins.test_w4a8_output_sums_groups_in_ascending_order_in_binary32]),
+    ("qgo_f32_to_bf16_rn(acc * t[m]);", "qgo_f32_to_bf16_rn(acc * t[m] * t[m]);",
+     [pins.test_w4a8_output_exact_case_is_rounded_integer_product]),
     ("float tm = a / 127.0f;", "float tm = a / 128.0f;", [pins.test_act_i8_closed_form_and_brute_force]),
     ("float s = amax / 7.0f;", "float s = amax / 8.0f;", [pins.test_w4_sym_absmax_bound_brute_force]),
     # AWQ search

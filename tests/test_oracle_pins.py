@@ -443,6 +443,69 @@ def test_w4a8_partials_and_reference():
     np.testing.assert_allclose(b, np.abs(xd) @ np.abs(wd), rtol=1e-12)
 
 
+def _bf16_bits_of_f64(v):
+    # f64 -> f32 is exact for the values used here; then torch's RNE conversion to bf16
+    return torch.from_numpy(np.asarray(v, np.float32)).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+
+
+def test_w4a8_output_exact_case_is_rounded_integer_product():
+    """Power-of-two group and token scales with small integer codes make every binary32
+    product and partial sum of the W4A8 output exact, so the output must be the exact
+    product (numpy's int64 matmul per group, scaled) rounded once to bf16."""
+    rng = np.random.default_rng(12)
+    M, K, N = 5, 8192, 24
+    Xq = rng.integers(-31, 32, (M, K)).astype(np.int8)
+    q = rng.integers(-7, 8, (K, N)).astype(np.int8)
+    e = rng.integers(-2, 1, (K // 128, N))
+    sg = (2.0 ** e).astype(np.float32)
+    t = (2.0 ** rng.integers(-9, -5, M)).astype(np.float32)
+    packed = oracle.pack_nibbles(q)
+    _, yref, _, y = oracle.gemm_w4a8(Xq, t, packed, sg, want_part=False, want_y=True)
+    exact = np.zeros((M, N))
+    for g in range(K // 128):
+        sl = slice(128 * g, 128 * (g + 1))
+        exact += (Xq[:, sl].astype(np.int64) @ q[sl].astype(np.int64)) * 2.0 ** e[g]
+    exact *= t.astype(np.float64)[:, None]
+    np.testing.assert_array_equal(yref, exact)
+    np.testing.assert_array_equal(y, _bf16_bits_of_f64(exact))
+
+
+def test_w4a8_output_sums_groups_in_ascending_order_in_binary32():
+    """Hand example: three groups whose scaled partials are 2^24, 1 and -2^24.  In
+    binary32 and ascending group order, 2^24 + 1 rounds to 2^24 (tie to even) and the
+    output is exactly 0; any other order, or a binary64 sum, gives 1."""
+    K, N = 384, 1
+    Xq = np.zeros((1, K), np.int8)
+    q = np.zeros((K, N), np.int8)
+    Xq[0, 0:128] = 64
+    q[0:128, 0] = 2             # P0 = 128 * 64 * 2 = 16384
+    Xq[0, 128] = 1
+    q[128, 0] = 1               # P1 = 1
+    Xq[0, 256:384] = 64
+    q[256:384, 0] = -2          # P2 = -16384
+    sg = np.array([[1024.0], [1.0], [1024.0]], np.float32)
+    t = np.ones(1, np.float32)
+    part, yref, _, y = oracle.gemm_w4a8(Xq, t, oracle.pack_nibbles(q), sg, want_y=True)
+    np.testing.assert_array_equal(part[0, :, 0], [16384, 1, -16384])
+    assert yref[0, 0] == 1.0
+    assert int(y[0, 0]) == 0x0000
+
+
+def test_w4a8_output_within_tolerance_of_reference():
+    rng = np.random.default_rng(13)
+    M, K, N = 6, 1024, 64
+    Xq = rng.integers(-127, 128, (M, K)).astype(np.int8)
+    q = rng.integers(-7, 8, (K, N)).astype(np.int8)
+    sg = rng.uniform(0.001, 0.01, (K // 128, N)).astype(np.float32)
+    t = rng.uniform(0.01, 1.0, M).astype(np.float32)
+    _, yref, b, y = oracle.gemm_w4a8(Xq, t, oracle.pack_nibbles(q), sg, want_part=False, want_y=True)
+    yv = (y.astype(np.uint32) << 16).view(np.float32)
+    assert oracle.within_tolerance(yv, yref, b).all()
+    # one bf16 rounding of a binary32 sum: within 2^-8 relative of the fp64 value, plus the
+    # binary32 summation error, far inside the tolerance
+    assert (np.abs(yv - yref) <= 2.0 ** -8 * np.abs(yref) + 1e-4 * b).all()
+
+
 def test_f64_gemm_matches_numpy():
     X, _ = synth.activations(3, 128, "bf16", seed=1)
     W = synth.weights(128, 20, 0.02, seed=1)
