@@ -8,6 +8,7 @@
 #include <string.h>
 
 #include <algorithm>
+#include <atomic>
 
 #include "../../include/qgemm.h"
 #include "act_quant.cuh"
@@ -43,25 +44,39 @@ qg_status cuda_fail(cudaError_t e, const char* where)
 
 bool misaligned(const void* p) { return p && (reinterpret_cast<uintptr_t>(p) & 15u); }
 
+// Per-device host caches (SM count, kernel occupancy, the no-alloc array's address)
+// hold one slot per device index below kMaxDevices.  Slots are atomics: several host
+// threads may make their first call on a device at once, and each then computes and
+// stores the same value.  A device index beyond the slots is served without caching.
 constexpr int kMaxDevices = 64;
 
-int current_device()
+// The calling thread's current device; QG_ERR_CUDA with the runtime's message when
+// it cannot be determined.
+qg_status current_device(int* dev)
 {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    return dev >= 0 && dev < kMaxDevices ? dev : 0;
+    const cudaError_t e = cudaGetDevice(dev);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+    return QG_OK;
 }
 
+bool cached_slot(int dev) { return dev >= 0 && dev < kMaxDevices; }
+
+// SM count of the current device (148 on a B200).  Launch plans and workspace sizes
+// are both derived from it, so a query failure here (reported again by the launch
+// that follows) only changes the plan, never its consistency.
 int num_sms()
 {
-    static int cache[kMaxDevices] = {0};
-    const int dev = current_device();
-    if (cache[dev] == 0) {
-        int n = 0;
-        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-        cache[dev] = n > 0 ? n : 148;
+    static std::atomic<int> cache[kMaxDevices];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cached_slot(dev)) {
+        const int c = cache[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
     }
-    return cache[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    if (cached_slot(dev)) cache[dev].store(n, std::memory_order_relaxed);
+    return n;
 }
 
 // Launch `kern` with a thread-block cluster of (1, cy, 1).
@@ -105,23 +120,31 @@ int choose_split(int nslabs, int groups, int ctas_per_sm)
 }
 
 // Per kernel instance and device: raise the dynamic shared memory limit once and
-// remember the occupancy, so that a launch makes no query calls after the first.
+// remember the occupancy, so that a launch makes no query calls after the first.  The
+// occupancy is stored (release) only after the attribute is set, so a thread that
+// reads it (acquire) launches with the attribute in place.
 struct KernelInfo {
-    int occ[kMaxDevices] = {0};
+    std::atomic<int> occ[kMaxDevices];
 };
 
 template <typename Kern>
 qg_status prepare_kernel(KernelInfo& info, Kern k, int threads, size_t smem, int* occ)
 {
-    const int dev = current_device();
-    if (info.occ[dev] == 0) {
-        if (smem > 48 * 1024)
-            QG_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
-        int n = 0;
-        QG_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, smem));
-        info.occ[dev] = n > 0 ? n : 1;
+    int dev = 0;
+    qg_status st = current_device(&dev);
+    if (st != QG_OK) return st;
+    if (cached_slot(dev)) {
+        const int c = info.occ[dev].load(std::memory_order_acquire);
+        if (c > 0) {
+            *occ = c;
+            return QG_OK;
+        }
     }
-    *occ = info.occ[dev];
+    if (smem > 48 * 1024) QG_CUDA(cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem));
+    int n = 0;
+    QG_CUDA(cudaOccupancyMaxActiveBlocksPerMultiprocessor(&n, k, threads, smem));
+    *occ = n > 0 ? n : 1;
+    if (cached_slot(dev)) info.occ[dev].store(*occ, std::memory_order_release);
     return QG_OK;
 }
 
@@ -1125,19 +1148,27 @@ static __device__ __align__(256) unsigned char qg_noalloc_scratch[kNoAllocScratc
 
 // Device address of the array, per device.  In host code the array's name is only a
 // host-side stand-in, so the address must come from cudaGetSymbolAddress, called
-// with the device current.
-void* g_noalloc_addr[kMaxDevices] = {nullptr};
+// with the device current.  Cached per device slot (atomic: first calls from several
+// host threads store the same address); a device beyond the slots queries each time.
+std::atomic<void*> g_noalloc_addr[kMaxDevices];
 
 qg_status noalloc_scratch(void** out)
 {
-    const int dev = current_device();
-    if (!g_noalloc_addr[dev]) {
-        void* ptr = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&ptr, qg_noalloc_scratch);
-        if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(qg_noalloc_scratch)");
-        g_noalloc_addr[dev] = ptr;
+    int dev = 0;
+    qg_status st = current_device(&dev);
+    if (st != QG_OK) return st;
+    if (cached_slot(dev)) {
+        void* p = g_noalloc_addr[dev].load(std::memory_order_acquire);
+        if (p) {
+            *out = p;
+            return QG_OK;
+        }
     }
-    *out = g_noalloc_addr[dev];
+    void* ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, qg_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(qg_noalloc_scratch)");
+    if (cached_slot(dev)) g_noalloc_addr[dev].store(ptr, std::memory_order_release);
+    *out = ptr;
     return QG_OK;
 }
 

@@ -21,6 +21,11 @@ Workloads (shapes only; no model weights are involved):
                     [512 x 4096] bf16 ~N(0,1) with 8 fixed channels x50; W [4096 x 12288]
                     ~N(0,0.02), 1% entries x8 (the decode weights); 21 grid points.
 
+Exact-arithmetic operands (``exact_*``): quantized operands drawn directly -- INT4 codes,
+zero points, power-of-two scales and small integer activations -- on which every
+product and partial sum of the GEMMs is exact in binary32 (the bounds are stated per
+function), so any correct kernel returns the exact product rounded once.
+
 Random streams: every draw comes from ``numpy.random.Generator(PCG64)`` seeded by
 ``SeedSequence([seed, stream, *shape])`` with one stream id per tensor role, so a
 tensor does not change when another one is added.  The outlier channels of X are a
@@ -31,7 +36,7 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-S_W, S_X, S_XCAL, S_MASK, S_CHANNELS = 1, 2, 3, 4, 5
+S_W, S_X, S_XCAL, S_MASK, S_CHANNELS, S_EXACT = 1, 2, 3, 4, 5, 6
 
 CONFIGS = {
     "w4a16_tiny": dict(M=[1], KN=[(1024, 1024)], xdtype="f16", w_std=0.02,
@@ -100,3 +105,45 @@ def workload_weights(name: str, K: int, N: int, seed: int = 0) -> np.ndarray:
 def workload_activations(name: str, M: int, K: int, seed: int = 0):
     cfg = CONFIGS[name]
     return activations(M, K, cfg["xdtype"], cfg.get("x_channels", 0), cfg.get("x_mult", 1.0), seed)
+
+
+# ---------------------------------------------------------------------------
+# exact-arithmetic operands
+# ---------------------------------------------------------------------------
+def exact_w4_asym(K: int, N: int, group: int = 128, e_min: int = -2, seed: int = 0):
+    """Asymmetric INT4 operands drawn directly: codes u8 in [0, 15], zero points u8 in
+    [0, 15], scales 2^e with e in [e_min, 0] as fp16 bit patterns [K/group][N].
+    Every (q - z) * 2^e is exact in bf16 and fp16."""
+    r = rng(seed, S_EXACT, 1, K, N)
+    codes = r.integers(0, 16, (K, N)).astype(np.uint8)
+    zeros = r.integers(0, 16, (K // group, N)).astype(np.uint8)
+    e = r.integers(e_min, 1, (K // group, N))
+    scales = np.asarray(2.0 ** e, np.float16).view(np.uint16).copy()
+    return codes, scales, zeros
+
+
+def exact_w4_sym(K: int, N: int, group: int = 128, e_min: int = -2, seed: int = 0):
+    """Symmetric INT4 operands drawn directly: codes int8 in [-7, 7], fp32 scales 2^e
+    with e in [e_min, 0], [K/group][N]."""
+    r = rng(seed, S_EXACT, 2, K, N)
+    codes = r.integers(-7, 8, (K, N)).astype(np.int8)
+    e = r.integers(e_min, 1, (K // group, N))
+    return codes, (2.0 ** e).astype(np.float32)
+
+
+def exact_activations(M: int, K: int, xmax: int = 8, dtype: str = "bf16", seed: int = 0):
+    """Integer activations in [-xmax, xmax] (exact in bf16 and fp16).
+    Returns (values as fp32, raw 16-bit patterns) like ``activations``."""
+    X = rng(seed, S_EXACT, 3, M, K).integers(-xmax, xmax + 1, (M, K)).astype(np.float32)
+    t = torch.from_numpy(X)
+    t16 = t.to(torch.bfloat16) if dtype == "bf16" else t.to(torch.float16)
+    return X, t16.view(torch.int16).numpy().view(np.uint16).copy()
+
+
+def exact_act_i8(M: int, K: int, qmax: int = 31, seed: int = 0):
+    """INT8 activation codes in [-qmax, qmax] with power-of-two token scales 2^f,
+    f in [-9, -6]."""
+    r = rng(seed, S_EXACT, 4, M, K)
+    Xq = r.integers(-qmax, qmax + 1, (M, K)).astype(np.int8)
+    t = (2.0 ** r.integers(-9, -5, M)).astype(np.float32)
+    return Xq, t

@@ -355,11 +355,16 @@ def test_nonfinite_weights_reported():
 
 
 # ---------------------------------------------------------------------------
-# prefill W4A16 at full size, sampled rows (oracle cost bounded)
+# prefill W4A16 at full size: every 64th row plus the first and the last, across all N
+# (every 256-token tile of the tile kernel is visited four times; oracle cost bounded)
 # ---------------------------------------------------------------------------
+def rows_every_64(M):
+    return np.array(sorted(set(range(0, M, 64)) | {0, M - 1}), np.int64)
+
+
 @pytest.mark.parametrize("K,N", synth.CONFIGS["w4a16_prefill"]["KN"])
 def test_gemm_w4a16_prefill_sampled(K, N):
-    _w4a16_case(K, N, "w4a16_prefill", [4096, 8192], "bf16", rows=lambda M: sample_rows(M, extra=3))
+    _w4a16_case(K, N, "w4a16_prefill", [4096, 8192], "bf16", rows=rows_every_64)
 
 
 # ---------------------------------------------------------------------------
