@@ -46,7 +46,7 @@ CONFIG = {"workload": "w4a16_decode: M in {1,4,16,32} x (K,N) in {(4096,12288),(
                       "(4096,22016),(11008,4096)}, group-128 asym INT4, bf16 X/Y",
           "l2": "every call reads its own weight copy; a shape's copies total > 2x L2, so no call "
                 "finds its weights in L2",
-          "launch": "one CUDA graph per step (16 calls, each a decode and a fixup kernel)"}
+          "launch": "one CUDA graph per step (16 calls, one decode kernel launch each)"}
 # DRAM bytes (read + write) of one decode launch over its algorithmic bytes, from an ncu
 # capture of one w4a16_decode_kernel launch at K=4096, N=22016, M=1 (47.237 MB read +
 # 0.016 MB written against 47.255 MB algorithmic; the weight stream is read exactly once,
@@ -213,9 +213,9 @@ class DecodeSweep:
         return sum(2 * c["M"] * sh["K"] * sh["N"] for sh, c in self.calls())
 
     def launches_per_step(self):
-        # every decode call is two kernels: w4a16_decode_kernel and its fixup (all sweep
-        # shapes have N % 16 == 0, the workspace path)
-        return 2 * sum(1 for _ in self.calls())
+        # every decode call (M <= 32, N % 16 == 0, the workspace path) is one launch of
+        # w4a16_decode_kernel: split column slabs are finished inside the kernel
+        return sum(1 for _ in self.calls())
 
     def copy_for(self, sh, s, ci):
         """Weight copy of call ci of shape sh in rotation step s: every call of a step
@@ -937,7 +937,7 @@ def main():
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "traffic": by * DECODE_TRAFFIC_RATIO,
                          "traffic_unit": "bytes per step", "peak_source": pk["source"],
-                         "kernel": "w4a16_decode_kernel + w4a16_decode_fixup_kernel, 16 calls per step"},
+                         "kernel": "w4a16_decode_kernel, 16 calls per step"},
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                     "mode": "eager C-ABI calls from Python (no graph), X and Y through pinned host memory"},

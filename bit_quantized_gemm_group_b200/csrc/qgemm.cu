@@ -9,6 +9,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <chrono>
 
 #include "../../include/qgemm.h"
 #include "act_quant.cuh"
@@ -80,8 +81,8 @@ int num_sms()
 }
 
 // Launch `kern` with a thread-block cluster of (1, cy, 1).
-template <typename Kern, typename Arg>
-qg_status launch_cluster(Kern kern, dim3 grid, dim3 block, size_t smem, int cy, qg_stream_t stream, const Arg& arg)
+template <typename Kern, typename... Args>
+qg_status launch_cluster(Kern kern, dim3 grid, dim3 block, size_t smem, int cy, qg_stream_t stream, Args... args)
 {
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = grid;
@@ -95,7 +96,7 @@ qg_status launch_cluster(Kern kern, dim3 grid, dim3 block, size_t smem, int cy, 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    QG_CUDA(cudaLaunchKernelEx(&cfg, kern, arg));
+    QG_CUDA(cudaLaunchKernelEx(&cfg, kern, args...));
     return QG_OK;
 }
 
@@ -245,14 +246,45 @@ qg_status make_tmap_3d(CUtensorMap* m, CUtensorMapDataType dt, const void* base,
     return QG_OK;
 }
 
+// N-D tiled map (rank 3..5): dims[0] is contiguous; strides[] are the byte strides of
+// dims 1..rank-1, in any order.
+qg_status make_tmap_nd(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int rank, const uint64_t* dims,
+                       const uint64_t* strides, const uint32_t* box, CUtensorMapSwizzle sw)
+{
+    auto enc = tmap_encoder();
+    if (!enc) {
+        snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled unavailable");
+        return QG_ERR_UNSUPPORTED;
+    }
+    cuuint64_t d[5], st[4];
+    cuuint32_t b[5], e[5];
+    for (int i = 0; i < rank; ++i) {
+        d[i] = dims[i];
+        b[i] = box[i];
+        e[i] = 1;
+        if (i > 0) st[i - 1] = strides[i - 1];
+    }
+    CUresult r = enc(m, dt, rank, const_cast<void*>(base), d, st, b, e, CU_TENSOR_MAP_INTERLEAVE_NONE, sw,
+                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        snprintf(g_last_error, sizeof(g_last_error), "cuTensorMapEncodeTiled (%d-D) failed (%d)", rank, (int)r);
+        return QG_ERR_CUDA;
+    }
+    return QG_OK;
+}
+
 // ---------------------------------------------------------------------------
-// W4A16 decode (stream-K, TMA-fed, workspace)
+// W4A16 decode (stream-K, TMA-fed, in-kernel finish of split slabs, workspace)
 // ---------------------------------------------------------------------------
 struct DecodePlan {
     int MP, G, nslabs, units, grid;
-    size_t partial_bytes;
+    size_t flags_bytes;    // [grid] u64 publication tokens, padded to 256 B
+    size_t partial_bytes;  // flags + [grid] partial tiles of 128 x MP fp32
 };
 
+int decode_cps(int MP);  // CTAs per SM of the configuration for MP tokens (below)
+
+// Launch plan of one decode launch of M <= 32 tokens.
 DecodePlan decode_plan(int M, int K, int N)
 {
     DecodePlan d;
@@ -261,12 +293,40 @@ DecodePlan decode_plan(int M, int K, int N)
     d.G = K / 128;
     d.nslabs = (N + qg::kDecBN - 1) / qg::kDecBN;
     d.units = d.G * d.nslabs;
-    d.grid = std::min(std::min(num_sms(), d.units), qg::kMaxPieces);
-    d.partial_bytes = (size_t)d.grid * 2 * qg::kDecBN * d.MP * sizeof(float);
+    d.grid = std::min(decode_cps(d.MP) * num_sms(), d.units);
+    d.flags_bytes = ((size_t)d.grid * 8 + 255) / 256 * 256;
+    d.partial_bytes = d.flags_bytes + (size_t)d.grid * qg::kDecBN * d.MP * sizeof(float);
     return d;
 }
 
+// Workspace of a call: its launches (32 tokens each, then the remainder) run one after
+// another in the stream and share it, so it covers the largest of their plans.
+size_t decode_workspace_bytes(int M, int K, int N)
+{
+    size_t b = decode_plan(std::min(M, 32), K, N).partial_bytes;
+    if (M > 32 && M % 32) b = std::max(b, decode_plan(M % 32, K, N).partial_bytes);
+    return b;
+}
+
 bool decode_eligible(int M, int N) { return M >= 1 && N % 16 == 0; }
+
+// Publication token of one decode launch: unique per launch within the process and
+// never 0 (0 marks a consumed slot).  The sequence starts at a value drawn from the
+// clock, so a workspace left over from another process (or any other contents)
+// matches a live token only by a 2^-64 coincidence.
+unsigned long long next_decode_token()
+{
+    static std::atomic<unsigned long long> ctr{0x9E3779B97F4A7C15ull ^
+                                               (unsigned long long)std::chrono::steady_clock::now()
+                                                   .time_since_epoch()
+                                                   .count() *
+                                                   0xBF58476D1CE4E5B9ull};
+    unsigned long long t;
+    do {
+        t = ctr.fetch_add(1, std::memory_order_relaxed);
+    } while (t == 0);
+    return t;
+}
 
 template <typename Kern, typename... Args>
 qg_status launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, qg_stream_t stream, Args... args)
@@ -287,46 +347,78 @@ qg_status launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, qg_stream_t 
     return QG_OK;
 }
 
+// Launch configuration per token tile (MT n8 tiles of 8 tokens): consumer warps NW,
+// groups per stage GPS, ring depth ST, dequantization mode FULL, producer warpgroup PWG
+// (register split) or single producer warp, CTAs per SM of one launch CPS (the grid is
+// CPS x the SM count) and the minimum resident CTAs per SM MINB the footprint is sized for
+// (2: a CTA of the next call in the stream can be resident beside this one).
+template <int MT> struct DecodeCfg;
+template <> struct DecodeCfg<1> { static constexpr int NW = 8, GPS = 4, ST = 5, CPS = 1, MINB = 1; static constexpr bool FULL = false, PWG = true; };
+template <> struct DecodeCfg<2> { static constexpr int NW = 8, GPS = 4, ST = 4, CPS = 1, MINB = 1; static constexpr bool FULL = true, PWG = true; };
+template <> struct DecodeCfg<4> { static constexpr int NW = 8, GPS = 2, ST = 4, CPS = 1, MINB = 1; static constexpr bool FULL = true, PWG = true; };
+
+int decode_cps(int MP) { return MP <= 8 ? DecodeCfg<1>::CPS : MP <= 16 ? DecodeCfg<2>::CPS : DecodeCfg<4>::CPS; }
+
 template <int MT, bool BF16>
 qg_status launch_w4a16_decode(const qg::SkinnyParams& sp, const uint32_t* packed, const uint16_t* scales,
                               const uint8_t* zeros, void* ws, qg_stream_t stream)
 {
-    constexpr int WS = MT == 1 ? 2 : 1;                 // two warps per group at M <= 8
-    constexpr int ST = MT == 1 ? 4 : MT == 2 ? 3 : 2;  // ring depth that fits next to the reduction tile
-    using L = qg::DecodeSmem<MT, ST, WS>;
-    static_assert(L::TOTAL <= 227 * 1024, "decode kernel shared memory");
-    auto kern = qg::w4a16_decode_kernel<MT, BF16, ST, WS>;
+    using C = DecodeCfg<MT>;
+    using L = qg::DecodeSmem<MT, C::NW, C::GPS, C::ST, C::PWG>;
+    static_assert(C::MINB * (L::TOTAL + 1024) <= 228 * 1024, "decode kernel shared memory");
+    auto kern = qg::w4a16_decode_kernel<MT, BF16, C::NW, C::GPS, C::ST, C::FULL, C::PWG, C::MINB>;
     const size_t smem = L::TOTAL;
     static KernelInfo info;
     int occ = 1;
     qg_status st = prepare_kernel(info, kern, L::THREADS, smem, &occ);
     if (st != QG_OK) return st;
     const DecodePlan d = decode_plan(sp.M, sp.K, sp.N);
+    if (d.grid > C::CPS * num_sms()) return QG_ERR_UNSUPPORTED;  // plan and configuration disagree
+    const bool narrow = sp.N % 32 != 0;
     qg::DecodeMaps m;
-    const uint64_t N = sp.N, KW = sp.K / 8, G = d.G, K = sp.K;
-    if ((st = make_tmap_2d(&m.w4, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, N, KW, 32, 64,
-                           CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK ||
-        (st = make_tmap_2d(&m.w1, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, N, KW, 32, 16,
-                           CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK ||
-        (st = make_tmap_2d(&m.s4, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, scales, N, G, 128, 4,
+    const uint64_t N = sp.N, K = sp.K, G = d.G;
+    if (narrow) {
+        // [K/8][N] words, boxes {32 columns, 16 rows} (columns past N read as zero)
+        if ((st = make_tmap_2d(&m.w1, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, N, K / 8, 32, 16,
+                               CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
+            return st;
+        m.wg = m.w1;
+    } else {
+        // {32 columns, 16 rows of a group, N/32 column blocks, G groups}
+        const uint64_t dims[4] = {32, 16, N / 32, G};
+        const uint64_t strides[3] = {N * 4, 128, 16 * N * 4};
+        const uint32_t boxg[4] = {32, 16, 4, (uint32_t)C::GPS};
+        const uint32_t box1[4] = {32, 16, 4, 1};
+        if ((st = make_tmap_nd(&m.wg, CU_TENSOR_MAP_DATA_TYPE_UINT32, packed, 4, dims, strides, boxg,
+                               CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK ||
+            (st = make_tmap_nd(&m.w1, CU_TENSOR_MAP_DATA_TYPE_UINT32, packed, 4, dims, strides, box1,
+                               CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
+            return st;
+    }
+    // scales and zeros: {128 columns, GPS | 1 groups} (columns past N read as zero)
+    if ((st = make_tmap_2d(&m.sg, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, scales, N, G, 128, C::GPS,
                            CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK ||
         (st = make_tmap_2d(&m.s1, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, scales, N, G, 128, 1,
                            CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK ||
-        (st = make_tmap_2d(&m.z4, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, zeros, N, G, 128, 4,
+        (st = make_tmap_2d(&m.zg, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, zeros, N, G, 128, C::GPS,
                            CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK ||
         (st = make_tmap_2d(&m.z1, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, zeros, N, G, 128, 1,
                            CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK)
         return st;
     // X as {64 k, M rows, K / 64 halves}: row stride K * 2 bytes, half stride 128 bytes
-    if ((st = make_tmap_3d(&m.x4, CU_TENSOR_MAP_DATA_TYPE_UINT16, sp.X, 64, sp.M, K / 64, K * 2, 128, 64, 8 * MT,
-                           2 * qg::kDecGroupsPerStage, CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK ||
+    if ((st = make_tmap_3d(&m.xg, CU_TENSOR_MAP_DATA_TYPE_UINT16, sp.X, 64, sp.M, K / 64, K * 2, 128, 64, 8 * MT,
+                           2 * C::GPS, CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK ||
         (st = make_tmap_3d(&m.x1, CU_TENSOR_MAP_DATA_TYPE_UINT16, sp.X, 64, sp.M, K / 64, K * 2, 128, 64, 8 * MT, 2,
                            CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
         return st;
     qg::DecodeParams p;
     p.X = sp.X;
+    p.scales = scales;
+    p.zeros = zeros;
     p.Y = sp.Y;
-    p.partials = static_cast<float*>(ws);
+    p.flags = static_cast<unsigned long long*>(ws);
+    p.partials = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + d.flags_bytes);
+    p.token = next_decode_token();
     p.M = sp.M;
     p.K = sp.K;
     p.N = sp.N;
@@ -334,8 +426,8 @@ qg_status launch_w4a16_decode(const qg::SkinnyParams& sp, const uint32_t* packed
     p.nslabs = d.nslabs;
     p.units = d.units;
     p.grid = d.grid;
-    if ((st = launch_pdl(kern, dim3(d.grid), dim3(L::THREADS), smem, stream, p, m)) != QG_OK) return st;
-    return launch_pdl(qg::w4a16_decode_fixup_kernel<BF16>, dim3(d.nslabs), dim3(256), 0, stream, p, 8 * MT);
+    p.narrow = narrow ? 1 : 0;
+    return launch_pdl(kern, dim3(d.grid), dim3(L::THREADS), smem, stream, p, m);
 }
 
 template <bool BF16>
@@ -676,7 +768,7 @@ size_t qg_workspace_size(qg_op op, int M, int K, int N)
     switch (op) {
         case QG_OP_GEMM_W4A16: {
             if (!decode_eligible(M, N)) return 0;
-            return decode_plan(M, K, N).partial_bytes;
+            return decode_workspace_bytes(M, K, N);
         }
         case QG_OP_GEMM_W8A8: {
             if (M >= qg::kTcMinM || N % 16) return 0;
@@ -711,8 +803,24 @@ qg_status qg_quantize_w4_group(const float* W, const float* s_smooth, int K, int
     if (K < 1 || N < 1 || group < 8 || group > 1024 || group % 8 || K % group) return QG_ERR_SHAPE;
     if (misaligned(W) || misaligned(s_smooth) || misaligned(codes) || misaligned(scales) || misaligned(zeros))
         return QG_ERR_ALIGN;
-    const dim3 grid((N + 255) / 256, K / group), block(256);
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (group == 64 || group == 128 || group == 256) {
+        // one pass over W, values held in registers
+        const dim3 g4((N + 127) / 128, K / group), b4(512);
+        uint16_t* sc16 = static_cast<uint16_t*>(scales);
+        if (group == 64)
+            symmetric ? qg::quantize_w4_regs_kernel<64, true><<<g4, b4, 0, s>>>(W, s_smooth, K, N, codes, scales, nullptr)
+                      : qg::quantize_w4_regs_kernel<64, false><<<g4, b4, 0, s>>>(W, s_smooth, K, N, codes, sc16, zeros);
+        else if (group == 128)
+            symmetric ? qg::quantize_w4_regs_kernel<128, true><<<g4, b4, 0, s>>>(W, s_smooth, K, N, codes, scales, nullptr)
+                      : qg::quantize_w4_regs_kernel<128, false><<<g4, b4, 0, s>>>(W, s_smooth, K, N, codes, sc16, zeros);
+        else
+            symmetric ? qg::quantize_w4_regs_kernel<256, true><<<g4, b4, 0, s>>>(W, s_smooth, K, N, codes, scales, nullptr)
+                      : qg::quantize_w4_regs_kernel<256, false><<<g4, b4, 0, s>>>(W, s_smooth, K, N, codes, sc16, zeros);
+        QG_CUDA(cudaGetLastError());
+        return QG_OK;
+    }
+    const dim3 grid((N + 255) / 256, K / group), block(256);
     if (symmetric)
         qg::quantize_w4_sym_kernel<<<grid, block, 0, s>>>(W, s_smooth, K, N, group, reinterpret_cast<int8_t*>(codes),
                                                            static_cast<float*>(scales));
@@ -1105,6 +1213,12 @@ qg_status qg_quantize_w8_channel(const float* W, const float* s, int K, int N, i
     if (!W || !Wq || !sw) return QG_ERR_NULL;
     if (K < 1 || N < 1) return QG_ERR_SHAPE;
     if (misaligned(W) || misaligned(s) || misaligned(Wq) || misaligned(sw)) return QG_ERR_ALIGN;
+    if (N % 8 == 0 && K <= 8 * qg::kW8StripRows) {
+        // one pass over W: 8-column strips, K split over a cluster of up to 8 CTAs
+        const int C = (K + qg::kW8StripRows - 1) / qg::kW8StripRows;
+        return launch_cluster(qg::quantize_w8_strip_kernel, dim3(N / 8, C), dim3(qg::kW8StripThreads), 0, C, stream,
+                              W, s, K, N, Wq, sw);
+    }
     qg::quantize_w8_channel_kernel<<<(N + 127) / 128, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(W, s, K, N,
                                                                                                           Wq, sw);
     QG_CUDA(cudaGetLastError());
@@ -1140,9 +1254,10 @@ qg_status qg_selftest_bounded_wait(uint64_t limit_ns, qg_stream_t stream)
 // ===========================================================================
 namespace {
 
-// 6 MiB per GPU that loads this library, held until the process exits.  The
-// largest decode launch (32 tokens, one CTA per SM, at most 160 CTAs) needs
-// 160 x 2 x 128 x 32 x 4 B of partial tiles = 5 MiB.
+// 6 MiB per GPU that loads this library, held until the process exits.  A decode
+// launch of 32 tokens needs, per CTA (at most one per SM), an 8-byte token and one
+// partial tile of 128 x 32 fp32 (16 KiB): 2.4 MiB on a 148-SM B200, and the array
+// covers GPUs of up to 380 SMs.
 constexpr size_t kNoAllocScratchBytes = size_t(6) << 20;
 static __device__ __align__(256) unsigned char qg_noalloc_scratch[kNoAllocScratchBytes];
 
@@ -1195,7 +1310,8 @@ extern "C" qg_status qg_gemm_w4a16_noalloc(const void* X, qg_dtype xdt, int M, i
     void* ws = nullptr;
     qg_status st = noalloc_scratch(&ws);
     if (st != QG_OK) return st;
-    // The decode kernel writes every partial tile before the fixup kernel reads it, so
-    // nothing in the array has to start at zero; it keeps the last call's contents.
+    // A partial tile is read only after its token (unique to the launch) is seen, and
+    // every launch clears the tokens it consumed, so nothing in the array has to start
+    // at zero; it keeps the last call's contents.
     return qg_gemm_w4a16(X, xdt, M, K, N, packed, scales, zeros, group, Y, ws, kNoAllocScratchBytes, stream);
 }

@@ -122,12 +122,21 @@ qg_status qg_pack_nibbles(const uint8_t* codes, int K, int N, uint32_t* packed, 
  * group    128 (the only group size the GEMM kernels take).
  * Rules: K % 128 == 0, N % 8 == 0.  Accumulation is fp32.
  * workspace: NULL, or a device buffer of at least
- *   qg_workspace_size(QG_OP_GEMM_W4A16, M, K, N) bytes (contents irrelevant).  With
- *   a workspace, decode shapes (N % 16 == 0) use the stream-K kernel, which writes
- *   the partial tiles of split column slabs there and sums them in a second kernel,
- *   in a fixed order.  The workspace must not be shared by calls that may run
- *   concurrently.  Without one, the split-K reduction runs in distributed shared
- *   memory (slower).
+ *   qg_workspace_size(QG_OP_GEMM_W4A16, M, K, N) bytes; its contents on entry do
+ *   not matter.  With a workspace, decode shapes (N % 16 == 0) use the stream-K
+ *   kernel: the pieces of a column slab that is split between CTAs leave fp32
+ *   partial tiles there, each published under a 64-bit token unique to the launch,
+ *   and the CTA holding the slab's first piece adds them in a fixed order and
+ *   writes Y (one launch per 32 tokens, deterministic).  Each launch leaves the
+ *   tokens it consumed cleared.  The workspace must not be shared by calls that may
+ *   run concurrently (calls in one stream are fine).  Without one, the split-K
+ *   reduction runs in distributed shared memory (slower).
+ *   The decode kernel starts streaming its weights, scales and zeros before the
+ *   previous kernel in the stream has finished when that kernel allows it
+ *   (programmatic dependent launch); X, Y and the workspace are touched only after
+ *   it.  So packed, scales and zeros must not be written by a kernel that runs just
+ *   before this call in the same stream and lets its dependents start early (no
+ *   kernel of this library does).
  * ------------------------------------------------------------------------ */
 qg_status qg_gemm_w4a16(const void* X, qg_dtype xdt, int M, int K, int N, const uint32_t* packed,
                         const uint16_t* scales, const uint8_t* zeros, int group, void* Y,

@@ -92,6 +92,52 @@ def test_smooth_scales_and_w8_channel_bitexact():
     np.testing.assert_array_equal(sw.cpu().numpy(), sw_o)
 
 
+@pytest.mark.parametrize("K,N,smooth", [(11008, 4096, True), (16384, 64, False), (2048, 24, True), (100, 136, True),
+                                         (4096, 100, True), (20000, 8, False)])
+def test_quantize_w8_channel_shapes_bitexact(K, N, smooth):
+    """Both paths of the INT8 channel quantizer: the one-pass strip kernel (N % 8 == 0,
+    K <= 16384: clusters of 1..8 CTAs along K, ragged last CTA) and the general kernel
+    (N % 8 != 0 or longer K); a zero column and smoothing on and off."""
+    W = synth.weights(K, N, 0.02, 0.01, 8.0, seed=K + N)
+    W[:, 3] = 0.0
+    s_o = None
+    if smooth:
+        s_o = np.random.default_rng(K).uniform(0.5, 2.0, K).astype(np.float32)
+    q = qlib()
+    Wq = torch.empty(K, N, dtype=torch.int8, device="cuda")
+    sw = torch.empty(N, dtype=torch.float32, device="cuda")
+    q.qg_quantize_w8_channel(cuda(W), None if s_o is None else cuda(s_o), Wq, sw)
+    _status_ok()
+    Wq_o, sw_o, _ = oracle.quantize_w8_channel(W, s_o)
+    np.testing.assert_array_equal(Wq.cpu().numpy(), Wq_o)
+    np.testing.assert_array_equal(sw.cpu().numpy(), sw_o)
+
+
+@pytest.mark.parametrize("group", [64, 256, 32])
+@pytest.mark.parametrize("sym", [False, True])
+def test_quantize_w4_other_group_sizes_bitexact(group, sym):
+    """Group sizes other than 128 (64 and 256 take the register kernel, 32 the per-column
+    kernel), with a ragged column count and smoothing."""
+    K, N = 1024, 200
+    W = synth.weights(K, N, 0.02, 0.01, 8.0, seed=group)
+    W[0:group, 5] = 0.0                   # zero group
+    W[group:2 * group, 7] = 0.01          # constant group
+    s_o = np.random.default_rng(group).uniform(0.5, 2.0, K).astype(np.float32)
+    if sym:
+        codes, scales, packed = quant_w4_sym(W, s_o, group=group)
+        c_o, sc_o, _ = oracle.quantize_w4_sym(W, group=group, s_smooth=s_o)
+        _status_ok()
+        np.testing.assert_array_equal(codes.cpu().numpy().view(np.int8), c_o)
+        np.testing.assert_array_equal(scales.cpu().numpy(), sc_o)
+    else:
+        codes, scales, zeros, packed = quant_w4_asym(W, s_o, group=group)
+        c_o, sc_o, z_o, _ = oracle.quantize_w4_asym(W, group=group, s_smooth=s_o)
+        _status_ok()
+        np.testing.assert_array_equal(codes.cpu().numpy(), c_o)
+        np.testing.assert_array_equal(u16(scales), sc_o)
+        np.testing.assert_array_equal(zeros.cpu().numpy(), z_o)
+
+
 def test_quantize_w4_sym_smoothed_bitexact():
     cfg = synth.CONFIGS["w4a8"]
     K, N = cfg["KN"][0]
