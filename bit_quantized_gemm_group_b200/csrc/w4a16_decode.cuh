@@ -88,7 +88,9 @@ struct DecodeSmem {
     static constexpr int Z_OFF = S_OFF + GPS * 256;   // u8 zeros [GPS][128]
     static constexpr int STAGE = (Z_OFF + GPS * 128 + 1023) / 1024 * 1024;
     static constexpr int FRAG = 4 * MT;               // float4 accumulator fragments per lane (64 columns x MP tokens per warp)
-    static constexpr int RED = (KW - 1) * 2 * FRAG * 32 * 16;
+    static constexpr int TS = kDecBN + 4;            // row stride (floats) of the [token][column] result tile
+    static constexpr int RED_K = (KW - 1) * 2 * FRAG * 32 * 16;  // k-warp reduction (fragment layout)
+    static constexpr int RED = RED_K > MP * TS * 4 ? RED_K : MP * TS * 4;  // the result tile aliases it
     static constexpr int TOTAL = ST * STAGE + RED + 2 * ST * 8 + 1024;
     // The producer is one warp after the consumers, or (PWG) a whole warpgroup of which
     // the first warp works, so that the register file can be split with setmaxnreg: the
@@ -466,36 +468,60 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG>::THREADS, MIN
         const int all_ok = named_bar_and(1, 32 * NW, ok);
         if (!all_ok) ok = false;
 
+        // 2. warps (0, 0) and (1, 0) hold the piece's 128 x MP result: into the tile
+        //    [token][column] (row stride TS floats), which aliases the reduction area
+        float* tile = reinterpret_cast<float*>(red);
         if (wk == 0 && ok) {
-            // 2. the piece's 128 x MP result is in warps (0, 0) and (1, 0)
+#pragma unroll
+            for (int h = 0; h < 2; ++h)
+#pragma unroll
+                for (int cp = 0; cp < 2; ++cp)
+#pragma unroll
+                    for (int j = 0; j < MT; ++j) {
+                        const int col = 64 * wn + 32 * h + 4 * g8 + 2 * cp, tok = 8 * j + 2 * t4;
+                        *reinterpret_cast<float2*>(tile + tok * L::TS + col) = make_float2(acc[h][cp][j][0], acc[h][cp][j][2]);
+                        *reinterpret_cast<float2*>(tile + (tok + 1) * L::TS + col) =
+                            make_float2(acc[h][cp][j][1], acc[h][cp][j][3]);
+                    }
+        }
+        named_bar_sync(1, 32 * NW);
+
+        // 3. every consumer thread takes float4 elements (token, 4 columns) of the tile
+        if (ok) {
+            constexpr int NE = MP * 32;             // float4 elements of the tile
+            constexpr int EPT = (NE + 32 * NW - 1) / (32 * NW);
+            const int ct = threadIdx.x;             // 0 .. 32 NW - 1
             const bool whole = sc.ga == 0 && sc.gb == G;
             const bool head = sc.ga == 0 && !whole;  // finishes a split slab (the CTA's last piece)
-            float4* mine = reinterpret_cast<float4*>(p.partials) + (size_t)blockIdx.x * (L::PARTIAL_FLOATS / 4) +
-                           wn * L::FRAG * 32;
+            const int n0 = sc.slab * kDecBN;
             if (!whole && !head) {
-                // publish this piece's partial tile (fragment layout), then its token
+                // publish this piece's tile ([token][128 columns] fp32), then its token: the
+                // barrier orders every thread's stores before the one fence and release
+                float4* mine = reinterpret_cast<float4*>(p.partials) + (size_t)blockIdx.x * (L::PARTIAL_FLOATS / 4);
 #pragma unroll
-                for (int h = 0; h < 2; ++h)
-#pragma unroll
-                    for (int cp = 0; cp < 2; ++cp)
-#pragma unroll
-                        for (int j = 0; j < MT; ++j)
-                            __stcg(mine + ((h * 2 + cp) * MT + j) * 32 + lane,
-                                   make_float4(acc[h][cp][j][0], acc[h][cp][j][1], acc[h][cp][j][2], acc[h][cp][j][3]));
-                // one release by one thread after the two warps' stores (the barrier orders
-                // them before its fence): the other 63 threads do not stall on a fence
-                named_bar_sync(2, 64);
-                if (warp == 0 && lane == 0) {
+                for (int i = 0; i < EPT; ++i) {
+                    const int e = ct + i * 32 * NW;
+                    if (e < NE) __stcg(mine + e, *reinterpret_cast<const float4*>(tile + (e >> 5) * L::TS + 4 * (e & 31)));
+                }
+                named_bar_sync(1, 32 * NW);
+                if (ct == 0) {
                     __threadfence();
                     st_release_u64(p.flags + blockIdx.x, p.token);
                 }
             } else {
+                float4 v[EPT];
+#pragma unroll
+                for (int i = 0; i < EPT; ++i) {
+                    const int e = ct + i * 32 * NW;
+                    v[i] = e < NE ? *reinterpret_cast<const float4*>(tile + (e >> 5) * L::TS + 4 * (e & 31))
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
+                }
                 bool fin_ok = true;
                 if (head) {
                     // add the other pieces of this slab, held by the next CTAs, in CTA order.
                     // Lane i of warp 0 watches the token of CTA blockIdx.x + 1 + i (all polls
-                    // in flight at once); then the partial tiles are loaded with every load
-                    // in flight and summed in CTA order.
+                    // in flight at once); then every thread loads its elements of every
+                    // partial tile at once and adds them in CTA order.
                     const int cl = dec_cta_of_unit(sc.slab * G + G - 1, p.units, p.grid);
                     const int np = cl - (int)blockIdx.x;  // partial tiles to add
                     int ready = 1;
@@ -504,10 +530,10 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG>::THREADS, MIN
                         const unsigned long long lim = g_wait_limit_ns;
                         for (int i0 = 0; i0 < np; i0 += 32) {
                             const int c = (int)blockIdx.x + 1 + i0 + lane;
-                            bool mine = i0 + lane >= np;  // lanes past the last piece have nothing to watch
+                            bool seen = i0 + lane >= np;  // lanes past the last piece have nothing to watch
                             for (uint32_t it = 0;; ++it) {
-                                if (!mine) mine = ld_acquire_u64(p.flags + c) == p.token;
-                                if (__all_sync(0xffffffffu, mine)) break;
+                                if (!seen) seen = ld_acquire_u64(p.flags + c) == p.token;
+                                if (__all_sync(0xffffffffu, seen)) break;
                                 __nanosleep(32);
                                 if ((it & 15u) == 15u && globaltimer_ns() - t0 > lim) {
                                     if (lane == 0) set_status(7u);
@@ -518,65 +544,52 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG>::THREADS, MIN
                             if (!ready) break;
                         }
                     }
-                    ready = named_bar_and(2, 64, ready);
-                    if (!ready) fin_ok = false;
-                    const float4* base = reinterpret_cast<const float4*>(p.partials) + wn * L::FRAG * 32 + lane;
-                    constexpr int NB = L::FRAG >= 8 ? 1 : 2;  // tiles loaded together (at most 32 registers of loads in flight)
+                    fin_ok = named_bar_and(1, 32 * NW, ready) != 0;
+                    const float4* base = reinterpret_cast<const float4*>(p.partials);
+                    constexpr int NB = EPT >= 8 ? 1 : 8 / EPT;  // partial tiles whose loads are in flight together (32 registers)
 #pragma unroll 1
                     for (int c0 = (int)blockIdx.x + 1; fin_ok && c0 <= cl; c0 += NB) {
-                        float4 v[NB][L::FRAG];
+                        float4 w[NB][EPT];
 #pragma unroll
                         for (int r = 0; r < NB; ++r)
-                            if (c0 + r <= cl)
 #pragma unroll
-                                for (int i = 0; i < L::FRAG; ++i)
-                                    v[r][i] = __ldcg(base + (size_t)(c0 + r) * (L::PARTIAL_FLOATS / 4) + i * 32);
+                            for (int i = 0; i < EPT; ++i) {
+                                const int e = ct + i * 32 * NW;
+                                if (c0 + r <= cl && e < NE) w[r][i] = __ldcg(base + (size_t)(c0 + r) * (L::PARTIAL_FLOATS / 4) + e);
+                            }
 #pragma unroll
                         for (int r = 0; r < NB; ++r)
-                            if (c0 + r <= cl)
 #pragma unroll
-                                for (int h = 0; h < 2; ++h)
-#pragma unroll
-                                    for (int cp = 0; cp < 2; ++cp)
-#pragma unroll
-                                        for (int j = 0; j < MT; ++j) {
-                                            const float4 w = v[r][(h * 2 + cp) * MT + j];
-                                            acc[h][cp][j][0] += w.x;
-                                            acc[h][cp][j][1] += w.y;
-                                            acc[h][cp][j][2] += w.z;
-                                            acc[h][cp][j][3] += w.w;
-                                        }
+                            for (int i = 0; i < EPT; ++i)
+                                if (c0 + r <= cl) {
+                                    v[i].x += w[r][i].x;
+                                    v[i].y += w[r][i].y;
+                                    v[i].z += w[r][i].z;
+                                    v[i].w += w[r][i].w;
+                                }
                     }
-                    named_bar_sync(2, 64);
+                    named_bar_sync(1, 32 * NW);
                     if (fin_ok && warp == 0)
                         for (int c = (int)blockIdx.x + 1 + lane; c <= cl; c += 32) p.flags[c] = 0ull;  // consumed: clear
                 }
                 if (fin_ok) {
-                    // write Y: lane holds columns 4g+2cp, 4g+2cp+1 for tokens 2t, 2t+1 of each tile
-                    const int n0 = sc.slab * kDecBN + 64 * wn;
+                    // Y: four adjacent columns of one token per element (N % 16 == 0)
 #pragma unroll
-                    for (int h = 0; h < 2; ++h)
-#pragma unroll
-                        for (int cp = 0; cp < 2; ++cp) {
-                            const int col = n0 + 32 * h + 4 * g8 + 2 * cp;
-                            if (col < p.N) {
-#pragma unroll
-                                for (int j = 0; j < MT; ++j)
-#pragma unroll
-                                    for (int e = 0; e < 2; ++e) {
-                                        const int tok = 8 * j + 2 * t4 + e;
-                                        if (tok < p.M) {
-                                            const uint32_t v = (uint32_t)H::to_bits(acc[h][cp][j][e]) |
-                                                               ((uint32_t)H::to_bits(acc[h][cp][j][e + 2]) << 16);
-                                            *reinterpret_cast<uint32_t*>(p.Y + (int64_t)tok * p.N + col) = v;
-                                        }
-                                    }
-                            }
+                    for (int i = 0; i < EPT; ++i) {
+                        const int e = ct + i * 32 * NW;
+                        const int tok = e >> 5, col = n0 + 4 * (e & 31);
+                        if (e < NE && tok < p.M && col < p.N) {
+                            const uint2 o = make_uint2((uint32_t)H::to_bits(v[i].x) | ((uint32_t)H::to_bits(v[i].y) << 16),
+                                                       (uint32_t)H::to_bits(v[i].z) | ((uint32_t)H::to_bits(v[i].w) << 16));
+                            *reinterpret_cast<uint2*>(p.Y + (int64_t)tok * p.N + col) = o;
                         }
+                    }
                 }
             }
         }
-        // 3. every consumer starts the next piece from zero
+        named_bar_sync(1, 32 * NW);  // the tile is free for the next piece
+
+        // 4. every consumer starts the next piece from zero
 #pragma unroll
         for (int h = 0; h < 2; ++h)
 #pragma unroll
