@@ -30,7 +30,7 @@ EXPORTS = ["qg_quantize_w4_group", "qg_pack_nibbles", "qg_gemm_w4a16", "qg_smoot
            "qg_last_error", "qg_selftest_bounded_wait", "qg_workspace_size", "qg_gemm_w4a16_noalloc",
            "qg_awq_act_mean", "qg_awq_scales", "qg_awq_scale_act", "qg_awq_search", "qg_outlier_split_w4",
            "qg_outlier_side_add", "qg_gemm_w4a16_outlier", "qg_prune24", "qg_pack24_vals", "qg_gemm_w4a16_24",
-           "qg_gptq"]
+           "qg_gptq", "qg_gptq_blocked"]
 
 
 class QgError(RuntimeError):
@@ -57,6 +57,7 @@ _SIGS = {
     "qg_outlier_side_add": [_P, _I, _I, _I, _I, _I, _I, _P, _P, _P, _P, _P],
     "qg_gemm_w4a16_outlier": [_P, _I, _I, _I, _I, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _SZ, _P],
     "qg_gptq": [_P, _I, _I, _P, _I, _I, ctypes.c_double, _P, _P, _P, _P, _SZ, _P],
+    "qg_gptq_blocked": [_P, _I, _I, _P, _I, _I, ctypes.c_double, _P, _P, _P, _P, _SZ, _P],
     "qg_prune24": [_P, _I, _I, _P, _P, _P],
     "qg_pack24_vals": [_P, _P, _I, _I, _P, _P],
     "qg_gemm_w4a16_24": [_P, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P, _P],
@@ -246,6 +247,14 @@ def qg_gptq(Xcal, W, codes, scales, zeros, group=128, damp=0.01, workspace="auto
     wp, wb = _ws(workspace, QG_OP_GPTQ, Mc, K, N, Xcal.device)
     _check(lib().qg_gptq(_ptr(Xcal), Mc, K, _ptr(W), N, group, float(damp), _ptr(codes), _ptr(scales), _ptr(zeros), wp,
                         wb, _stream(stream)), "qg_gptq")
+
+
+def qg_gptq_blocked(Xcal, W, codes, scales, zeros, group=128, damp=0.01, workspace="auto", stream=None):
+    Mc, K = Xcal.shape
+    N = W.shape[1]
+    wp, wb = _ws(workspace, QG_OP_GPTQ, Mc, K, N, Xcal.device)
+    _check(lib().qg_gptq_blocked(_ptr(Xcal), Mc, K, _ptr(W), N, group, float(damp), _ptr(codes), _ptr(scales),
+                                _ptr(zeros), wp, wb, _stream(stream)), "qg_gptq_blocked")
 
 
 def qg_prune24(W, Wp, meta, stream=None):

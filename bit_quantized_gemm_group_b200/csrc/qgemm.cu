@@ -15,6 +15,7 @@
 #include "act_quant.cuh"
 #include "awq.cuh"
 #include "gptq.cuh"
+#include "gptq_blocked.cuh"
 #include "common.cuh"
 #include "int8_skinny.cuh"
 #include "outlier.cuh"
@@ -696,6 +697,44 @@ GptqWs gptq_carve(void* base, int K, int N)
     return w;
 }
 
+// Workspace of the blocked form: the reversed Hessian and its Cholesky factor (in
+// place), the factor's inverse, the compensated weights, one block of row errors, the
+// reversed calibration tokens and the inverses of the 64 x 64 diagonal blocks.
+struct GptqBlockedWs {
+    double *a, *inv, *wc, *err, *xr, *dinv;
+    size_t bytes;
+};
+
+GptqBlockedWs gptq_blocked_carve(void* base, int Mc, int K, int N)
+{
+    GptqBlockedWs w{};
+    size_t off = 0;
+    auto take = [&](size_t b) {
+        const size_t o = off;
+        off += (b + 255) & ~size_t(255);
+        return base ? reinterpret_cast<double*>(static_cast<uint8_t*>(base) + o) : nullptr;
+    };
+    const size_t nblk = (size_t)(K + qg::kCholNb - 1) / qg::kCholNb;
+    w.a = take(8 * (size_t)K * K);
+    w.inv = take(8 * (size_t)K * K);
+    w.wc = take(8 * (size_t)K * N);
+    w.err = take(8 * (size_t)std::min(K, 1024) * N);
+    w.xr = take(8 * (size_t)Mc * K);
+    w.dinv = take(8 * nblk * qg::kCholNb * qg::kCholNb);
+    w.bytes = off;
+    return w;
+}
+
+template <int BM, int BN>
+qg_status dgemm(const qg::DgemmArgs& a, cudaStream_t st)
+{
+    if (a.M <= 0 || a.N <= 0) return QG_OK;
+    const dim3 grid((a.N + BN - 1) / BN, (a.M + BM - 1) / BM);
+    qg::dgemm_strided_kernel<BM, BN><<<grid, 256, 0, st>>>(a);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+
 // ---------------------------------------------------------------------------
 // int8 skinny paths
 // ---------------------------------------------------------------------------
@@ -762,7 +801,7 @@ size_t qg_workspace_size(qg_op op, int M, int K, int N)
 {
     if (op == QG_OP_GPTQ) {  // any K that a group size divides (K % 8 == 0), any N
         if (M < 1 || K < 8 || K % 8 || K > 16384 || N < 1) return 0;
-        return gptq_carve(nullptr, K, N).bytes;
+        return std::max(gptq_carve(nullptr, K, N).bytes, gptq_blocked_carve(nullptr, M, K, N).bytes);
     }
     if (M < 1 || K < 128 || N < 8 || K % 128) return 0;
     switch (op) {
@@ -1124,6 +1163,82 @@ qg_status qg_gptq(const uint16_t* Xcal, int Mc, int K, const float* W, int N, in
         }
     }
     QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+
+qg_status qg_gptq_blocked(const uint16_t* Xcal, int Mc, int K, const float* W, int N, int group, double damp,
+                          uint8_t* codes, uint16_t* scales, uint8_t* zeros, void* workspace, size_t ws_bytes,
+                          qg_stream_t stream)
+{
+    if (!Xcal || !W || !codes || !scales || !zeros || !workspace) return QG_ERR_NULL;
+    if (Mc < 1 || K < 8 || K > 16384 || N < 1 || group < 8 || group > 1024 || group % 8 || K % group ||
+        !(damp > 0.0 && damp < 1e30))
+        return QG_ERR_SHAPE;
+    if (misaligned(Xcal) || misaligned(W) || misaligned(codes) || misaligned(scales) || misaligned(zeros) ||
+        misaligned(workspace))
+        return QG_ERR_ALIGN;
+    if (ws_bytes < gptq_blocked_carve(nullptr, Mc, K, N).bytes) return QG_ERR_WORKSPACE;
+    const GptqBlockedWs w = gptq_blocked_carve(workspace, Mc, K, N);
+    cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+    constexpr int NB = qg::kCholNb;
+    const int grid_ew = std::max(1, 8 * num_sms());
+    // Hr = (2/Mc) Xr^T Xr (lower triangle), then the ridge on its diagonal
+    const int64_t xt = (int64_t)Mc * K;
+    qg::gptq_xrev_kernel<<<(int)std::min<int64_t>((xt + 255) / 256, grid_ew), 256, 0, st>>>(Xcal, Mc, K, w.xr);
+    QG_CUDA(cudaGetLastError());
+    qg_status r = dgemm<64, 64>({K, K, Mc, 2.0 / Mc, 0.0, w.xr, 1, K, w.xr, K, 1, w.a, K, 1, 0}, st);
+    if (r != QG_OK) return r;
+    qg::gptq_ridge_kernel<<<1, 32, 0, st>>>(w.a, K, damp);
+    QG_CUDA(cudaGetLastError());
+    // Lr: right-looking blocked Cholesky, 64-wide panels
+    for (int p = 0; p < K; p += NB) {
+        const int nb = std::min(NB, K - p), rows = K - p - nb;
+        qg::chol_diag_kernel<<<1, 256, 0, st>>>(w.a, K, p, nb, w.dinv);
+        QG_CUDA(cudaGetLastError());
+        if (rows > 0) {
+            qg::chol_panel_kernel<<<(rows + 127) / 128, 128, 0, st>>>(w.a, K, p, nb, w.dinv);
+            QG_CUDA(cudaGetLastError());
+            double* pan = w.a + (int64_t)(p + nb) * K + p;
+            r = dgemm<64, 64>({rows, rows, nb, -1.0, 1.0, pan, K, 1, pan, 1, K, pan + nb, K, 1, 0}, st);
+            if (r != QG_OK) return r;
+        }
+    }
+    // Lr^-1 by block rows (its upper triangle stays zero)
+    QG_CUDA(cudaMemsetAsync(w.inv, 0, 8 * (size_t)K * K, st));
+    for (int r0 = 0; r0 < K; r0 += NB) {
+        const int nb = std::min(NB, K - r0);
+        if (r0 > 0) {
+            r = dgemm<32, 32>({nb, r0, r0, 1.0, 0.0, w.a + (int64_t)r0 * K, K, 1, w.inv, K, 1, w.inv + (int64_t)r0 * K, K,
+                               0, 1},
+                              st);
+            if (r != QG_OK) return r;
+        }
+        qg::trinv_rows_kernel<<<(r0 + nb + 127) / 128, 128, 0, st>>>(w.inv, K, r0, nb, w.dinv);
+        QG_CUDA(cudaGetLastError());
+    }
+    // the rows, one group-sized block at a time; U[i][j] = Lr^-1[K-1-i][K-1-j]
+    const int64_t total = (int64_t)K * N;
+    qg::gptq_load_kernel<<<(int)std::min<int64_t>((total + 255) / 256, grid_ew), 256, 0, st>>>(W, total, w.wc);
+    QG_CUDA(cudaGetLastError());
+    const int NC = group <= 256 ? 32 : 8;
+    const size_t smem = (size_t)group * NC * 8;
+    static KernelInfo block_info;
+    int occ = 0;
+    r = prepare_kernel(block_info, qg::gptq_block_kernel, NC * 8, 64 * 1024, &occ);
+    if (r != QG_OK) return r;
+    for (int b = 0; b < K; b += group) {
+        qg::gptq_block_kernel<<<(N + NC - 1) / NC, NC * 8, smem, st>>>(w.wc, K, N, b, group, w.inv, codes, scales,
+                                                                        zeros, w.err, NC);
+        QG_CUDA(cudaGetLastError());
+        const int rest = K - b - group;
+        if (rest > 0) {
+            const double* ub = w.inv + (int64_t)(K - 1 - b) * K + (K - 1 - b - group);
+            r = dgemm<64, 64>({rest, N, group, -1.0, 1.0, ub, -1, -(int64_t)K, w.err, N, 1,
+                               w.wc + (int64_t)(b + group) * N, N, 0, 0},
+                              st);
+            if (r != QG_OK) return r;
+        }
+    }
     return QG_OK;
 }
 

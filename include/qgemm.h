@@ -321,7 +321,8 @@ qg_status qg_gemm_w4a16_24(const void* X, qg_dtype xdt, int M, int K, int N, con
  * Rules: Mc >= 1, 8 <= group <= 1024, group % 8 == 0, K % group == 0, K <= 16384,
  *   0 < damp (0.01 is the usual ridge).
  * workspace (required): at least qg_workspace_size(QG_OP_GPTQ, Mc, K, N) bytes
- *   (2 K^2 + K N doubles and a few vectors), contents irrelevant.
+ *   (2 K^2 + K N doubles and a few vectors; more when the blocked form needs it),
+ *   contents irrelevant.
  * Device errors: QG_ERR_NONFINITE (a non-finite weight), QG_ERR_RANGE (a scale above
  *   fp16, or a zero pivot).  An offline step: about 7 K kernel launches and
  *   O(K^3 + K^2 N) binary64 operations.
@@ -329,6 +330,28 @@ qg_status qg_gemm_w4a16_24(const void* X, qg_dtype xdt, int M, int K, int N, con
 qg_status qg_gptq(const uint16_t* Xcal, int Mc, int K, const float* W, int N, int group,
                   double damp, uint8_t* codes, uint16_t* scales, uint8_t* zeros, void* workspace,
                   size_t ws_bytes, qg_stream_t stream);
+
+/* GPTQ in its blocked Cholesky form (the fast offline path).   [A] sec. 3.1-3.3
+ *
+ *   Same H, lambda, group rules and outputs as qg_gptq.  After rows 0..k-1 are
+ *   eliminated, row k of the remaining H^-1 over the square root of its diagonal is
+ *   row k of the upper Cholesky factor U of H^-1 (H^-1 = U^T U), so with
+ *   err_k = (w_k - (q_k - z) s) / U[k][k] and w_j -= err_k U[k][j] (j > k) each row is
+ *   compensated as in qg_gptq.  U comes from one Cholesky factorization and one
+ *   triangular inverse (U = J Lr^-1 J, Hr = J H J = Lr Lr^T, J the index reversal);
+ *   the rows of a group are compensated inside the group as they are rounded and the
+ *   later rows receive the group's errors in one GEMM per group.  All in binary64,
+ *   summed in another order than qg_gptq: a code may differ from qg_gptq's where the
+ *   compensated weight lies within rounding noise of a rounding boundary.
+ * Arguments and rules as qg_gptq; workspace: qg_workspace_size(QG_OP_GPTQ, Mc, K, N)
+ *   covers both forms.  Device errors: QG_ERR_NONFINITE (a non-finite weight),
+ *   QG_ERR_RANGE (a scale above fp16, or a pivot that is not positive: H not positive
+ *   definite in binary64).  About 6 K / 64 + 2 K / group kernel launches and
+ *   O(K^3 / 3 + K^2 (Mc + N) / 2) binary64 multiply-adds.
+ * ------------------------------------------------------------------------ */
+qg_status qg_gptq_blocked(const uint16_t* Xcal, int Mc, int K, const float* W, int N, int group,
+                          double damp, uint8_t* codes, uint16_t* scales, uint8_t* zeros,
+                          void* workspace, size_t ws_bytes, qg_stream_t stream);
 
 /* --------------------------------------------------------------------------
  * AWQ: activation-aware per-input-channel scales for the INT4 weights.   [A]

@@ -93,3 +93,71 @@ def test_feeds_the_w4a16_gemm_with_a_lower_layer_error():
     y_gptq, _ = oracle.gemm_w4a16_ref(X, oracle.pack_nibbles(c_o), s_o, z_o)
     exact = oracle.gemm_f64(X, W)
     assert np.sum((exact - y_gptq) ** 2) < 0.8 * np.sum((exact - y_rtn) ** 2)
+
+
+# ---------------------------------------------------------------------------
+# the blocked Cholesky form (qg_gptq_blocked)
+# ---------------------------------------------------------------------------
+def _gptq_blocked(Xb, W, group):
+    q = qlib()
+    K, N = W.shape
+    codes = torch.full((K, N), 255, dtype=torch.uint8, device="cuda")
+    scales = torch.zeros((K // group, N), dtype=torch.int16, device="cuda")
+    zeros = torch.full((K // group, N), 255, dtype=torch.uint8, device="cuda")
+    q.qg_gptq_blocked(x_device(Xb, torch.bfloat16), cuda(W), codes, scales, zeros, group=group)
+    _status_ok()
+    return codes.cpu().numpy(), u16(scales), zeros.cpu().numpy()
+
+
+# a partial last 64-wide panel (K = 296), groups of 8 .. 512 (the 512 case takes the
+# narrow column tiling), more columns than one tile
+@pytest.mark.parametrize("Mc,K,N,group", [(300, 256, 40, 128), (64, 128, 24, 64), (200, 256, 136, 32),
+                                          (17, 384, 8, 128), (100, 296, 40, 8), (160, 1024, 24, 512),
+                                          (256, 1024, 200, 128)])
+def test_blocked_replay(Mc, K, N, group):
+    """The blocked form compensates each row as the sequential definition does, with the
+    sums in another order: every code must be the rounding of its teacher-forced replayed
+    value up to rounding noise (slack <= 1e-6 grid steps), every scale and zero the
+    group's own; and on these well-conditioned cases the codes equal the oracle's except
+    where a value sits on a rounding boundary (at most 1 in 1000)."""
+    X, Xb = _calib(Mc, K, seed=K + N)
+    W = synth.weights(K, N, 0.02, 0.01, 8.0, seed=N)
+    codes, scales, zeros = _gptq_blocked(Xb, W, group)
+    slack, sm, zm, st = oracle.gptq_replay(X, W, codes, scales, zeros, group, scale_ulps=0)
+    assert st == 0
+    assert slack <= 1e-6 and sm == 0 and zm == 0, (slack, sm, zm)
+    c_o, s_o, z_o, _ = oracle.gptq(X, W, group)
+    assert (codes != c_o).mean() <= 1e-3
+
+
+def test_blocked_full_size_against_the_sequential_device_path():
+    """4096 x 4096 with 512 calibration tokens (the benchmark's GPTQ case).  The sequential
+    device path is the oracle's definition bit for bit (test_bitexact); the blocked form
+    must give the same codes up to rounding-boundary cases (<= 1e-4 of them), scales
+    within one fp16 step and zeros within 1 on every group, and a calibration-batch layer
+    error no larger than round-to-nearest's."""
+    q = qlib()
+    K, N = 4096, 4096
+    Mc = synth.CONFIGS["awq"]["calib_tokens"]
+    W = synth.workload_weights("w4a16_decode", K, N)
+    X, xcb = synth.calibration(K, synth.CONFIGS["awq"])
+    Xd, Wd = x_device(xcb, torch.bfloat16), cuda(W)
+    outs = []
+    for fn in (q.qg_gptq, q.qg_gptq_blocked):
+        codes = torch.full((K, N), 255, dtype=torch.uint8, device="cuda")
+        scales = torch.zeros((K // 128, N), dtype=torch.int16, device="cuda")
+        zeros = torch.full((K // 128, N), 255, dtype=torch.uint8, device="cuda")
+        fn(Xd, Wd, codes, scales, zeros)
+        _status_ok()
+        outs.append((codes.cpu().numpy(), u16(scales), zeros.cpu().numpy()))
+    (c_s, s_s, z_s), (c_b, s_b, z_b) = outs
+    assert (c_s != c_b).mean() <= 1e-4
+    assert np.abs(s_s.astype(np.int32) - s_b.astype(np.int32)).max() <= 1
+    assert np.abs(z_s.astype(np.int32) - z_b.astype(np.int32)).max() <= 1
+    # layer error on the calibration batch (a sample of 64 tokens)
+    Xs = X[:64]
+    exact = oracle.gemm_f64(Xs, W)
+    c0, s0, z0, _ = oracle.quantize_w4_asym(W)
+    y_rtn, _ = oracle.gemm_w4a16_ref(Xs, oracle.pack_nibbles(c0), s0, z0)
+    y_b, _ = oracle.gemm_w4a16_ref(Xs, oracle.pack_nibbles(c_b), s_b, z_b)
+    assert np.sum((exact - y_b) ** 2) <= np.sum((exact - y_rtn) ** 2)
