@@ -715,8 +715,9 @@ def bench_outlier(q, pk, L2):
 
 def bench_sparse24(q, pk, L2):
     """The decode layer 4096 x 12288 pruned 2:4 and quantized to INT4 (0.375 bytes per
-    weight with positions): the SIMT sparse GEMM at M = 1 and 16, beside the dense W4A16
-    call on the same pruned matrix, weights rotated over copies > 2 x L2."""
+    weight with positions): the tensor-core (mma.sp) decode kernel and the SIMT kernel at
+    M = 1 and 16, beside the dense W4A16 call on the same pruned matrix, weights rotated
+    over copies > 2 x L2."""
     K, N = synth.CONFIGS["w4a16_decode"]["KN"][0]
     W = torch.from_numpy(synth.workload_weights("w4a16_decode", K, N)).cuda()
     Wp = torch.empty_like(W)
@@ -729,21 +730,27 @@ def bench_sparse24(q, pk, L2):
     q.qg_quantize_w4_group(Wp, None, 128, False, codes, sc, z)
     vals = torch.empty(K // 16, N, dtype=torch.int32, device="cuda")
     q.qg_pack24_vals(codes, meta, vals)
+    vtc = torch.empty_like(vals)
+    q.qg_pack24_tc(vals, vtc)
     pw = torch.empty(K // 8, N, dtype=torch.int32, device="cuda")
     q.qg_pack_nibbles(codes, pw)
     del Wp, codes
     wb = K * N * 3 // 8 + 3 * (K // 128) * N
     rot = max(1, math.ceil(2 * L2 / wb))
-    sets = [(vals, meta, sc, z, pw)] + [tuple(t.clone() for t in (vals, meta, sc, z, pw)) for _ in range(rot - 1)]
+    sets = [(vals, meta, sc, z, pw, vtc)] + [tuple(t.clone() for t in (vals, meta, sc, z, pw, vtc))
+                                             for _ in range(rot - 1)]
     res = {}
     for M in (1, 16):
         X = x_bf16("w4a16_decode", M, K)
         Y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        ms_t = time_calls(lambda i: q.qg_gemm_w4a16_24_tc(X, sets[i][5], sets[i][1], sets[i][2], sets[i][3], Y), 16, rot)
         ms_s = time_calls(lambda i: q.qg_gemm_w4a16_24(X, *sets[i][:4], Y), 16, rot)
         ms_d = time_calls(lambda i: q.qg_gemm_w4a16(X, sets[i][4], sets[i][2], sets[i][3], Y), 16, rot)
         by = wb + 2 * M * K + 2 * M * N
-        res[f"M={M}"] = {"us": ms_s * 1e3, "us_dense_w4a16": ms_d * 1e3, "gbs": by / (ms_s * 1e-3) / 1e9,
-                         "bytes": by, "roofline_frac": by / (pk["hbm_gbs"] * 1e9) / (ms_s * 1e-3)}
+        res[f"M={M}"] = {"us": ms_t * 1e3, "us_simt": ms_s * 1e3, "us_dense_w4a16": ms_d * 1e3,
+                         "gbs": by / (ms_t * 1e-3) / 1e9, "bytes": by,
+                         "roofline_frac": by / (pk["hbm_gbs"] * 1e9) / (ms_t * 1e-3),
+                         "speedup_vs_dense": ms_d / ms_t}
     assert q.qg_device_status() == q.QG_OK
     return res
 

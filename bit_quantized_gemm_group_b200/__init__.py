@@ -30,7 +30,7 @@ EXPORTS = ["qg_quantize_w4_group", "qg_pack_nibbles", "qg_gemm_w4a16", "qg_smoot
            "qg_last_error", "qg_selftest_bounded_wait", "qg_workspace_size", "qg_gemm_w4a16_noalloc",
            "qg_awq_act_mean", "qg_awq_scales", "qg_awq_scale_act", "qg_awq_search", "qg_outlier_split_w4",
            "qg_outlier_side_add", "qg_gemm_w4a16_outlier", "qg_prune24", "qg_pack24_vals", "qg_gemm_w4a16_24",
-           "qg_gptq", "qg_gptq_blocked"]
+           "qg_gptq", "qg_gptq_blocked", "qg_pack24_tc", "qg_gemm_w4a16_24_tc"]
 
 
 class QgError(RuntimeError):
@@ -58,6 +58,8 @@ _SIGS = {
     "qg_gemm_w4a16_outlier": [_P, _I, _I, _I, _I, _P, _P, _P, _I, _I, _P, _P, _P, _P, _P, _SZ, _P],
     "qg_gptq": [_P, _I, _I, _P, _I, _I, ctypes.c_double, _P, _P, _P, _P, _SZ, _P],
     "qg_gptq_blocked": [_P, _I, _I, _P, _I, _I, ctypes.c_double, _P, _P, _P, _P, _SZ, _P],
+    "qg_pack24_tc": [_P, _I, _I, _P, _P],
+    "qg_gemm_w4a16_24_tc": [_P, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P, _P, _SZ, _P],
     "qg_prune24": [_P, _I, _I, _P, _P, _P],
     "qg_pack24_vals": [_P, _P, _I, _I, _P, _P],
     "qg_gemm_w4a16_24": [_P, _I, _I, _I, _I, _P, _P, _P, _P, _I, _P, _P],
@@ -272,6 +274,19 @@ def qg_gemm_w4a16_24(X, vals, meta, scales, zeros, Y, group=128, stream=None):
     N = vals.shape[1]
     _check(lib().qg_gemm_w4a16_24(_ptr(X), _xdt(X), M, K, N, _ptr(vals), _ptr(meta), _ptr(scales), _ptr(zeros), group,
                                  _ptr(Y), _stream(stream)), "qg_gemm_w4a16_24")
+
+
+def qg_pack24_tc(vals, vals_tc, stream=None):
+    K16, N = vals.shape
+    _check(lib().qg_pack24_tc(_ptr(vals), 16 * K16, N, _ptr(vals_tc), _stream(stream)), "qg_pack24_tc")
+
+
+def qg_gemm_w4a16_24_tc(X, vals_tc, meta, scales, zeros, Y, group=128, workspace="auto", stream=None):
+    M, K = X.shape
+    N = vals_tc.shape[1]
+    wp, wb = _ws(workspace, QG_OP_GEMM_W4A16, M, K, N, X.device)
+    _check(lib().qg_gemm_w4a16_24_tc(_ptr(X), _xdt(X), M, K, N, _ptr(vals_tc), _ptr(meta), _ptr(scales), _ptr(zeros),
+                                    group, _ptr(Y), wp, wb, _stream(stream)), "qg_gemm_w4a16_24_tc")
 
 
 def qg_awq_act_mean(Xcal, xm, stream=None):

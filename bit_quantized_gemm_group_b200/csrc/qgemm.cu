@@ -9,6 +9,7 @@
 
 #include <algorithm>
 #include <atomic>
+#include <type_traits>
 #include <chrono>
 
 #include "../../include/qgemm.h"
@@ -360,14 +361,27 @@ template <> struct DecodeCfg<4> { static constexpr int NW = 8, GPS = 2, ST = 4, 
 
 int decode_cps(int MP) { return MP <= 8 ? DecodeCfg<1>::CPS : MP <= 16 ? DecodeCfg<2>::CPS : DecodeCfg<4>::CPS; }
 
-template <int MT, bool BF16>
+// 2:4 sparse INT4 (mma.sp): always the full dequantization; a group's weights take 6 KB
+// of a stage instead of 8 KB, so the rings hold more groups.  CPS matches the dense
+// configurations (one plan serves both).
+template <int MT> struct DecodeCfgSp;
+template <> struct DecodeCfgSp<1> { static constexpr int NW = 8, GPS = 4, ST = 6, CPS = 1, MINB = 1; static constexpr bool FULL = true, PWG = true; };
+template <> struct DecodeCfgSp<2> { static constexpr int NW = 8, GPS = 4, ST = 4, CPS = 1, MINB = 1; static constexpr bool FULL = true, PWG = true; };
+template <> struct DecodeCfgSp<4> { static constexpr int NW = 8, GPS = 2, ST = 5, CPS = 1, MINB = 1; static constexpr bool FULL = true, PWG = true; };
+static_assert(DecodeCfgSp<1>::CPS == DecodeCfg<1>::CPS && DecodeCfgSp<2>::CPS == DecodeCfg<2>::CPS &&
+                  DecodeCfgSp<4>::CPS == DecodeCfg<4>::CPS,
+              "one decode plan for the dense and the 2:4 kernels");
+
+// SP: `packed` is the 2:4 kept-code array in the tensor-core layout (qg_pack24_tc) and
+// `meta24` the position words; otherwise `packed` holds the dense words and meta24 is unused.
+template <int MT, bool BF16, bool SP = false>
 qg_status launch_w4a16_decode(const qg::SkinnyParams& sp, const uint32_t* packed, const uint16_t* scales,
-                              const uint8_t* zeros, void* ws, qg_stream_t stream)
+                              const uint8_t* zeros, void* ws, qg_stream_t stream, const uint32_t* meta24 = nullptr)
 {
-    using C = DecodeCfg<MT>;
-    using L = qg::DecodeSmem<MT, C::NW, C::GPS, C::ST, C::PWG>;
+    using C = std::conditional_t<SP, DecodeCfgSp<MT>, DecodeCfg<MT>>;
+    using L = qg::DecodeSmem<MT, C::NW, C::GPS, C::ST, C::PWG, SP>;
     static_assert(C::MINB * (L::TOTAL + 1024) <= 228 * 1024, "decode kernel shared memory");
-    auto kern = qg::w4a16_decode_kernel<MT, BF16, C::NW, C::GPS, C::ST, C::FULL, C::PWG, C::MINB>;
+    auto kern = qg::w4a16_decode_kernel<MT, BF16, C::NW, C::GPS, C::ST, C::FULL, C::PWG, C::MINB, SP>;
     const size_t smem = L::TOTAL;
     static KernelInfo info;
     int occ = 1;
@@ -376,9 +390,27 @@ qg_status launch_w4a16_decode(const qg::SkinnyParams& sp, const uint32_t* packed
     const DecodePlan d = decode_plan(sp.M, sp.K, sp.N);
     if (d.grid > C::CPS * num_sms()) return QG_ERR_UNSUPPORTED;  // plan and configuration disagree
     const bool narrow = sp.N % 32 != 0;
+    if (SP && narrow) return QG_ERR_SHAPE;
     qg::DecodeMaps m;
     const uint64_t N = sp.N, K = sp.K, G = d.G;
-    if (narrow) {
+    if (SP) {
+        // kept codes {32 columns, 8 rows of a group, N/32 blocks, G groups}; position words
+        // {32 columns, 4 rows of a group, N/32 blocks, G groups}; no swizzle (the lanes of a
+        // warp read whole 128-byte rows)
+        const uint64_t dv[4] = {32, 8, N / 32, G}, sv[3] = {N * 4, 128, 8 * N * 4};
+        const uint64_t dm[4] = {32, 4, N / 32, G}, sm[3] = {N * 4, 128, 4 * N * 4};
+        const uint32_t bvg[4] = {32, 8, 4, (uint32_t)C::GPS}, bv1[4] = {32, 8, 4, 1};
+        const uint32_t bmg[4] = {32, 4, 4, (uint32_t)C::GPS}, bm1[4] = {32, 4, 4, 1};
+        if ((st = make_tmap_nd(&m.wg, CU_TENSOR_MAP_DATA_TYPE_UINT32, packed, 4, dv, sv, bvg,
+                               CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK ||
+            (st = make_tmap_nd(&m.w1, CU_TENSOR_MAP_DATA_TYPE_UINT32, packed, 4, dv, sv, bv1,
+                               CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK ||
+            (st = make_tmap_nd(&m.mg, CU_TENSOR_MAP_DATA_TYPE_UINT32, meta24, 4, dm, sm, bmg,
+                               CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK ||
+            (st = make_tmap_nd(&m.m1, CU_TENSOR_MAP_DATA_TYPE_UINT32, meta24, 4, dm, sm, bm1,
+                               CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK)
+            return st;
+    } else if (narrow) {
         // [K/8][N] words, boxes {32 columns, 16 rows} (columns past N read as zero)
         if ((st = make_tmap_2d(&m.w1, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, packed, N, K / 8, 32, 16,
                                CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
@@ -1117,6 +1149,49 @@ qg_status qg_gemm_w4a16_24(const void* X, qg_dtype xdt, int M, int K, int N, con
     else
         qg::gemm_w4a16_24_kernel<MT, false><<<grid, block, 0, st>>>(x, M, K, N, vals, meta, scales, zeros, y);
     QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+
+qg_status qg_pack24_tc(const uint32_t* vals, int K, int N, uint32_t* vals_tc, qg_stream_t stream)
+{
+    if (!vals || !vals_tc) return QG_ERR_NULL;
+    if (K < 128 || K % 128 || N < 1) return QG_ERR_SHAPE;
+    if (misaligned(vals) || misaligned(vals_tc)) return QG_ERR_ALIGN;
+    if (vals == vals_tc) return QG_ERR_SHAPE;  // not in place
+    qg::pack24_tc_kernel<<<dim3((N + 255) / 256, K / 128), 256, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        vals, K, N, vals_tc);
+    QG_CUDA(cudaGetLastError());
+    return QG_OK;
+}
+
+qg_status qg_gemm_w4a16_24_tc(const void* X, qg_dtype xdt, int M, int K, int N, const uint32_t* vals_tc,
+                              const uint32_t* meta, const uint16_t* scales, const uint8_t* zeros, int group, void* Y,
+                              void* workspace, size_t ws_bytes, qg_stream_t stream)
+{
+    if (xdt != QG_F16 && xdt != QG_BF16) return QG_ERR_DTYPE;
+    if (M < 0 || K < 128 || K % 128 || N < 32 || N % 32 || group != 128) return QG_ERR_SHAPE;
+    if (M == 0) return QG_OK;
+    if (!X || !vals_tc || !meta || !scales || !zeros || !Y || !workspace) return QG_ERR_NULL;
+    if (misaligned(X) || misaligned(vals_tc) || misaligned(meta) || misaligned(scales) || misaligned(zeros) ||
+        misaligned(Y) || misaligned(workspace))
+        return QG_ERR_ALIGN;
+    if (ws_bytes < qg_workspace_size(QG_OP_GEMM_W4A16, M, K, N)) return QG_ERR_WORKSPACE;
+    const uint16_t* x = static_cast<const uint16_t*>(X);
+    uint16_t* y = static_cast<uint16_t*>(Y);
+    for (int m0 = 0; m0 < M; m0 += 32) {
+        qg::SkinnyParams q{x + (int64_t)m0 * K, vals_tc, scales, zeros, y + (int64_t)m0 * N, std::min(32, M - m0), K, N};
+        qg_status st;
+        if (xdt == QG_BF16) {
+            if (q.M <= 8) st = launch_w4a16_decode<1, true, true>(q, vals_tc, scales, zeros, workspace, stream, meta);
+            else if (q.M <= 16) st = launch_w4a16_decode<2, true, true>(q, vals_tc, scales, zeros, workspace, stream, meta);
+            else st = launch_w4a16_decode<4, true, true>(q, vals_tc, scales, zeros, workspace, stream, meta);
+        } else {
+            if (q.M <= 8) st = launch_w4a16_decode<1, false, true>(q, vals_tc, scales, zeros, workspace, stream, meta);
+            else if (q.M <= 16) st = launch_w4a16_decode<2, false, true>(q, vals_tc, scales, zeros, workspace, stream, meta);
+            else st = launch_w4a16_decode<4, false, true>(q, vals_tc, scales, zeros, workspace, stream, meta);
+        }
+        if (st != QG_OK) return st;
+    }
     return QG_OK;
 }
 

@@ -69,6 +69,35 @@ __global__ void __launch_bounds__(256) pack24_kernel(const uint8_t* __restrict__
     vals[(int64_t)vw * N + n] = word;
 }
 
+// The tensor-core layout of the kept codes (the mma.sp decode kernel's operand): per
+// group of 128 rows (32 blocks) and column, word u = 2 t + hb (t = 0..3, hb = 0..1) holds,
+// for the group's four 32-row steps s, the kept pair of block 8 s + t + 4 hb: its first
+// kept code at bits 4 s, its second at bits 16 + 4 s.  vals_tc[8 gq + u][n]; one thread per
+// (group, column) reads the group's 8 canonical words and writes its 8 words.
+__global__ void __launch_bounds__(256) pack24_tc_kernel(const uint32_t* __restrict__ vals, int K, int N,
+                                                        uint32_t* __restrict__ vals_tc)
+{
+    const int n = blockIdx.x * blockDim.x + threadIdx.x;
+    const int gq = blockIdx.y;
+    if (n >= N) return;
+    uint32_t v[8];
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v[w] = __ldg(vals + (int64_t)(8 * gq + w) * N + n);  // blocks 4w .. 4w + 3
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const int t = u >> 1, hb = u & 1;
+        uint32_t out = 0;
+#pragma unroll
+        for (int st = 0; st < 4; ++st) {
+            const int bl = 8 * st + t + 4 * hb;
+            const uint32_t byte = (v[bl >> 2] >> (8 * (bl & 3))) & 0xFFu;  // (second << 4) | first
+            out |= (byte & 0xFu) << (4 * st);
+            out |= (byte >> 4) << (16 + 4 * st);
+        }
+        vals_tc[(int64_t)(8 * gq + u) * N + n] = out;
+    }
+}
+
 // Y[m][n] = rn(sum over kept k of X[m][k] * (q - z) * s): one thread per column and MT
 // tokens; per group of 128 rows the thread reads its fp16 scale, zero, 8 value words and
 // 4 metadata words (each coalesced along N) and gathers X from L1/L2.  (q - z) * s is

@@ -16,14 +16,14 @@
 // of the other pieces, adds their tiles in CTA order (deterministic, no float atomics),
 // writes Y and clears the tokens.  One launch per call: no fix-up kernel.
 //
-// Footprint and overlap.  A CTA uses at most half of an SM (registers and shared
-// memory), so a second CTA can be resident beside it.  The kernel allows its
-// dependents to launch at once (programmatic dependent launch) and requests its first
-// ring-full of weights, scales and zeros before waiting for the previous grid: while
-// one call finishes, the next call's weights are already streaming.  X, Y and the
-// workspace are touched only after griddepcontrol.wait.
+// Overlap.  The kernel allows its dependents to launch at once (programmatic dependent
+// launch); a CTA of the next call starts on an SM as soon as this call's CTA there exits
+// and requests its first ring-full of weights, scales and zeros without waiting for the
+// previous grid.  X, Y and the workspace are touched only after griddepcontrol.wait: one
+// warp of the producer warpgroup waits and then requests each stage's activations right
+// after the stage's weights.
 //
-// Data movement.  One producer thread streams into a ring of stages, by TMA: the packed
+// Data movement.  Two producer threads stream into a ring of stages, by TMA: the packed
 // words (one 4-D box per stage, [group][32-column block][16 rows][128 B], 128-byte
 // swizzled), the fp16 scales and u8 zeros ([group][128 columns]) and the activation
 // tile ([half of 64 k][token][128 B], swizzled).  Consumer warp (wn, wg, ws) takes the 64 columns of half wn of group
@@ -64,6 +64,8 @@ struct DecodeParams {
 
 constexpr int kDecBN = 128;          // columns per slab
 constexpr int kDecGroupW = 8192;     // packed words of one group: 16 rows x 128 columns x 4 B
+constexpr int kDecGroupV24 = 4096;   // 2:4 kept codes of one group: 8 rows x 128 columns x 4 B
+constexpr int kDecGroupM24 = 2048;   // 2:4 position words of one group: 4 rows x 128 columns x 4 B
 
 QG_DEV_INLINE int dec_first_unit(int c, int units, int grid) { return (int)((int64_t)c * units / grid); }
 
@@ -78,12 +80,14 @@ QG_DEV_INLINE int dec_cta_of_unit(int u, int units, int grid)
 
 // Shared memory of one CTA: ST stages of GPS groups, the k-warp reduction tiles and
 // the stage mbarriers.
-template <int MT, int NW, int GPS, int ST, bool PWG>
+template <int MT, int NW, int GPS, int ST, bool PWG, bool SP = false>
 struct DecodeSmem {
     static constexpr int MP = 8 * MT;
+    // weight bytes of one group: packed words, or (2:4) kept codes then position words
+    static constexpr int WB = SP ? kDecGroupV24 + kDecGroupM24 : kDecGroupW;
     static constexpr int KW = NW / 2;                 // k-warps per column half
     static constexpr int XG = MP * 256;               // X bytes per group: [2 halves][MP][128 B]
-    static constexpr int X_OFF = GPS * kDecGroupW;
+    static constexpr int X_OFF = GPS * WB;
     static constexpr int S_OFF = X_OFF + GPS * XG;    // fp16 scales [GPS][128]
     static constexpr int Z_OFF = S_OFF + GPS * 256;   // u8 zeros [GPS][128]
     static constexpr int STAGE = (Z_OFF + GPS * 128 + 1023) / 1024 * 1024;
@@ -91,16 +95,16 @@ struct DecodeSmem {
     static constexpr int TS = kDecBN + 4;            // row stride (floats) of the [token][column] result tile
     static constexpr int RED_K = (KW - 1) * 2 * FRAG * 32 * 16;  // k-warp reduction (fragment layout)
     static constexpr int RED = RED_K > MP * TS * 4 ? RED_K : MP * TS * 4;  // the result tile aliases it
-    static constexpr int TOTAL = ST * STAGE + RED + 2 * ST * 8 + 1024;
+    static constexpr int TOTAL = ST * STAGE + RED + 3 * ST * 8 + 1024;
     // The producer is one warp after the consumers, or (PWG) a whole warpgroup of which
     // the first warp works, so that the register file can be split with setmaxnreg: the
-    // producer keeps 32 registers a thread and the consumers take the rest.
+    // producer warps keep 56 registers a thread and the consumers take the rest.
     static constexpr int THREADS = 32 * NW + (PWG ? 128 : 32);
     static constexpr int REG_LAUNCH = (65536 / THREADS) / 8 * 8 > 255 ? 248 : (65536 / THREADS) / 8 * 8;
-    static constexpr int REG_PRODUCER = 32;
+    static constexpr int REG_PRODUCER = 56;
     static constexpr int REG_CONSUMER_RAW = (REG_LAUNCH * THREADS - REG_PRODUCER * 128) / (32 * NW) / 8 * 8;
     static constexpr int REG_CONSUMER = REG_CONSUMER_RAW > 248 ? 248 : REG_CONSUMER_RAW;
-    static constexpr uint32_t GROUP_TX = kDecGroupW + XG + 384;  // TMA bytes of one group
+    static constexpr uint32_t GROUP_TX = WB + XG + 384;  // TMA bytes of one group
     static constexpr int PARTIAL_FLOATS = 2 * FRAG * 32 * 4;  // one CTA's partial tile (128 x MP)
 };
 
@@ -112,6 +116,7 @@ struct DecodeMaps {
     CUtensorMap sg, s1, zg, z1;  // fp16 scales / u8 zeros: {128 columns, GPS | 1 groups}
     CUtensorMap wg, w1;  // packed words, GPS groups / 1 group (4-D), or the 2-D per-block map in w1
     CUtensorMap xg, x1;  // activations, GPS groups / 1 group
+    CUtensorMap mg, m1;  // 2:4 position words {32 columns, 4 rows, N/32 blocks, G groups}, GPS groups / 1 group
 };
 
 QG_DEV_INLINE void tma_load_4d(const CUtensorMap* m, uint64_t* bar, void* smem_dst, int x, int y, int z, int w)
@@ -155,12 +160,13 @@ struct DecodeSchedule {
     }
 };
 
-template <int MT, bool BF16, int NW, int GPS, int ST, bool FULL, bool PWG, int MINB>
-__global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG>::THREADS, MINB)
+template <int MT, bool BF16, int NW, int GPS, int ST, bool FULL, bool PWG, int MINB, bool SP>
+__global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG, SP>::THREADS, MINB)
     w4a16_decode_kernel(const DecodeParams p, const __grid_constant__ DecodeMaps maps)
 {
     using H = HalfOps<BF16>;
-    using L = DecodeSmem<MT, NW, GPS, ST, PWG>;
+    using L = DecodeSmem<MT, NW, GPS, ST, PWG, SP>;
+    static_assert(!SP || FULL, "the 2:4 path dequantizes in full");
     constexpr int MP = L::MP;
     constexpr int KW = L::KW;
     constexpr int WS = KW / GPS;   // warps sharing one group of a column half
@@ -172,6 +178,7 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG>::THREADS, MIN
     float4* red = reinterpret_cast<float4*>(smem + ST * L::STAGE);
     uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * L::STAGE + L::RED);
     uint64_t* empty = full + ST;
+    uint64_t* armed = empty + ST;  // the producer has set up a stage's fill (its expected bytes)
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.G;
@@ -182,34 +189,59 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG>::THREADS, MIN
         for (int i = 0; i < ST; ++i) {
             mbar_init(&full[i], 1);
             mbar_init(&empty[i], NW);
+            mbar_init(&armed[i], 1);
         }
         fence_mbar_init();
     }
     __syncthreads();
 
+    static_assert(PWG, "the producer warpgroup holds the weight and the activation issuers");
     if (warp >= NW) {
-        // ---------------- producer warpgroup (warp NW works) ----------------
-        if constexpr (PWG) {
-            asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(L::REG_PRODUCER));
-            if (warp != NW) return;
+        // ---------------- producer warpgroup ----------------
+        // Warp NW streams the weights (with scales and zeros) from the start: they do not
+        // depend on the previous grid.  Warp NW + 1 waits for the previous grid once and
+        // then requests each fill's activations as soon as the weight issuer has set the
+        // fill up, so a CTA that starts late (after the previous grid ended) gets its first
+        // stage's activations right behind that stage's weights, not behind the whole ring.
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(L::REG_PRODUCER));
+        if (warp > NW + 1) return;
+        if (warp == NW + 1) {
+            if (lane == 0) {
+                tma_prefetch_desc(&maps.xg);
+                tma_prefetch_desc(&maps.x1);
+            }
+            asm volatile("griddepcontrol.wait;" ::: "memory");
+            int stage = 0;
+            uint32_t phase = 0;
+            DecodeSchedule sc(u0, u1, G);
+            for (bool ok = true; !sc.done() && ok; sc.next_piece()) {
+                for (int g0 = sc.ga; g0 < sc.gb; g0 += GPS) {
+                    const int ng = min(GPS, sc.gb - g0);
+                    if (!__all_sync(0xffffffffu, mbar_wait(&armed[stage], phase))) { ok = false; break; }
+                    if (lane == 0) {
+                        uint8_t* st = ring + stage * L::STAGE;
+                        if (ng == GPS)
+                            tma_load_3d(&maps.xg, &full[stage], st + L::X_OFF, 0, 0, 2 * g0);
+                        else
+                            for (int i = 0; i < ng; ++i)
+                                tma_load_3d(&maps.x1, &full[stage], st + L::X_OFF + i * L::XG, 0, 0, 2 * (g0 + i));
+                    }
+                    if (++stage == ST) { stage = 0; phase ^= 1; }
+                }
+            }
+            return;
         }
         if (lane == 0) {
             tma_prefetch_desc(&maps.wg);
             tma_prefetch_desc(&maps.w1);
-            tma_prefetch_desc(&maps.xg);
-            tma_prefetch_desc(&maps.x1);
+            if constexpr (SP) {
+                tma_prefetch_desc(&maps.mg);
+                tma_prefetch_desc(&maps.m1);
+            }
         }
         int stage = 0, issued = 0;
         uint32_t phase = 0;
-        bool waited = false, ok = true;
-        int pend_g0[ST], pend_ng[ST];
-        auto load_x = [&](int st_i, int g0, int ng) {
-            uint8_t* st = ring + st_i * L::STAGE;
-            if (ng == GPS)
-                tma_load_3d(&maps.xg, &full[st_i], st + L::X_OFF, 0, 0, 2 * g0);
-            else
-                for (int i = 0; i < ng; ++i) tma_load_3d(&maps.x1, &full[st_i], st + L::X_OFF + i * L::XG, 0, 0, 2 * (g0 + i));
-        };
+        bool ok = true;
         DecodeSchedule sc(u0, u1, G);
         for (; !sc.done() && ok; sc.next_piece()) {
             const int x = sc.slab * kDecBN;
@@ -221,7 +253,20 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG>::THREADS, MIN
                 uint8_t* st = ring + stage * L::STAGE;
                 if (lane == 0) {
                     mbar_arrive_expect_tx(&full[stage], (uint32_t)ng * L::GROUP_TX);
-                    if (p.narrow) {
+                    if constexpr (SP) {
+                        // kept codes [group][block][8 rows][128 B], then position words
+                        // [group][block][4 rows][128 B]
+                        if (ng == GPS) {
+                            tma_load_4d(&maps.wg, &full[stage], st, 0, 0, x / 32, g0);
+                            tma_load_4d(&maps.mg, &full[stage], st + GPS * kDecGroupV24, 0, 0, x / 32, g0);
+                        } else {
+                            for (int i = 0; i < ng; ++i) {
+                                tma_load_4d(&maps.w1, &full[stage], st + i * kDecGroupV24, 0, 0, x / 32, g0 + i);
+                                tma_load_4d(&maps.m1, &full[stage], st + GPS * kDecGroupV24 + i * kDecGroupM24, 0, 0,
+                                            x / 32, g0 + i);
+                            }
+                        }
+                    } else if (p.narrow) {
                         for (int i = 0; i < ng; ++i)
 #pragma unroll
                             for (int b = 0; b < 4; ++b)
@@ -233,8 +278,6 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG>::THREADS, MIN
                         for (int i = 0; i < ng; ++i)
                             tma_load_4d(&maps.w1, &full[stage], st + i * kDecGroupW, 0, 0, x / 32, g0 + i);
                     }
-                }
-                if (lane == 0) {
                     if (ng == GPS) {
                         tma_load_2d(&maps.sg, &full[stage], st + L::S_OFF, x, g0);
                         tma_load_2d(&maps.zg, &full[stage], st + L::Z_OFF, x, g0);
@@ -244,33 +287,14 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG>::THREADS, MIN
                             tma_load_2d(&maps.z1, &full[stage], st + L::Z_OFF + i * 128, x, g0 + i);
                         }
                     }
-                }
-                if (lane == 0) {
-                    if (!waited && issued < ST) {
-                        pend_g0[issued] = g0;
-                        pend_ng[issued] = ng;
-                    }
-                    if (waited) load_x(stage, g0, ng);
-                }
-                if (!waited && (issued + 1 == ST)) {
-                    // ring full: wait for the previous grid, then request the activations
-                    asm volatile("griddepcontrol.wait;" ::: "memory");
-                    waited = true;
-                    if (lane == 0)
-                        for (int j = 0; j <= issued; ++j) load_x(j, pend_g0[j], pend_ng[j]);
+                    mbar_arrive(&armed[stage]);  // the activation issuer may now add its copy
                 }
                 ++issued;
                 if (++stage == ST) { stage = 0; phase ^= 1; }
             }
         }
-        if (!waited) {
-            // the schedule (or a bounded wait) ended inside the first ring-full: complete
-            // the stages requested so far so that every copy in flight can land
-            asm volatile("griddepcontrol.wait;" ::: "memory");
-            if (lane == 0)
-                for (int j = 0; j < issued; ++j) load_x(j, pend_g0[j], pend_ng[j]);
-        }
-        // every TMA copy still in flight lands before the CTA exits
+        // every TMA copy still in flight lands before the CTA exits (bounded waits: a fill
+        // whose activations were never requested gives up)
         if (lane == 0)
             for (int j = issued - ST > 0 ? issued - ST : 0; j < issued; ++j) mbar_wait(&full[j % ST], (j / ST) & 1);
         return;
@@ -328,6 +352,64 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG>::THREADS, MIN
                                 z2[h][c] = H::splat(zb);   // exact (integer <= 143, or 1024 + z)
                             }
                     }
+                    if constexpr (SP) {
+                        // 2:4: mma.sp m16n8k32, weights compressed (two kept codes of each
+                        // 4-block) as the m16 operand.  The lane's kept-code words: rows
+                        // 2 t4 (its block t4 of each step) and 2 t4 + 1 (block t4 + 4) of
+                        // columns 4 g8 .. 4 g8 + 3; nibble pair s of a word (bits 4s and 16 + 4s)
+                        // is step s's pair, extracted with one shift and one LOP3.
+                        const uint8_t* vbase = st + gi * kDecGroupV24;
+                        const uint8_t* mbase = st + GPS * kDecGroupV24 + gi * kDecGroupM24;
+                        const uint8_t* xgrp = st + L::X_OFF + gi * L::XG;
+                        uint4 va[2][2];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h)
+#pragma unroll
+                            for (int hb = 0; hb < 2; ++hb)
+                                va[h][hb] = *reinterpret_cast<const uint4*>(vbase + (2 * wn + h) * 1024 +
+                                                                            (2 * t4 + hb) * 128 + g8 * 16);
+                        // position words: lanes t4 = 0 / 1 give the MMA blocks 0-3 / 4-7 of
+                        // both rows (selector 0); the other lanes' are not read
+                        const uint32_t msel = (t4 & 1) ? 0x7632u : 0x5410u;
+#pragma unroll
+                        for (int si = 0; si < SPW; ++si) {
+                            const int s = ws * SPW + si;
+                            // activations in natural k order: B rows 2 t4 + 8 i (+1), i = 0..3
+                            uint32_t xb[MT][4];
+                            const uint8_t* xs = xgrp + (s >> 1) * (MP * 128);
+#pragma unroll
+                            for (int j = 0; j < MT; ++j) {
+                                const int tok = 8 * j + g8;  // rows >= M are zero (TMA fill)
+#pragma unroll
+                                for (int i = 0; i < 4; ++i)
+                                    xb[j][i] = *reinterpret_cast<const uint32_t*>(
+                                        xs + tok * 128 + (((4 * (s & 1) + i) ^ (tok & 7)) << 4) + 4 * t4);
+                            }
+#pragma unroll
+                            for (int h = 0; h < 2; ++h) {
+                                const uint4 mv = *reinterpret_cast<const uint4*>(mbase + (2 * wn + h) * 512 + s * 128 + g8 * 16);
+                                const uint32_t w0[4] = {va[h][0].x, va[h][0].y, va[h][0].z, va[h][0].w};
+                                const uint32_t w1[4] = {va[h][1].x, va[h][1].y, va[h][1].z, va[h][1].w};
+#pragma unroll
+                                for (int cp = 0; cp < 2; ++cp) {
+                                    // MMA row g8 <-> column 4 g8 + 2 cp, row g8 + 8 <-> column 4 g8 + 2 cp + 1
+                                    uint32_t a0 = lop3_and_or(w0[2 * cp] >> (4 * s), 0x000F000Fu, H::MAGIC);
+                                    uint32_t a1 = lop3_and_or(w0[2 * cp + 1] >> (4 * s), 0x000F000Fu, H::MAGIC);
+                                    uint32_t a2 = lop3_and_or(w1[2 * cp] >> (4 * s), 0x000F000Fu, H::MAGIC);
+                                    uint32_t a3 = lop3_and_or(w1[2 * cp + 1] >> (4 * s), 0x000F000Fu, H::MAGIC);
+                                    a0 = H::mul2(H::sub2(a0, z2[h][2 * cp]), s2[h][2 * cp]);
+                                    a1 = H::mul2(H::sub2(a1, z2[h][2 * cp + 1]), s2[h][2 * cp + 1]);
+                                    a2 = H::mul2(H::sub2(a2, z2[h][2 * cp]), s2[h][2 * cp]);
+                                    a3 = H::mul2(H::sub2(a3, z2[h][2 * cp + 1]), s2[h][2 * cp + 1]);
+                                    const uint32_t meta = prmt(cp ? mv.z : mv.x, cp ? mv.w : mv.y, msel);
+#pragma unroll
+                                    for (int j = 0; j < MT; ++j)
+                                        mma_sp_16832<BF16>(acc[h][cp][j], a0, a1, a2, a3, xb[j][0], xb[j][1], xb[j][2],
+                                                           xb[j][3], meta);
+                                }
+                            }
+                        }
+                    } else {
                     float D[2][2][MT][4], Dx[MT][4];
                     if constexpr (!FULL) {
 #pragma unroll
@@ -420,6 +502,7 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG>::THREADS, MIN
                                     for (int e = e0; e < e0 + 2; ++e)
                                         acc[h][cp][j][e] = fmaf(sv, fmaf(-zb, Dx[j][e & 1], D[h][cp][j][e]), acc[h][cp][j][e]);
                             }
+                    }
                     }
                 }
             }

@@ -52,6 +52,25 @@ struct HalfOps {
     QG_DEV_INLINE static uint16_t to_bits(float v) { return BF16 ? f32_to_bf16_bits(v) : f32_to_f16_bits(v); }
 };
 
+// Sparse m16n8k32 (2:4 along k): a0..a3 hold the kept pairs of the compressed A
+// (row g, block t | row g + 8, block t | row g, block t + 4 | row g + 8, block t + 4),
+// b0..b3 the dense B rows 2t + 8i (+1), e the position nibbles (selector 0: lanes t = 0, 1).
+template <bool BF16>
+QG_DEV_INLINE void mma_sp_16832(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
+                                uint32_t b1, uint32_t b2, uint32_t b3, uint32_t e)
+{
+    if constexpr (BF16)
+        asm("mma.sp::ordered_metadata.sync.aligned.m16n8k32.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, "
+            "{%4,%5,%6,%7}, {%8,%9,%10,%11}, {%0,%1,%2,%3}, %12, 0x0;"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(b2), "r"(b3), "r"(e));
+    else
+        asm("mma.sp::ordered_metadata.sync.aligned.m16n8k32.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, "
+            "{%4,%5,%6,%7}, {%8,%9,%10,%11}, {%0,%1,%2,%3}, %12, 0x0;"
+            : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1), "r"(b2), "r"(b3), "r"(e));
+}
+
 template <bool BF16>
 QG_DEV_INLINE void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3, uint32_t b0,
                              uint32_t b1)

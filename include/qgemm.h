@@ -306,6 +306,30 @@ qg_status qg_gemm_w4a16_24(const void* X, qg_dtype xdt, int M, int K, int N, con
                            int group, void* Y, qg_stream_t stream);
 
 /* --------------------------------------------------------------------------
+ * Tensor-core form of the 2:4 GEMM (few tokens).   [G] sec. 3.2
+ *
+ * qg_pack24_tc: the kept codes of qg_pack24_vals rearranged for the sparse tensor-core
+ *   instruction (mma.sp m16n8k32; an offline step, like packing): per group of 128 rows
+ *   (32 blocks of 4) and column n, word vals_tc[8 gq + u][n], u = 2 t + hb (t = 0..3,
+ *   hb = 0..1), holds for each 32-row step s = 0..3 of the group the two kept codes of
+ *   block 8 s + t + 4 hb: the first (smaller k) at bits 4 s, the second at bits 16 + 4 s.
+ *   vals u32 [K/16][N] (qg_pack24_vals) -> vals_tc u32 [K/16][N]; not in place.
+ *   Rules: K % 128 == 0.
+ * qg_gemm_w4a16_24_tc: Y = X * deq(W) as qg_gemm_w4a16_24 (pruned positions contribute
+ *   exactly 0), from vals_tc, the position words meta (qg_prune24's, unchanged) and the
+ *   asymmetric scales and zeros: a stream-K kernel streaming 0.375 byte per weight, each
+ *   kept pair dequantized to (q - z) s in the activation dtype (exact subtraction, one
+ *   rounding) and accumulated in fp32 by mma.sp.  Launches of up to 32 tokens.
+ *   Rules: group == 128, K % 128 == 0, N % 32 == 0; workspace required, at least
+ *   qg_workspace_size(QG_OP_GEMM_W4A16, M, K, N) bytes (the decode kernel's contract:
+ *   contents need no initialisation; concurrent calls must not share one).
+ * ------------------------------------------------------------------------ */
+qg_status qg_pack24_tc(const uint32_t* vals, int K, int N, uint32_t* vals_tc, qg_stream_t stream);
+qg_status qg_gemm_w4a16_24_tc(const void* X, qg_dtype xdt, int M, int K, int N, const uint32_t* vals_tc,
+                              const uint32_t* meta, const uint16_t* scales, const uint8_t* zeros, int group,
+                              void* Y, void* workspace, size_t ws_bytes, qg_stream_t stream);
+
+/* --------------------------------------------------------------------------
  * GPTQ: INT4 weights with Hessian-weighted error compensation.   [A] sec. 3.1-3.3
  *
  *   H = (2/Mc) Xcal^T Xcal + lambda I, lambda = damp * trace / K (damp if the trace

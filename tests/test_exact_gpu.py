@@ -153,9 +153,14 @@ def test_w4a8_exact(M, workspace):
 # ---------------------------------------------------------------------------
 # 2:4 sparse INT4
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("M", [1, 4, 17])
-def test_w4a16_24_exact(M):
-    K, N = 4096, 1024
+@pytest.mark.parametrize("M", [1, 4, 17, 32, 45])
+@pytest.mark.parametrize("tc", [False, True])
+def test_w4a16_24_exact(M, tc):
+    """Both 2:4 GEMMs: the SIMT kernel on the canonical layout and the mma.sp decode
+    kernel on the tensor-core layout (qg_pack24_tc), on a full decode width."""
+    K, N = 4096, 1024 if not tc else 12288
+    if not tc and M > 17:
+        pytest.skip("the SIMT kernel is covered at M <= 17")
     codes, scales, zeros = synth.exact_w4_asym(K, N, seed=9)
     # a 2:4 pattern along K: two positions per block of four, drawn at random; the
     # oracle's pruning keeps exactly them (kept magnitudes 2..3, dropped 0..1)
@@ -170,9 +175,16 @@ def test_w4a16_24_exact(M):
     X, Xb = synth.exact_activations(M, K, seed=M)
     q = qlib()
     Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
-    q.qg_gemm_w4a16_24(x_device(Xb, torch.bfloat16), cuda(vals.view(np.int32)), cuda(meta.view(np.int32)),
-                       cuda(scales.view(np.int16)), cuda(zeros), Y)
+    vd = cuda(vals.view(np.int32))
+    if tc:
+        vt = torch.full_like(vd, -1)
+        q.qg_pack24_tc(vd, vt)
+        q.qg_gemm_w4a16_24_tc(x_device(Xb, torch.bfloat16), vt, cuda(meta.view(np.int32)),
+                              cuda(scales.view(np.int16)), cuda(zeros), Y)
+    else:
+        q.qg_gemm_w4a16_24(x_device(Xb, torch.bfloat16), vd, cuda(meta.view(np.int32)),
+                           cuda(scales.view(np.int16)), cuda(zeros), Y)
     st = q.qg_device_status()
     assert st == q.QG_OK, q.qg_status_string(st)
     yref, _ = oracle.gemm_w4a16_24_ref(X, vals, meta, scales, zeros)
-    assert_bits(u16(Y), expected_bits(yref, "bf16"), f"2:4 M={M}")
+    assert_bits(u16(Y), expected_bits(yref, "bf16"), f"2:4 M={M} tc={tc}")

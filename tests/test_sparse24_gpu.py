@@ -92,3 +92,71 @@ def test_gemm_within_tolerance(M, N, xdt):
     yref, b = oracle.gemm_w4a16_24_ref(X, *ref)
     ok = oracle.within_tolerance(y, yref, b)
     assert ok.all(), f"{(~ok).sum()} outside tolerance"
+
+
+# ---------------------------------------------------------------------------
+# the tensor-core form: qg_pack24_tc + qg_gemm_w4a16_24_tc (mma.sp decode kernel)
+# ---------------------------------------------------------------------------
+def _tc_layout(vals):
+    """The documented tensor-core layout, restated here from its definition in the header:
+    word u = 2t + hb of group gq holds, for step s, block 8s + t + 4hb's first kept code at
+    bits 4s and its second at bits 16 + 4s."""
+    K16, N = vals.shape
+    out = np.zeros_like(vals)
+    for gq in range(K16 // 8):
+        v = vals[8 * gq:8 * gq + 8].astype(np.uint64)
+        for u in range(8):
+            t, hb = u >> 1, u & 1
+            w = np.zeros(N, np.uint64)
+            for s in range(4):
+                bl = 8 * s + t + 4 * hb
+                byte = (v[bl >> 2] >> np.uint64(8 * (bl & 3))) & np.uint64(0xFF)
+                w |= (byte & np.uint64(0xF)) << np.uint64(4 * s)
+                w |= (byte >> np.uint64(4)) << np.uint64(16 + 4 * s)
+            out[8 * gq + u] = w.astype(np.uint32)
+    return out
+
+
+def _tc_operands(vals):
+    q = qlib()
+    vals_tc = torch.full_like(vals, -1)
+    q.qg_pack24_tc(vals, vals_tc)
+    _status_ok()
+    np.testing.assert_array_equal(vals_tc.cpu().numpy().view(np.uint32), _tc_layout(vals.cpu().numpy().view(np.uint32)))
+    return vals_tc
+
+
+@pytest.mark.parametrize("M,N,xdt", [(1, 12288, "bf16"), (16, 12288, "bf16"), (4, 384, "bf16"), (17, 160, "bf16"),
+                                     (32, 256, "bf16"), (45, 96, "bf16"), (3, 224, "f16")])
+def test_tc_gemm_within_tolerance(M, N, xdt):
+    q = qlib()
+    K = 4096 if N == 12288 else 512
+    W = synth.weights(K, N, 0.02, 0.01, 8.0, seed=M + N + 1)
+    (vals, meta, scales, zeros), ref = _sparse_weights(W)
+    vals_tc = _tc_operands(vals)
+    X, Xb = synth.activations(M, K, xdt, seed=M)
+    dt = torch.bfloat16 if xdt == "bf16" else torch.float16
+    Y = torch.full((M, N), float("nan"), dtype=dt, device="cuda")
+    q.qg_gemm_w4a16_24_tc(x_device(Xb, dt), vals_tc, meta, scales, zeros, Y)
+    _status_ok()
+    y = (bf16_to_f32 if xdt == "bf16" else f16_to_f32)(u16(Y))
+    yref, b = oracle.gemm_w4a16_24_ref(X, *ref)
+    ok = oracle.within_tolerance(y, yref, b)
+    assert ok.all(), f"{(~ok).sum()} outside tolerance"
+
+
+def test_tc_repeat_calls_identical():
+    q = qlib()
+    K, N, M = 4096, 12288, 4
+    W = synth.weights(K, N, 0.02, 0.01, 8.0, seed=3)
+    (vals, meta, scales, zeros), _ = _sparse_weights(W)
+    vals_tc = _tc_operands(vals)
+    _, Xb = synth.activations(M, K, "bf16", seed=3)
+    Xd = x_device(Xb, torch.bfloat16)
+    outs = []
+    for _ in range(3):
+        Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+        q.qg_gemm_w4a16_24_tc(Xd, vals_tc, meta, scales, zeros, Y)
+        outs.append(u16(Y))
+    _status_ok()
+    assert np.array_equal(outs[0], outs[1]) and np.array_equal(outs[0], outs[2])
