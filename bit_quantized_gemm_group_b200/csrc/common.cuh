@@ -191,6 +191,13 @@ QG_DEV_INLINE void named_bar_sync(uint32_t id, uint32_t count)
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+// Arrive on named barrier `id` without waiting (the threads that bar.sync on it wait for
+// `count` arrivals in all); the caller's earlier shared-memory writes are visible to them.
+QG_DEV_INLINE void named_bar_arrive(uint32_t id, uint32_t count)
+{
+    asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 QG_DEV_INLINE void fence_proxy_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------

@@ -368,20 +368,37 @@ template <int MT> struct DecodeCfgSp;
 template <> struct DecodeCfgSp<1> { static constexpr int NW = 8, GPS = 4, ST = 6, CPS = 1, MINB = 1; static constexpr bool FULL = true, PWG = true; };
 template <> struct DecodeCfgSp<2> { static constexpr int NW = 8, GPS = 4, ST = 4, CPS = 1, MINB = 1; static constexpr bool FULL = true, PWG = true; };
 template <> struct DecodeCfgSp<4> { static constexpr int NW = 8, GPS = 2, ST = 5, CPS = 1, MINB = 1; static constexpr bool FULL = true, PWG = true; };
+// The outlier side path fused (OUT): each stage also holds the groups' outlier offsets,
+// codes and scales (6 KB for 4 groups), so the rings are one stage shorter.
+template <int MT> struct DecodeCfgOut;
+template <> struct DecodeCfgOut<1> { static constexpr int NW = 8, GPS = 4, ST = 4, CPS = 1, MINB = 1; static constexpr bool FULL = false, PWG = true; };
+template <> struct DecodeCfgOut<2> { static constexpr int NW = 8, GPS = 4, ST = 3, CPS = 1, MINB = 1; static constexpr bool FULL = true, PWG = true; };
+template <> struct DecodeCfgOut<4> { static constexpr int NW = 8, GPS = 2, ST = 3, CPS = 1, MINB = 1; static constexpr bool FULL = true, PWG = true; };
 static_assert(DecodeCfgSp<1>::CPS == DecodeCfg<1>::CPS && DecodeCfgSp<2>::CPS == DecodeCfg<2>::CPS &&
-                  DecodeCfgSp<4>::CPS == DecodeCfg<4>::CPS,
-              "one decode plan for the dense and the 2:4 kernels");
+                  DecodeCfgSp<4>::CPS == DecodeCfg<4>::CPS && DecodeCfgOut<1>::CPS == DecodeCfg<1>::CPS &&
+                  DecodeCfgOut<2>::CPS == DecodeCfg<2>::CPS && DecodeCfgOut<4>::CPS == DecodeCfg<4>::CPS,
+              "one decode plan for the dense, the 2:4 and the side-path kernels");
+
+// The outlier side path of one decode launch (qg_gemm_w4a16_outlier's arrays).
+struct DecodeOutliers {
+    const uint8_t* idx;
+    const int8_t* codes8;
+    const float* s8;
+    int count;
+};
 
 // SP: `packed` is the 2:4 kept-code array in the tensor-core layout (qg_pack24_tc) and
 // `meta24` the position words; otherwise `packed` holds the dense words and meta24 is unused.
-template <int MT, bool BF16, bool SP = false>
+// OUT: the outlier side path `out` is fused (dense weights only).
+template <int MT, bool BF16, bool SP = false, bool OUT = false>
 qg_status launch_w4a16_decode(const qg::SkinnyParams& sp, const uint32_t* packed, const uint16_t* scales,
-                              const uint8_t* zeros, void* ws, qg_stream_t stream, const uint32_t* meta24 = nullptr)
+                              const uint8_t* zeros, void* ws, qg_stream_t stream, const uint32_t* meta24 = nullptr,
+                              const DecodeOutliers* out = nullptr)
 {
-    using C = std::conditional_t<SP, DecodeCfgSp<MT>, DecodeCfg<MT>>;
-    using L = qg::DecodeSmem<MT, C::NW, C::GPS, C::ST, C::PWG, SP>;
+    using C = std::conditional_t<SP, DecodeCfgSp<MT>, std::conditional_t<OUT, DecodeCfgOut<MT>, DecodeCfg<MT>>>;
+    using L = qg::DecodeSmem<MT, C::NW, C::GPS, C::ST, C::PWG, SP, OUT>;
     static_assert(C::MINB * (L::TOTAL + 1024) <= 228 * 1024, "decode kernel shared memory");
-    auto kern = qg::w4a16_decode_kernel<MT, BF16, C::NW, C::GPS, C::ST, C::FULL, C::PWG, C::MINB, SP>;
+    auto kern = qg::w4a16_decode_kernel<MT, BF16, C::NW, C::GPS, C::ST, C::FULL, C::PWG, C::MINB, SP, OUT>;
     const size_t smem = L::TOTAL;
     static KernelInfo info;
     int occ = 1;
@@ -445,6 +462,21 @@ qg_status launch_w4a16_decode(const qg::SkinnyParams& sp, const uint32_t* packed
                            CU_TENSOR_MAP_SWIZZLE_128B)) != QG_OK)
         return st;
     qg::DecodeParams p;
+    p.ocount = 0;
+    p.side_tx = 0;
+    if (OUT) {
+        if (!out || out->count < 1 || out->count > qg::kDecOutMax) return QG_ERR_SHAPE;
+        const uint32_t cnt = (uint32_t)out->count;
+        if ((st = make_tmap_3d(&m.oi, CU_TENSOR_MAP_DATA_TYPE_UINT8, out->idx, N, cnt, G, N, cnt * N, 128, cnt, C::GPS,
+                               CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK ||
+            (st = make_tmap_3d(&m.oc, CU_TENSOR_MAP_DATA_TYPE_UINT8, out->codes8, N, cnt, G, N, cnt * N, 128, cnt,
+                               C::GPS, CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK ||
+            (st = make_tmap_2d(&m.os, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, out->s8, N, G, 128, C::GPS,
+                               CU_TENSOR_MAP_SWIZZLE_NONE)) != QG_OK)
+            return st;
+        p.ocount = out->count;
+        p.side_tx = (uint32_t)C::GPS * (2 * cnt * 128 + 512);
+    }
     p.X = sp.X;
     p.scales = scales;
     p.zeros = zeros;
@@ -1101,6 +1133,31 @@ qg_status qg_gemm_w4a16_outlier(const void* X, qg_dtype xdt, int M, int K, int N
 {
     qg_status st = outlier_side_args(X, xdt, M, K, N, group, count, idx, codes8, s8, Y);
     if (st != QG_OK) return st;
+    if (M == 0) return QG_OK;
+    if (workspace && count >= 1 && count <= qg::kDecOutMax && group == 128 && K >= 128 && K % 128 == 0 &&
+        decode_eligible(M, N) && !(xdt == QG_BF16 && M >= qg::kTcMinM)) {
+        // the side path fused into the decode kernel: Y rounded once
+        if (!packed || !scales || !zeros) return QG_ERR_NULL;
+        if (misaligned(packed) || misaligned(scales) || misaligned(zeros) || misaligned(workspace)) return QG_ERR_ALIGN;
+        if (ws_bytes < qg_workspace_size(QG_OP_GEMM_W4A16, M, K, N)) return QG_ERR_WORKSPACE;
+        const DecodeOutliers o{idx, codes8, s8, count};
+        const uint16_t* x = static_cast<const uint16_t*>(X);
+        uint16_t* y = static_cast<uint16_t*>(Y);
+        for (int m0 = 0; m0 < M; m0 += 32) {
+            qg::SkinnyParams q{x + (int64_t)m0 * K, packed, scales, zeros, y + (int64_t)m0 * N, std::min(32, M - m0), K, N};
+            if (xdt == QG_BF16) {
+                if (q.M <= 8) st = launch_w4a16_decode<1, true, false, true>(q, packed, scales, zeros, workspace, stream, nullptr, &o);
+                else if (q.M <= 16) st = launch_w4a16_decode<2, true, false, true>(q, packed, scales, zeros, workspace, stream, nullptr, &o);
+                else st = launch_w4a16_decode<4, true, false, true>(q, packed, scales, zeros, workspace, stream, nullptr, &o);
+            } else {
+                if (q.M <= 8) st = launch_w4a16_decode<1, false, false, true>(q, packed, scales, zeros, workspace, stream, nullptr, &o);
+                else if (q.M <= 16) st = launch_w4a16_decode<2, false, false, true>(q, packed, scales, zeros, workspace, stream, nullptr, &o);
+                else st = launch_w4a16_decode<4, false, false, true>(q, packed, scales, zeros, workspace, stream, nullptr, &o);
+            }
+            if (st != QG_OK) return st;
+        }
+        return QG_OK;
+    }
     if ((st = qg_gemm_w4a16(X, xdt, M, K, N, packed, scales, zeros, group, Y, workspace, ws_bytes, stream)) != QG_OK)
         return st;
     return outlier_side_launch(X, xdt, M, K, N, group, count, idx, codes8, s8, Y, stream);

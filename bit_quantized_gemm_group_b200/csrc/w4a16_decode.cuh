@@ -60,12 +60,15 @@ struct DecodeParams {
     int M, K, N;
     int G, nslabs, units, grid;
     int narrow;                    // N % 32 != 0: packed words by 2-D boxes per 32-column block
+    int ocount;                    // outliers per group and column (the fused side path), 1..4
+    uint32_t side_tx;              // side-path bytes of one stage: GPS (2 ocount 128 + 512)
 };
 
 constexpr int kDecBN = 128;          // columns per slab
 constexpr int kDecGroupW = 8192;     // packed words of one group: 16 rows x 128 columns x 4 B
 constexpr int kDecGroupV24 = 4096;   // 2:4 kept codes of one group: 8 rows x 128 columns x 4 B
 constexpr int kDecGroupM24 = 2048;   // 2:4 position words of one group: 4 rows x 128 columns x 4 B
+constexpr int kDecOutMax = 4;        // outliers per group and column that the fused side path takes
 
 QG_DEV_INLINE int dec_first_unit(int c, int units, int grid) { return (int)((int64_t)c * units / grid); }
 
@@ -80,7 +83,7 @@ QG_DEV_INLINE int dec_cta_of_unit(int u, int units, int grid)
 
 // Shared memory of one CTA: ST stages of GPS groups, the k-warp reduction tiles and
 // the stage mbarriers.
-template <int MT, int NW, int GPS, int ST, bool PWG, bool SP = false>
+template <int MT, int NW, int GPS, int ST, bool PWG, bool SP = false, bool OUT = false>
 struct DecodeSmem {
     static constexpr int MP = 8 * MT;
     // weight bytes of one group: packed words, or (2:4) kept codes then position words
@@ -90,18 +93,26 @@ struct DecodeSmem {
     static constexpr int X_OFF = GPS * WB;
     static constexpr int S_OFF = X_OFF + GPS * XG;    // fp16 scales [GPS][128]
     static constexpr int Z_OFF = S_OFF + GPS * 256;   // u8 zeros [GPS][128]
-    static constexpr int STAGE = (Z_OFF + GPS * 128 + 1023) / 1024 * 1024;
+    // outlier side path (OUT): offsets u8 [GPS][ocount][128], codes i8 [GPS][ocount][128],
+    // scales fp32 [GPS][128]
+    static constexpr int OI_OFF = Z_OFF + GPS * 128;
+    static constexpr int OC_OFF = OI_OFF + GPS * kDecOutMax * 128;
+    static constexpr int OS_OFF = OC_OFF + GPS * kDecOutMax * 128;
+    static constexpr int END = OUT ? OS_OFF + GPS * 512 : Z_OFF + GPS * 128;
+    static constexpr int STAGE = (END + 1023) / 1024 * 1024;
     static constexpr int FRAG = 4 * MT;               // float4 accumulator fragments per lane (64 columns x MP tokens per warp)
     static constexpr int TS = kDecBN + 4;            // row stride (floats) of the [token][column] result tile
     static constexpr int RED_K = (KW - 1) * 2 * FRAG * 32 * 16;  // k-warp reduction (fragment layout)
     static constexpr int RED = RED_K > MP * TS * 4 ? RED_K : MP * TS * 4;  // the result tile aliases it
-    static constexpr int TOTAL = ST * STAGE + RED + 3 * ST * 8 + 1024;
+    static constexpr int SIDE = OUT ? 2 * MP * kDecBN * 4 : 0;  // side-path sums of a piece, 2 x [token][128] fp32
+    static constexpr int TOTAL = ST * STAGE + RED + SIDE + 3 * ST * 8 + 16 + 1024;
     // The producer is one warp after the consumers, or (PWG) a whole warpgroup of which
     // the first warp works, so that the register file can be split with setmaxnreg: the
-    // producer warps keep 56 registers a thread and the consumers take the rest.
+    // producer warps keep 56 registers a thread (136 with the side path) and the consumers
+    // take the rest.
     static constexpr int THREADS = 32 * NW + (PWG ? 128 : 32);
     static constexpr int REG_LAUNCH = (65536 / THREADS) / 8 * 8 > 255 ? 248 : (65536 / THREADS) / 8 * 8;
-    static constexpr int REG_PRODUCER = 56;
+    static constexpr int REG_PRODUCER = OUT ? 136 : 56;
     static constexpr int REG_CONSUMER_RAW = (REG_LAUNCH * THREADS - REG_PRODUCER * 128) / (32 * NW) / 8 * 8;
     static constexpr int REG_CONSUMER = REG_CONSUMER_RAW > 248 ? 248 : REG_CONSUMER_RAW;
     static constexpr uint32_t GROUP_TX = WB + XG + 384;  // TMA bytes of one group
@@ -117,6 +128,7 @@ struct DecodeMaps {
     CUtensorMap wg, w1;  // packed words, GPS groups / 1 group (4-D), or the 2-D per-block map in w1
     CUtensorMap xg, x1;  // activations, GPS groups / 1 group
     CUtensorMap mg, m1;  // 2:4 position words {32 columns, 4 rows, N/32 blocks, G groups}, GPS groups / 1 group
+    CUtensorMap oi, oc, os;  // outlier offsets / codes {N, ocount, G} and scales {N, G}, GPS groups
 };
 
 QG_DEV_INLINE void tma_load_4d(const CUtensorMap* m, uint64_t* bar, void* smem_dst, int x, int y, int z, int w)
@@ -160,12 +172,13 @@ struct DecodeSchedule {
     }
 };
 
-template <int MT, bool BF16, int NW, int GPS, int ST, bool FULL, bool PWG, int MINB, bool SP>
-__global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG, SP>::THREADS, MINB)
+template <int MT, bool BF16, int NW, int GPS, int ST, bool FULL, bool PWG, int MINB, bool SP, bool OUT>
+__global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG, SP, OUT>::THREADS, MINB)
     w4a16_decode_kernel(const DecodeParams p, const __grid_constant__ DecodeMaps maps)
 {
     using H = HalfOps<BF16>;
-    using L = DecodeSmem<MT, NW, GPS, ST, PWG, SP>;
+    using L = DecodeSmem<MT, NW, GPS, ST, PWG, SP, OUT>;
+    static_assert(!(SP && OUT), "the side path is fused into the dense kernel only");
     static_assert(!SP || FULL, "the 2:4 path dequantizes in full");
     constexpr int MP = L::MP;
     constexpr int KW = L::KW;
@@ -176,9 +189,13 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG, SP>::THREADS,
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint8_t* ring = smem;
     float4* red = reinterpret_cast<float4*>(smem + ST * L::STAGE);
-    uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * L::STAGE + L::RED);
+    float* side = reinterpret_cast<float*>(smem + ST * L::STAGE + L::RED);  // 2 x [MP][128] (OUT)
+    uint64_t* full = reinterpret_cast<uint64_t*>(smem + ST * L::STAGE + L::RED + L::SIDE);
     uint64_t* empty = full + ST;
     uint64_t* armed = empty + ST;  // the producer has set up a stage's fill (its expected bytes)
+    volatile int* side_fail = reinterpret_cast<volatile int*>(armed + ST);  // a side-path wait gave up (OUT)
+    constexpr int NSIDE = OUT ? 2 : 0;  // side-path warps: NW + 2, NW + 3
+    constexpr int SIDEBAR = 32 * (NW + NSIDE);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int G = p.G;
@@ -188,9 +205,10 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG, SP>::THREADS,
     if (threadIdx.x == 0) {
         for (int i = 0; i < ST; ++i) {
             mbar_init(&full[i], 1);
-            mbar_init(&empty[i], NW);
+            mbar_init(&empty[i], NW + NSIDE);
             mbar_init(&armed[i], 1);
         }
+        *side_fail = 0;
         fence_mbar_init();
     }
     __syncthreads();
@@ -204,7 +222,128 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG, SP>::THREADS,
         // fill up, so a CTA that starts late (after the previous grid ended) gets its first
         // stage's activations right behind that stage's weights, not behind the whole ring.
         asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(L::REG_PRODUCER));
-        if (warp > NW + 1) return;
+        if constexpr (OUT) {
+            if (warp >= NW + 2) {
+                // ---------------- outlier side path (warps NW + 2, NW + 3) ----------------
+                // Side warp sw (0, 1) takes the groups gi = sw, sw + 2, .. of every stage; its
+                // lane l takes columns 4l .. 4l + 3 (one 4-byte load gives an outlier slot of
+                // all four).  Per group: sums[m][c] += sum_r x[m][g 128 + idx_r] (code_r s8),
+                // in group then slot order, into the warp's own sums; at the piece's end both
+                // warps' sums are in shared memory and the consumers add them to the piece's
+                // tile (so Y is rounded once).  The warps walk the same schedule as the
+                // consumers and release each stage with them.
+                const int sw = warp - (NW + 2), c0 = 4 * lane;
+                const int cnt = p.ocount, M = p.M;
+                float* mine = side + sw * (MP * kDecBN);
+                // up to 8 tokens the piece's sums stay in registers; with more a group's sums
+                // are added to the warp's shared-memory sums
+                constexpr bool SREG = MP <= 8;
+                float sacc[4][SREG ? MP : 1];
+                int stage = 0;
+                uint32_t phase = 0;
+                bool sok = true, bad = false;
+                DecodeSchedule sc(u0, u1, G);
+                for (bool firstp = true; !sc.done(); sc.next_piece(), firstp = false) {
+                    if constexpr (SREG) {
+#pragma unroll
+                        for (int j = 0; j < 4; ++j)
+#pragma unroll
+                            for (int m = 0; m < MP; ++m) sacc[j][m] = 0.0f;
+                    } else {
+                        if (!firstp) named_bar_sync(3, SIDEBAR);  // the consumers took the previous piece's sums
+                        for (int m = 0; m < MP; ++m)
+                            *reinterpret_cast<float4*>(mine + m * kDecBN + c0) = make_float4(0.f, 0.f, 0.f, 0.f);
+                    }
+                    for (int g0 = sc.ga; g0 < sc.gb; g0 += GPS) {
+                        const int ng = min(GPS, sc.gb - g0);
+                        if (sok && !mbar_wait_backoff(&full[stage], phase)) sok = false;
+                        if (sok) {
+                            const uint8_t* st = ring + stage * L::STAGE;
+#pragma unroll
+                            for (int gg = 0; gg < (GPS + 1) / 2; ++gg) {
+                                const int gi = 2 * gg + sw;
+                                if (gi < ng) {
+                                    // the group's slots for the four columns: offsets, weights
+                                    const float4 s4 = *reinterpret_cast<const float4*>(st + L::OS_OFF + (gi * kDecBN + c0) * 4);
+                                    const float s8v[4] = {s4.x, s4.y, s4.z, s4.w};
+                                    uint32_t i4[kDecOutMax], q4[kDecOutMax];
+#pragma unroll
+                                    for (int r = 0; r < kDecOutMax; ++r) {
+                                        i4[r] = r < cnt ? *reinterpret_cast<const uint32_t*>(st + L::OI_OFF + (gi * cnt + r) * kDecBN + c0) : 0u;
+                                        q4[r] = r < cnt ? *reinterpret_cast<const uint32_t*>(st + L::OC_OFF + (gi * cnt + r) * kDecBN + c0) : 0u;
+                                    }
+                                    const uint8_t* xgrp = st + L::X_OFF + gi * L::XG;
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j) {
+                                        float gacc[MP];
+#pragma unroll
+                                        for (int m = 0; m < MP; ++m) gacc[m] = SREG ? sacc[j][SREG ? m : 0] : 0.0f;
+#pragma unroll
+                                        for (int r = 0; r < kDecOutMax; ++r) {
+                                            if (r < cnt) {
+                                                int k = (int)((i4[r] >> (8 * j)) & 0xFFu);
+                                                const float w = __fmul_rn((float)(int8_t)((q4[r] >> (8 * j)) & 0xFFu), s8v[j]);
+                                                if (k >= kDecBN) {  // not an offset inside the group: skipped, reported
+                                                    bad = true;
+                                                    continue;
+                                                }
+                                                const uint8_t* xk = xgrp + (k >> 6) * (MP * 128) + (k & 7) * 2;
+                                                const int ch = (k & 63) >> 3;
+                                                if (M == 1) {  // one token: row 0 of the tile, no swizzle offset
+                                                    const uint16_t xb = *reinterpret_cast<const uint16_t*>(xk + (ch << 4));
+                                                    const float xv = BF16 ? bf16_bits_to_f32(xb) : __half2float(__ushort_as_half(xb));
+                                                    gacc[0] = fmaf(xv, w, gacc[0]);
+                                                    continue;
+                                                }
+#pragma unroll
+                                                for (int mb = 0; mb < MP / 8; ++mb) {
+                                                    if (8 * mb < M) {
+#pragma unroll
+                                                        for (int mm = 0; mm < 8; ++mm) {
+                                                            const int m = 8 * mb + mm;
+                                                            if (m < M) {
+                                                                const uint16_t xb = *reinterpret_cast<const uint16_t*>(xk + m * 128 + ((ch ^ (m & 7)) << 4));
+                                                                const float xv = BF16 ? bf16_bits_to_f32(xb) : __half2float(__ushort_as_half(xb));
+                                                                gacc[m] = fmaf(xv, w, gacc[m]);
+                                                            }
+                                                        }
+                                                    }
+                                                }
+                                            }
+                                        }
+                                        if constexpr (SREG) {
+#pragma unroll
+                                            for (int m = 0; m < MP; ++m) sacc[j][SREG ? m : 0] = gacc[m];
+                                        } else {
+#pragma unroll
+                                            for (int m = 0; m < MP; ++m)
+                                                if (m < M) mine[m * kDecBN + c0 + j] += gacc[m];
+                                        }
+                                    }
+                                }
+                            }
+                        }
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&empty[stage]);
+                        if (++stage == ST) { stage = 0; phase ^= 1; }
+                    }
+                    if constexpr (SREG) {
+                        if (!firstp) named_bar_sync(3, SIDEBAR);  // the consumers took the previous piece's sums
+#pragma unroll
+                        for (int m = 0; m < MP; ++m)
+                            *reinterpret_cast<float4*>(mine + m * kDecBN + c0) = make_float4(sacc[0][SREG ? m : 0], sacc[1][SREG ? m : 0],
+                                                                                           sacc[2][SREG ? m : 0], sacc[3][SREG ? m : 0]);
+                    }
+                    if (!sok) *side_fail = 1;
+                    named_bar_arrive(2, SIDEBAR);  // this piece's side sums are complete
+                }
+                if (bad) set_status(6u);
+                named_bar_sync(3, SIDEBAR);
+                return;
+            }
+        } else {
+            if (warp > NW + 1) return;
+        }
         if (warp == NW + 1) {
             if (lane == 0) {
                 tma_prefetch_desc(&maps.xg);
@@ -234,6 +373,11 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG, SP>::THREADS,
         if (lane == 0) {
             tma_prefetch_desc(&maps.wg);
             tma_prefetch_desc(&maps.w1);
+            if constexpr (OUT) {
+                tma_prefetch_desc(&maps.oi);
+                tma_prefetch_desc(&maps.oc);
+                tma_prefetch_desc(&maps.os);
+            }
             if constexpr (SP) {
                 tma_prefetch_desc(&maps.mg);
                 tma_prefetch_desc(&maps.m1);
@@ -252,7 +396,13 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG, SP>::THREADS,
                 if (!__all_sync(0xffffffffu, mbar_wait(&empty[stage], phase ^ 1))) { ok = false; break; }
                 uint8_t* st = ring + stage * L::STAGE;
                 if (lane == 0) {
-                    mbar_arrive_expect_tx(&full[stage], (uint32_t)ng * L::GROUP_TX);
+                    mbar_arrive_expect_tx(&full[stage], (uint32_t)ng * L::GROUP_TX + (OUT ? p.side_tx : 0u));
+                    if constexpr (OUT) {
+                        // always GPS groups (groups past G read as zero; others unused)
+                        tma_load_3d(&maps.oi, &full[stage], st + L::OI_OFF, x, 0, g0);
+                        tma_load_3d(&maps.oc, &full[stage], st + L::OC_OFF, x, 0, g0);
+                        tma_load_2d(&maps.os, &full[stage], st + L::OS_OFF, x, g0);
+                    }
                     if constexpr (SP) {
                         // kept codes [group][block][8 rows][128 B], then position words
                         // [group][block][4 rows][128 B]
@@ -568,6 +718,20 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG, SP>::THREADS,
                     }
         }
         named_bar_sync(1, 32 * NW);
+        if constexpr (OUT) {
+            // the side-path warps' sums of this piece: add them to the tile (each thread the
+            // elements it takes in step 3); the side warps overwrite them for the next piece
+            // only after the arrival below
+            named_bar_sync(2, SIDEBAR);
+            if (*side_fail) ok = false;
+            for (int e = threadIdx.x; e < MP * 32; e += 32 * NW) {
+                float4* tv = reinterpret_cast<float4*>(tile + (e >> 5) * L::TS + 4 * (e & 31));
+                const float4 a = *tv, b = *reinterpret_cast<const float4*>(side + (e >> 5) * kDecBN + 4 * (e & 31)),
+                             c = *reinterpret_cast<const float4*>(side + MP * kDecBN + (e >> 5) * kDecBN + 4 * (e & 31));
+                *tv = make_float4(a.x + (b.x + c.x), a.y + (b.y + c.y), a.z + (b.z + c.z), a.w + (b.w + c.w));
+            }
+            named_bar_arrive(3, SIDEBAR);
+        }
 
         // 3. every consumer thread takes float4 elements (token, 4 columns) of the tile
         if (ok) {

@@ -275,8 +275,14 @@ qg_status qg_outlier_side_add(const void* X, qg_dtype xdt, int M, int K, int N, 
                               int count, const uint8_t* idx, const int8_t* codes8,
                               const float* s8, void* Y, qg_stream_t stream);
 
-/* The layer with the side path: qg_gemm_w4a16 on the dense INT4 part, then
- * qg_outlier_side_add.  Every argument of both is validated before either launches. */
+/* The layer with the side path: Y = X deq4 + X deq8(outliers).
+ * Fused (workspace given, at least qg_workspace_size(QG_OP_GEMM_W4A16, M, K, N) bytes;
+ *   1 <= count <= 4, group == 128, N % 16 == 0, and not bf16 with M >= 128): the decode
+ *   kernel streams each group's offsets, codes and scales beside its INT4 words and adds
+ *   the side sums (fp32, group then slot order) to the slab's fp32 sums, so Y is rounded
+ *   once to the output dtype.  An offset not below the group sets QG_ERR_RANGE (skipped).
+ * Otherwise: qg_gemm_w4a16 on the dense INT4 part, then qg_outlier_side_add (Y rounded
+ *   twice).  Every argument is validated before anything launches. */
 qg_status qg_gemm_w4a16_outlier(const void* X, qg_dtype xdt, int M, int K, int N,
                                 const uint32_t* packed, const uint16_t* scales,
                                 const uint8_t* zeros, int group, int count, const uint8_t* idx,

@@ -103,3 +103,74 @@ def test_layer_with_side_path(M, xdt):
     _status_ok()
     y0 = (bf16_to_f32 if xdt == "bf16" else f16_to_f32)(u16(Y0))
     assert np.abs(y - yref).sum() < 0.5 * np.abs(y0 - yref).sum()
+
+
+# ---------------------------------------------------------------------------
+# the side path fused into the decode kernel (workspace given, 1..4 outliers, M < 128):
+# the side sums join each slab piece's fp32 tile, so Y is rounded once
+# ---------------------------------------------------------------------------
+def _exact_side(K, N, count, seed):
+    """Exact operands: INT4 codes with power-of-two scales, and `count` distinct offsets per
+    group and column with INT8 codes |c| <= 15 and power-of-two scales 2^-2..2^0, so every
+    product and partial sum of the layer is exact in binary32."""
+    G = K // 128
+    r = synth.rng(seed, synth.S_EXACT, 7, K, N)
+    idx = np.argsort(r.random((G, 128, N)), axis=1)[:, :count, :].astype(np.uint8)
+    c8 = r.integers(-15, 16, (G, count, N)).astype(np.int8)
+    s8 = np.ldexp(1.0, r.integers(-2, 1, (G, N))).astype(np.float32)
+    return idx, c8, s8
+
+
+@pytest.mark.parametrize("M,count,N", [(1, 3, 12288), (16, 3, 12288), (5, 1, 384), (27, 4, 1024), (40, 2, 256)])
+def test_fused_side_path_exact(M, count, N):
+    q = qlib()
+    K = 4096 if N == 12288 else 1024
+    codes, scales, zeros = synth.exact_w4_asym(K, N, seed=M)
+    packed = oracle.pack_nibbles(codes)
+    idx, c8, s8 = _exact_side(K, N, count, seed=M + count)
+    X, Xb = synth.exact_activations(M, K, seed=M)
+    Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    q.qg_gemm_w4a16_outlier(x_device(Xb, torch.bfloat16), cuda(packed.view(np.int32)), cuda(scales.view(np.int16)),
+                            cuda(zeros), cuda(idx), cuda(c8), cuda(s8), Y)
+    _status_ok()
+    yref, _ = oracle.gemm_w4a16_outlier_ref(X, packed, scales, zeros, idx, c8, s8)
+    y32 = yref.astype(np.float32)
+    assert np.array_equal(y32.astype(np.float64), yref), "operands are not an exact case"
+    want = torch.from_numpy(y32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    got = u16(Y)
+    bad = got != want
+    assert not bad.any(), f"{int(bad.sum())} of {bad.size} outputs differ (M={M}, count={count}, N={N})"
+
+
+@pytest.mark.parametrize("M", [1, 16])
+@pytest.mark.parametrize("workspace", ["auto", None])
+def test_layer_decode_width(M, workspace):
+    """The decode layer's full 4096 x 12288 weight, fused (workspace) and two-step (none)."""
+    q = qlib()
+    K, N = 4096, 12288
+    W = synth.workload_weights("w4a16_decode", K, N)
+    idx, c8, s8, dense, (i_o, c_o, s_o, d_o) = _check_split(W)
+    codes, scales, zeros, packed = quant_w4_asym(d_o)
+    c_ref, sc_ref, z_ref, _ = oracle.quantize_w4_asym(d_o)
+    X, Xb = synth.activations(M, K, "bf16", seed=M)
+    Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    q.qg_gemm_w4a16_outlier(x_device(Xb, torch.bfloat16), packed, scales, zeros, idx, c8, s8, Y, workspace=workspace)
+    _status_ok()
+    yref, b = oracle.gemm_w4a16_outlier_ref(X, oracle.pack_nibbles(c_ref), sc_ref, z_ref, i_o, c_o, s_o)
+    ok = oracle.within_tolerance(bf16_to_f32(u16(Y)), yref, b)
+    assert ok.all(), f"{(~ok).sum()} outside tolerance"
+
+
+def test_fused_offset_out_of_range_is_reported():
+    """An offset past the group is skipped and reported (QG_ERR_RANGE); no read past X."""
+    q = qlib()
+    K, N, M = 1024, 256, 2
+    codes, scales, zeros = synth.exact_w4_asym(K, N, seed=1)
+    packed = oracle.pack_nibbles(codes)
+    idx, c8, s8 = _exact_side(K, N, 3, seed=1)
+    idx[2, 1, 7] = 200
+    _, Xb = synth.exact_activations(M, K, seed=1)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device="cuda")
+    q.qg_gemm_w4a16_outlier(x_device(Xb, torch.bfloat16), cuda(packed.view(np.int32)), cuda(scales.view(np.int16)),
+                            cuda(zeros), cuda(idx), cuda(c8), cuda(s8), Y)
+    assert q.qg_device_status() == q.QG_ERR_RANGE
