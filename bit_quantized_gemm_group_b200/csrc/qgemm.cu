@@ -907,6 +907,22 @@ qg_status qg_quantize_w4_group(const float* W, const float* s_smooth, int K, int
     if (misaligned(W) || misaligned(s_smooth) || misaligned(codes) || misaligned(scales) || misaligned(zeros))
         return QG_ERR_ALIGN;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if ((group == 64 || group == 128 || group == 256) && N % 4 == 0) {
+        // one pass over W with 16-byte accesses, values held in registers
+        const dim3 g4((N + 127) / 128, K / group), b4(512);
+        uint16_t* sc16 = static_cast<uint16_t*>(scales);
+        if (group == 64)
+            symmetric ? qg::quantize_w4_vec_kernel<64, true><<<g4, b4, 0, s>>>(W, s_smooth, K, N, codes, scales, nullptr)
+                      : qg::quantize_w4_vec_kernel<64, false><<<g4, b4, 0, s>>>(W, s_smooth, K, N, codes, sc16, zeros);
+        else if (group == 128)
+            symmetric ? qg::quantize_w4_vec_kernel<128, true><<<g4, b4, 0, s>>>(W, s_smooth, K, N, codes, scales, nullptr)
+                      : qg::quantize_w4_vec_kernel<128, false><<<g4, b4, 0, s>>>(W, s_smooth, K, N, codes, sc16, zeros);
+        else
+            symmetric ? qg::quantize_w4_vec_kernel<256, true><<<g4, b4, 0, s>>>(W, s_smooth, K, N, codes, scales, nullptr)
+                      : qg::quantize_w4_vec_kernel<256, false><<<g4, b4, 0, s>>>(W, s_smooth, K, N, codes, sc16, zeros);
+        QG_CUDA(cudaGetLastError());
+        return QG_OK;
+    }
     if (group == 64 || group == 128 || group == 256) {
         // one pass over W, values held in registers
         const dim3 g4((N + 127) / 128, K / group), b4(512);
@@ -1460,6 +1476,32 @@ qg_status qg_quantize_w8_channel(const float* W, const float* s, int K, int N, i
     if (!W || !Wq || !sw) return QG_ERR_NULL;
     if (K < 1 || N < 1) return QG_ERR_SHAPE;
     if (misaligned(W) || misaligned(s) || misaligned(Wq) || misaligned(sw)) return QG_ERR_ALIGN;
+    if (N % 4 == 0) {
+        // two streaming passes (absmax through sw as integer bits, then quantize), then
+        // sw = absmax / 127 in place
+        cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+        QG_CUDA(cudaMemsetAsync(sw, 0, sizeof(float) * (size_t)N, st));
+        const dim3 grid((N + 127) / 128, (K + 255) / 256);
+        unsigned int* amax = reinterpret_cast<unsigned int*>(sw);
+        qg::w8_absmax_kernel<<<grid, 256, 0, st>>>(W, s, K, N, amax);
+        QG_CUDA(cudaGetLastError());
+        qg::w8_quant_kernel<<<grid, 256, 0, st>>>(W, s, K, N, amax, Wq);
+        QG_CUDA(cudaGetLastError());
+        qg::w8_scale_kernel<<<(N + 255) / 256, 256, 0, st>>>(sw, N);
+        QG_CUDA(cudaGetLastError());
+        return QG_OK;
+    }
+    if (N % 32 == 0 && K <= 8192) {
+        // one pass over W: 32-column strips, K split over a cluster of up to 8 CTAs
+        if (K <= 4096) {
+            const int C = (K + 511) / 512;
+            return launch_cluster(qg::quantize_w8_strip32_kernel<8>, dim3(N / 32, C), dim3(512), 0, C, stream, W, s, K,
+                                  N, Wq, sw);
+        }
+        const int C = (K + 1023) / 1024;
+        return launch_cluster(qg::quantize_w8_strip32_kernel<16>, dim3(N / 32, C), dim3(512), 0, C, stream, W, s, K, N,
+                              Wq, sw);
+    }
     if (N % 8 == 0 && K <= 8 * qg::kW8StripRows) {
         // one pass over W: 8-column strips, K split over a cluster of up to 8 CTAs
         const int C = (K + qg::kW8StripRows - 1) / qg::kW8StripRows;

@@ -163,6 +163,136 @@ __global__ void __launch_bounds__(512) quantize_w4_regs_kernel(const float* __re
     }
 }
 
+// ---------------------------------------------------------------------------
+// The same, with 16-byte accesses (N % 4 == 0): a CTA covers 128 columns of one group
+// with 512 threads; thread (q, r) takes columns 4q .. 4q + 3 and rows r, r + 16, ..
+// of the group, so a warp reads and writes whole 512-byte / 128-byte row segments.
+// The 16 row slices' ranges meet in shared memory; one thread per column derives the
+// scale and zero point (the binary32 operations of the per-column kernels) and every
+// thread quantizes its values from registers.
+// ---------------------------------------------------------------------------
+template <int GROUP, bool SYM>
+__global__ void __launch_bounds__(512, GROUP <= 128 ? 2 : 1) quantize_w4_vec_kernel(const float* __restrict__ W,
+                                                              const float* __restrict__ s_smooth, int K, int N,
+                                                              uint8_t* __restrict__ codes, void* __restrict__ scales,
+                                                              uint8_t* __restrict__ zeros)
+{
+    constexpr int RPT = GROUP / 16;  // rows per thread
+    __shared__ float qmn[16][128], qmx[16][128];
+    __shared__ int qbad[16][128];
+    __shared__ float fs[128];
+    __shared__ int fz[128], fok[128];
+    const int cq = threadIdx.x & 31, rr = threadIdx.x >> 5;
+    const int n0 = blockIdx.x * 128 + 4 * cq;
+    const int g = blockIdx.y;
+    const bool quad_ok = n0 < N;  // N % 4 == 0: a quad is wholly inside or outside
+    float v[RPT][4];
+    float mn[4] = {0.f, 0.f, 0.f, 0.f}, mx[4] = {0.f, 0.f, 0.f, 0.f};  // asym: the range holds 0
+    bool bad[4] = {false, false, false, false};
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const int64_t k = (int64_t)g * GROUP + rr + 16 * i;
+        float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (quad_ok) w = __ldg(reinterpret_cast<const float4*>(W + k * N + n0));
+        if (s_smooth) {
+            const float sk = __ldg(s_smooth + k);
+            w = make_float4(__fmul_rn(w.x, sk), __fmul_rn(w.y, sk), __fmul_rn(w.z, sk), __fmul_rn(w.w, sk));
+        }
+        v[i][0] = w.x; v[i][1] = w.y; v[i][2] = w.z; v[i][3] = w.w;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            bad[c] |= !isfinite(v[i][c]);
+            if (SYM) {
+                mx[c] = fmaxf(mx[c], fabsf(v[i][c]));
+            } else {
+                if (v[i][c] < mn[c]) mn[c] = v[i][c];
+                if (v[i][c] > mx[c]) mx[c] = v[i][c];
+            }
+        }
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        qmn[rr][4 * cq + c] = mn[c];
+        qmx[rr][4 * cq + c] = mx[c];
+        qbad[rr][4 * cq + c] = bad[c];
+    }
+    __syncthreads();
+    if (threadIdx.x < 128) {
+        const int cl = threadIdx.x, n = blockIdx.x * 128 + cl;
+        float a = 0.0f, b = 0.0f;
+        bool gb = false;
+        for (int r = 0; r < 16; ++r) {
+            gb |= qbad[r][cl] != 0;
+            if (qmn[r][cl] < a) a = qmn[r][cl];
+            if (qmx[r][cl] > b) b = qmx[r][cl];
+        }
+        int ok = n < N && !gb;
+        float sv = 0.0f;
+        int zv = 0;
+        if (n < N && gb) set_status(5u);
+        if (ok) {
+            if (SYM) {
+                sv = __fdiv_rn(b, 7.0f);
+                static_cast<float*>(scales)[(int64_t)g * N + n] = sv;
+            } else {
+                const float r = __fsub_rn(b, a);
+                const float s32 = __fdiv_rn(r, 15.0f);
+                if (s32 > 65504.0f) {
+                    set_status(6u);
+                    ok = 0;
+                } else {
+                    __half s16 = __float2half_ru(s32);
+                    sv = __half2float(s16);
+                    if (r == 0.0f) {
+                        s16 = __ushort_as_half((unsigned short)0);
+                        sv = 0.0f;
+                    } else {
+                        zv = min(max(__float2int_rn(__fdiv_rn(-a, sv)), 0), 15);
+                    }
+                    static_cast<uint16_t*>(scales)[(int64_t)g * N + n] = __half_as_ushort(s16);
+                    zeros[(int64_t)g * N + n] = (uint8_t)zv;
+                }
+            }
+        }
+        fs[cl] = sv;
+        fz[cl] = zv;
+        fok[cl] = ok;
+    }
+    __syncthreads();
+    if (!quad_ok) return;
+    float sc[4];
+    int zc[4], okc[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        sc[c] = fs[4 * cq + c];
+        zc[c] = fz[4 * cq + c];
+        okc[c] = fok[4 * cq + c];
+    }
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const int64_t k = (int64_t)g * GROUP + rr + 16 * i;
+        uint32_t word = 0;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+            int q = 0;
+            if (sc[c] != 0.0f) {
+                if (SYM) q = min(max(__float2int_rn(__fdiv_rn(v[i][c], sc[c])), -7), 7);
+                else q = min(max(__float2int_rn(__fdiv_rn(v[i][c], sc[c])) + zc[c], 0), 15);  // round(x/s) + z
+            }
+            word |= (uint32_t)(q & 0xFF) << (8 * c);
+        }
+        // a column whose group was not finite or overflowed keeps whatever its codes held
+        uint8_t* dst = codes + k * N + n0;
+        if (okc[0] && okc[1] && okc[2] && okc[3]) {
+            *reinterpret_cast<uint32_t*>(dst) = word;
+        } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c)
+                if (okc[c]) dst[c] = (uint8_t)(word >> (8 * c));
+        }
+    }
+}
+
 // Symmetric INT4: s = max|w|/7 (fp32), codes in [-7, 7] ("AI Infra guide, ch.4"
 // sec. 1.2 symmetric scale, 4-bit analogue).
 __global__ void __launch_bounds__(256) quantize_w4_sym_kernel(const float* __restrict__ W,
@@ -299,6 +429,180 @@ __global__ void smooth_finalize_kernel(float* __restrict__ s_io /*in: ax*/, floa
 // shuffles, then across the cluster through distributed shared memory; each CTA then
 // quantizes the values it holds.  For N % 8 == 0 and K <= 16384.
 // ---------------------------------------------------------------------------
+// Wider strips for the same computation (N % 32 == 0): a strip of 32 columns, K split
+// over a cluster of C CTAs of 512 threads; thread (q, r) takes columns 4q .. 4q + 3
+// and rows r, r + 64, .. of its CTA's range (RPT of them), so a warp reads 4 rows x
+// 128 bytes per load and writes 4 rows x 32 bytes per store.  The column absmax meets
+// in shared memory, then across the cluster through distributed shared memory.
+template <int RPT>
+__global__ void __launch_bounds__(512) quantize_w8_strip32_kernel(const float* __restrict__ W,
+                                                                  const float* __restrict__ s, int K, int N,
+                                                                  int8_t* __restrict__ Wq, float* __restrict__ sw)
+{
+    __shared__ float wmax[16][32];
+    __shared__ __align__(16) float cmax[32];
+    __shared__ float csc[32];
+    const int n0 = 32 * blockIdx.x;
+    const uint32_t rank = cluster_ctarank();
+    const int C = (int)gridDim.y;  // the whole y extent is one cluster
+    const int kb = (int)((int64_t)K * rank / C), ke = (int)((int64_t)K * (rank + 1) / C);
+    const int cq = threadIdx.x & 7, rr = threadIdx.x >> 3;
+    float v[RPT][4];
+    float a[4] = {0.f, 0.f, 0.f, 0.f};
+    bool bad = false;
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const int k = kb + rr + 64 * i;
+        if (k < ke) {
+            float4 w = __ldg(reinterpret_cast<const float4*>(W + (int64_t)k * N + n0 + 4 * cq));
+            if (s) {
+                const float sk = __ldg(s + k);
+                w = make_float4(__fmul_rn(w.x, sk), __fmul_rn(w.y, sk), __fmul_rn(w.z, sk), __fmul_rn(w.w, sk));
+            }
+            v[i][0] = w.x; v[i][1] = w.y; v[i][2] = w.z; v[i][3] = w.w;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                bad |= !isfinite(v[i][c]);
+                a[c] = fmaxf(a[c], fabsf(v[i][c]));
+            }
+        } else {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) v[i][c] = 0.0f;
+        }
+    }
+    if (bad) set_status(5u);
+    // lanes with the same column quad: lane bits 3 and 4
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        a[c] = fmaxf(a[c], __shfl_xor_sync(0xffffffffu, a[c], 8));
+        a[c] = fmaxf(a[c], __shfl_xor_sync(0xffffffffu, a[c], 16));
+    }
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    if (lane < 8)
+#pragma unroll
+        for (int c = 0; c < 4; ++c) wmax[warp][4 * lane + c] = a[c];
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        float m = 0.0f;
+        for (int w = 0; w < 16; ++w) m = fmaxf(m, wmax[w][threadIdx.x]);
+        cmax[threadIdx.x] = m;
+    }
+    cluster_sync();
+    if (threadIdx.x < 32) {
+        float m = 0.0f;
+        const uint32_t la = smem_u32(&cmax[threadIdx.x]);
+        for (int r = 0; r < C; ++r) m = fmaxf(m, ld_dsmem_f32(dsmem_addr(la, (uint32_t)r)));
+        const float sc = __fdiv_rn(m, 127.0f);  // the column scale
+        csc[threadIdx.x] = sc;
+        if (rank == 0) sw[n0 + threadIdx.x] = sc;
+    }
+    cluster_sync();  // every CTA has read every cmax before any CTA moves on (and csc is set)
+    float sc[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) sc[c] = csc[4 * cq + c];
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const int k = kb + rr + 64 * i;
+        if (k < ke) {
+            uint32_t word = 0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                int q = 0;
+                if (sc[c] != 0.0f && isfinite(v[i][c])) q = min(max(__float2int_rn(__fdiv_rn(v[i][c], sc[c])), -127), 127);
+                word |= (uint32_t)(q & 0xFF) << (8 * c);
+            }
+            *reinterpret_cast<uint32_t*>(Wq + (int64_t)k * N + n0 + 4 * cq) = word;
+        }
+    }
+}
+
+// Per-output-channel INT8 in two streaming passes (N % 4 == 0): pass 1 takes the column
+// absmax of W~ = diag(s) W (|w| as integer bits, combined with atomicMax: the maximum of
+// non-negative floats, exact in any order; non-finite values are reported and left
+// out), pass 2 quantizes with sw = absmax / 127, and a last pass turns the absmax into
+// sw in place.  Every pass is a CTA of 256 threads over 128 columns x 256 rows with
+// 16-byte loads (a warp reads one 512-byte row segment) and 4-byte stores: W is read
+// twice, but at the copy rate, which beats one pass that must meet across K.
+__global__ void __launch_bounds__(256) w8_absmax_kernel(const float* __restrict__ W, const float* __restrict__ s,
+                                                        int K, int N, unsigned int* __restrict__ amax_bits)
+{
+    __shared__ unsigned int part[8][128];
+    const int cq = threadIdx.x & 31, rr = threadIdx.x >> 5;
+    const int n0 = blockIdx.x * 128 + 4 * cq;
+    const int k0 = blockIdx.y * 256;
+    unsigned int a[4] = {0u, 0u, 0u, 0u};
+    bool bad = false;
+    if (n0 < N) {
+#pragma unroll 8
+        for (int i = 0; i < 32; ++i) {
+            const int k = k0 + rr + 8 * i;
+            if (k < K) {
+                float4 w = __ldg(reinterpret_cast<const float4*>(W + (int64_t)k * N + n0));
+                if (s) {
+                    const float sk = __ldg(s + k);
+                    w = make_float4(__fmul_rn(w.x, sk), __fmul_rn(w.y, sk), __fmul_rn(w.z, sk), __fmul_rn(w.w, sk));
+                }
+                const float v[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    if (isfinite(v[c])) a[c] = max(a[c], __float_as_uint(fabsf(v[c])));
+                    else bad = true;
+                }
+            }
+        }
+    }
+    if (bad) set_status(5u);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) part[rr][4 * cq + c] = a[c];
+    __syncthreads();
+    if (threadIdx.x < 128) {
+        const int n = blockIdx.x * 128 + threadIdx.x;
+        unsigned int m = 0u;
+#pragma unroll
+        for (int r = 0; r < 8; ++r) m = max(m, part[r][threadIdx.x]);
+        if (n < N && m != 0u) atomicMax(amax_bits + n, m);
+    }
+}
+
+__global__ void __launch_bounds__(256) w8_quant_kernel(const float* __restrict__ W, const float* __restrict__ s, int K,
+                                                       int N, const unsigned int* __restrict__ amax_bits,
+                                                       int8_t* __restrict__ Wq)
+{
+    const int cq = threadIdx.x & 31, rr = threadIdx.x >> 5;
+    const int n0 = blockIdx.x * 128 + 4 * cq;
+    const int k0 = blockIdx.y * 256;
+    if (n0 >= N) return;
+    const uint4 ab = *reinterpret_cast<const uint4*>(amax_bits + n0);
+    const float sc[4] = {__fdiv_rn(__uint_as_float(ab.x), 127.0f), __fdiv_rn(__uint_as_float(ab.y), 127.0f),
+                         __fdiv_rn(__uint_as_float(ab.z), 127.0f), __fdiv_rn(__uint_as_float(ab.w), 127.0f)};
+#pragma unroll 8
+    for (int i = 0; i < 32; ++i) {
+        const int k = k0 + rr + 8 * i;
+        if (k < K) {
+            float4 w = __ldg(reinterpret_cast<const float4*>(W + (int64_t)k * N + n0));
+            if (s) {
+                const float sk = __ldg(s + k);
+                w = make_float4(__fmul_rn(w.x, sk), __fmul_rn(w.y, sk), __fmul_rn(w.z, sk), __fmul_rn(w.w, sk));
+            }
+            const float v[4] = {w.x, w.y, w.z, w.w};
+            uint32_t word = 0;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                int q = 0;
+                if (sc[c] != 0.0f && isfinite(v[c])) q = min(max(__float2int_rn(__fdiv_rn(v[c], sc[c])), -127), 127);
+                word |= (uint32_t)(q & 0xFF) << (8 * c);
+            }
+            *reinterpret_cast<uint32_t*>(Wq + (int64_t)k * N + n0) = word;
+        }
+    }
+}
+
+__global__ void __launch_bounds__(256) w8_scale_kernel(float* __restrict__ sw, int N)
+{
+    const int n = blockIdx.x * blockDim.x + threadIdx.x;
+    if (n < N) sw[n] = __fdiv_rn(__uint_as_float(__float_as_uint(sw[n])), 127.0f);
+}
+
 constexpr int kW8StripThreads = 512;
 constexpr int kW8StripRowsPerThread = 4;
 constexpr int kW8StripRows = kW8StripThreads * kW8StripRowsPerThread;  // rows of K per CTA

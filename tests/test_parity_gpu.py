@@ -49,8 +49,10 @@ def _status_ok():
 # ---------------------------------------------------------------------------
 # quantizers (bit-exact)
 # ---------------------------------------------------------------------------
+# N % 4 == 0 takes the 16-byte kernel (a ragged last CTA at N = 136, 8); N = 30 the
+# column-per-thread register kernel
 W4_SHAPES = [(1024, 1024, "w4a16_tiny"), (4096, 12288, "w4a16_decode"), (11008, 4096, "w4a16_decode"),
-             (384, 136, "w4a16_decode"), (128, 8, "w4a16_decode")]
+             (384, 136, "w4a16_decode"), (128, 8, "w4a16_decode"), (256, 30, "w4a16_decode")]
 
 
 @pytest.mark.parametrize("K,N,cfg", W4_SHAPES)
@@ -93,11 +95,13 @@ def test_smooth_scales_and_w8_channel_bitexact():
 
 
 @pytest.mark.parametrize("K,N,smooth", [(11008, 4096, True), (16384, 64, False), (2048, 24, True), (100, 136, True),
-                                         (4096, 100, True), (20000, 8, False)])
+                                         (4096, 100, True), (20000, 8, False), (6000, 96, True), (700, 64, False),
+                                         (8192, 32, True), (4096, 11008, False)])
 def test_quantize_w8_channel_shapes_bitexact(K, N, smooth):
-    """Both paths of the INT8 channel quantizer: the one-pass strip kernel (N % 8 == 0,
-    K <= 16384: clusters of 1..8 CTAs along K, ragged last CTA) and the general kernel
-    (N % 8 != 0 or longer K); a zero column and smoothing on and off."""
+    """Every path of the INT8 channel quantizer: the 32-column strip kernel (N % 32 == 0,
+    K <= 8192: clusters of 1..8 CTAs along K with 8 or 16 rows a thread, ragged last CTA),
+    the 8-column strip kernel (N % 8 == 0, K <= 16384) and the general kernel (other
+    shapes); a zero column and smoothing on and off."""
     W = synth.weights(K, N, 0.02, 0.01, 8.0, seed=K + N)
     W[:, 3] = 0.0
     s_o = None
