@@ -48,11 +48,11 @@ CONFIG = {"workload": "w4a16_decode: M in {1,4,16,32} x (K,N) in {(4096,12288),(
                 "finds its weights in L2",
           "launch": "one CUDA graph per step (16 calls, one decode kernel launch each)"}
 # DRAM bytes (read + write) of one decode launch over its algorithmic bytes, from an ncu
-# capture of one w4a16_decode_kernel launch at K=4096, N=22016, M=1 (47.237 MB read +
-# 0.016 MB written against 47.255 MB algorithmic; the weight stream is read exactly once,
-# so traffic scales with the algorithmic bytes of each call).  Take it again whenever the
+# capture of one w4a16_decode_kernel launch at K=4096, N=12288, M=1 (26.403 MB read, no
+# write counted, against 26.378 MB algorithmic; the weight stream is read exactly once, so
+# traffic scales with the algorithmic bytes of each call).  Take it again whenever the
 # decode kernel changes.
-DECODE_TRAFFIC_RATIO = (47.236608e6 + 15.616e3) / (4096 * 22016 // 2 + 4096 // 128 * 22016 * 3 + 2 * 4096 + 2 * 22016)
+DECODE_TRAFFIC_RATIO = 26.403328e6 / (4096 * 12288 // 2 + 4096 // 128 * 12288 * 3 + 2 * 4096 + 2 * 12288)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 

@@ -35,6 +35,11 @@ QG_DEV_INLINE unsigned long long globaltimer_ns()
 // ---------------------------------------------------------------------------
 // 16-bit float bit helpers
 // ---------------------------------------------------------------------------
+// Exact int32 -> fp32 for |v| < 2^22 on the full-rate pipes (integer add, fp32 add):
+// add into the mantissa of 1.5 * 2^23, subtract it back.  (The conversion instruction
+// itself issues at a fraction of the fp32 rate.)
+QG_DEV_INLINE float i2f_small(uint32_t v) { return __uint_as_float(v + 0x4B400000u) - 12582912.0f; }
+
 QG_DEV_INLINE float bf16_bits_to_f32(uint32_t b) { return __uint_as_float(b << 16); }
 
 QG_DEV_INLINE uint32_t pack_bf16x2_rn(float lo, float hi)
@@ -169,6 +174,43 @@ QG_DEV_INLINE bool mbar_wait_backoff(uint64_t* bar, uint32_t parity)
             return false;
         }
     }
+}
+
+QG_DEV_INLINE unsigned long long ld_acquire_u64(const unsigned long long* p)
+{
+    unsigned long long v;
+    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+    return v;
+}
+
+QG_DEV_INLINE void st_release_u64(unsigned long long* p, unsigned long long v)
+{
+    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+// Split-slab pieces between the CTAs of one decode launch: a CTA publishes its piece's
+// partial tile under the launch's 64-bit token (never 0); the CTA that finishes the slab
+// watches the tokens of CTAs c_first .. c_last with the lanes of one warp (all polls in
+// flight at once), bounded: false (and QG_ERR_TIMEOUT recorded) if one never appears.
+QG_DEV_INLINE bool watch_tokens(const unsigned long long* flags, int c_first, int c_last, unsigned long long token,
+                                int lane)
+{
+    const unsigned long long t0 = globaltimer_ns();
+    const unsigned long long lim = g_wait_limit_ns;
+    for (int i0 = c_first; i0 <= c_last; i0 += 32) {
+        const int c = i0 + lane;
+        bool seen = c > c_last;  // lanes past the last piece have nothing to watch
+        for (uint32_t it = 0;; ++it) {
+            if (!seen) seen = ld_acquire_u64(flags + c) == token;
+            if (__all_sync(0xffffffffu, seen)) break;
+            __nanosleep(32);
+            if ((it & 15u) == 15u && globaltimer_ns() - t0 > lim) {
+                if (lane == 0) set_status(7u);
+                return false;
+            }
+        }
+    }
+    return true;
 }
 
 // Named barrier `id` over `count` threads that also ANDs a predicate across them.

@@ -15,10 +15,11 @@
 //
 // Work split (stream-K), as in the W4A16 decode kernel: units are (128-column slab,
 // 128-k block); the persistent grid divides them into equal contiguous ranges; a piece
-// that covers a whole slab finishes Y itself, a partial piece writes its int32 tile to
-// the workspace (slot 0: the CTA's first piece, 1: its last) and
-// `w8a8_decode_fixup_kernel` adds the pieces of every split slab (integer sums, exact in
-// any order) and finishes Y.
+// that covers a whole slab finishes Y itself.  Of a split slab, the piece holding the
+// slab's first unit (always its CTA's last piece) finishes it: it waits (bounded) for the
+// 64-bit tokens under which the slab's other pieces (always their CTAs' first pieces)
+// published their int32 tiles in the workspace, adds them (integer sums, exact in any
+// order) and writes Y.  One launch per call.
 //
 // Roles (256 threads): warp 0 issues TMA; warps 1-2 issue the MMAs, warp 1 + e taking
 // the CTA's units i = e (mod 2) (a thread's tcgen05.mma instructions are accepted one
@@ -37,7 +38,9 @@ struct I8DecodeParams {
     const float* sw;    // fp32 [N]
     uint16_t* Y;        // bf16 [M][N]
     int32_t* dbg;       // NULL or int32 [M][N]: receives acc
-    int32_t* partials;  // [grid][2][NT][128]
+    int32_t* partials;  // [grid][NT][128]: the CTA's published piece
+    unsigned long long* flags;  // [grid] publication tokens
+    unsigned long long token;   // this launch's token (never 0)
     int M, K, N;
     int KB, nslabs, units, grid;  // KB = K / 128 units per slab
 };
@@ -209,45 +212,75 @@ __global__ void __launch_bounds__(I8DecCfg<NT>::THREADS, 1)
         const int q = warp & 3, col = 32 * q + lane;
         const int M = p.M;
         int i = 0, pc = 0;
-        bool first_piece = true;
+        bool ok = true;  // after a wait gives up, the schedule is still walked (named barriers) without work
         while (i < n_it) {
             const int slab = (u0 + i) / KB;
             const int ie = min(n_it, (slab + 1) * KB - u0);
             const int pb = pc & 1;
-            bool ok = true;
             for (int e = 0; e < C::NI; ++e)
-                if (!mbar_wait_backoff(&dfull[e * DP + pb], (pc >> 1) & 1)) ok = false;
-            if (!ok) break;
-            tc_fence_after();
+                if (ok && !mbar_wait_backoff(&dfull[e * DP + pb], (pc >> 1) & 1)) ok = false;
             // issuer e holds units of this piece iff some it in [i, ie) has it % 2 == e
             const bool has1 = ie - i >= 2 || ((i & 1) == 1);
             const bool has0 = ie - i >= 2 || ((i & 1) == 0);
             const int n0 = slab * 128, n = n0 + col;
-            const bool whole = (u0 + i) % KB == 0 && (u0 + ie) % KB == 0 && ie - i == KB;
-            const float swn = (whole && n < p.N) ? __ldg(p.sw + n) : 0.0f;
-            int32_t* mine = p.partials + ((size_t)blockIdx.x * 2 + (first_piece ? 0 : 1)) * NT * 128 + col;
+            const bool whole = (u0 + i) % KB == 0 && ie - i == KB;
+            const bool head = (u0 + i) % KB == 0 && !whole;  // finishes a split slab (the CTA's last piece)
+            int cl = 0;
+            if (head) {
+                // the slab's other pieces: CTAs blockIdx.x + 1 .. cl
+                cl = i8_cta_of_unit(slab * KB + KB - 1, p.units, p.grid);
+                bool ready = true;
+                if (warp == 4 && ok) ready = watch_tokens(p.flags, (int)blockIdx.x + 1, cl, p.token, lane);
+                if (!named_bar_and(1, 128, ok && ready)) ok = false;
+            }
+            if (ok) {
+                tc_fence_after();
+                const float swn = ((whole || head) && n < p.N) ? __ldg(p.sw + n) : 0.0f;
+                int32_t* mine = p.partials + (size_t)blockIdx.x * NT * 128 + col;
 #pragma unroll 1
-            for (int t0 = 0; t0 < NT && t0 < M; t0 += 16) {
-                uint32_t a[16], b[16];
-                const uint32_t lanes = (uint32_t)(32 * q) << 16;
-                if (has0) tmem_ld_32x32b_x16(tmem + lanes + (0 * DP + pb) * NT + t0, a);
-                if (has1) tmem_ld_32x32b_x16(tmem + lanes + (1 * DP + pb) * NT + t0, b);
-                tmem_ld_wait();
+                for (int t0 = 0; t0 < NT && t0 < M; t0 += 16) {
+                    uint32_t a[16], b[16];
+                    const uint32_t lanes = (uint32_t)(32 * q) << 16;
+                    if (has0) tmem_ld_32x32b_x16(tmem + lanes + (0 * DP + pb) * NT + t0, a);
+                    if (has1) tmem_ld_32x32b_x16(tmem + lanes + (1 * DP + pb) * NT + t0, b);
+                    tmem_ld_wait();
+                    int32_t v[16];
 #pragma unroll
-                for (int t = 0; t < 16; ++t) {
-                    const int32_t v = (has0 ? (int32_t)a[t] : 0) + (has1 ? (int32_t)b[t] : 0);
-                    if (t0 + t < M) {
-                        if (whole) {
-                            if (n < p.N) i8_finish(p, t0 + t, n, v, swn);
-                        } else {
-                            mine[(t0 + t) * 128] = v;
+                    for (int t = 0; t < 16; ++t) v[t] = (has0 ? (int32_t)a[t] : 0) + (has1 ? (int32_t)b[t] : 0);
+                    if (head) {
+                        // the other pieces' rows t0 .. t0+15 (inside the NT-row slot even past
+                        // M), sixteen loads in flight per piece
+                        for (int c = (int)blockIdx.x + 1; c <= cl; ++c) {
+                            const int32_t* o = p.partials + (size_t)c * NT * 128 + t0 * 128 + col;
+                            int32_t w[16];
+#pragma unroll
+                            for (int t = 0; t < 16; ++t) w[t] = __ldcg(o + t * 128);
+#pragma unroll
+                            for (int t = 0; t < 16; ++t) v[t] += w[t];
+                        }
+                    }
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) {
+                        if (t0 + t < M) {
+                            if (whole || head) {
+                                if (n < p.N) i8_finish(p, t0 + t, n, v[t], swn);
+                            } else {
+                                __stcg(mine + (t0 + t) * 128, v[t]);
+                            }
                         }
                     }
                 }
+                tc_fence_before();
+                for (int e = 0; e < C::NI; ++e) mbar_arrive(&dempty[e * DP + pb]);
             }
-            tc_fence_before();
-            for (int e = 0; e < C::NI; ++e) mbar_arrive(&dempty[e * DP + pb]);
-            first_piece = false;
+            if (!whole && !head) {
+                // publish: every epilogue thread's stores, then one fence and the token
+                named_bar_sync(1, 128);
+                if (ok && threadIdx.x == 128) {
+                    __threadfence();
+                    st_release_u64(p.flags + blockIdx.x, p.token);
+                }
+            }
             i = ie;
             ++pc;
         }
@@ -259,57 +292,6 @@ __global__ void __launch_bounds__(I8DecCfg<NT>::THREADS, 1)
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
-    }
-}
-
-// Adds the int32 pieces of every slab the decode grid split between CTAs and finishes
-// Y; slabs held by one CTA were finished by the decode kernel.  One CTA per slab; a
-// thread step covers 4 adjacent columns of one token, with the pieces' 16-byte loads
-// issued four at a time (integer sums: the order does not matter).
-__global__ void __launch_bounds__(256) w8a8_decode_fixup_kernel(const I8DecodeParams p, int NT)
-{
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const int slab = blockIdx.x;
-    const int KB = p.KB;
-    const int cf = i8_cta_of_unit(slab * KB, p.units, p.grid);
-    const int cl = i8_cta_of_unit(slab * KB + KB - 1, p.units, p.grid);
-    if (cf == cl) return;
-    __shared__ int off[160];
-    for (int c = cf + threadIdx.x; c <= cl; c += blockDim.x) {
-        const int sl = i8_first_unit(c, p.units, p.grid) >= slab * KB ? 0 : 1;  // first piece of CTA c?
-        off[c - cf] = (c * 2 + sl) * NT * 128;
-    }
-    __syncthreads();
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int np = cl - cf + 1;
-    const int mrows = min(p.M, NT);
-    for (int e = threadIdx.x; e < mrows * 32; e += blockDim.x) {
-        const int t = e >> 5, c4 = 4 * (e & 31), n = slab * 128 + c4;
-        if (n >= p.N) continue;  // N % 16 == 0: the 4 columns are all in range or all out
-        const int o = t * 128 + c4;
-        int4 v = make_int4(0, 0, 0, 0);
-        int i = 0;
-        for (; i + 4 <= np; i += 4) {
-            int4 a[4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) a[r] = __ldcg(reinterpret_cast<const int4*>(p.partials + off[i + r] + o));
-#pragma unroll
-            for (int r = 0; r < 4; ++r) { v.x += a[r].x; v.y += a[r].y; v.z += a[r].z; v.w += a[r].w; }
-        }
-        for (; i < np; ++i) {
-            const int4 a = __ldcg(reinterpret_cast<const int4*>(p.partials + off[i] + o));
-            v.x += a.x; v.y += a.y; v.z += a.z; v.w += a.w;
-        }
-        const float tm = __ldg(p.t + t);
-        const float4 s4 = __ldg(reinterpret_cast<const float4*>(p.sw + n));
-        const int32_t acc[4] = {v.x, v.y, v.z, v.w};
-        const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-        uint16_t y[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) y[r] = f32_to_bf16_bits(__fmul_rn(__fmul_rn(__int2float_rn(acc[r]), tm), sv[r]));
-        *reinterpret_cast<uint2*>(p.Y + (int64_t)t * p.N + n) =
-            make_uint2((uint32_t)y[0] | ((uint32_t)y[1] << 16), (uint32_t)y[2] | ((uint32_t)y[3] << 16));
-        if (p.dbg) *reinterpret_cast<int4*>(p.dbg + (int64_t)t * p.N + n) = v;
     }
 }
 

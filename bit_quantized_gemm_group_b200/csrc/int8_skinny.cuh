@@ -282,10 +282,10 @@ __global__ void __launch_bounds__(WN* WK * 32, 1) w4a8_skinny_kernel(const Int8S
 #pragma unroll
                 for (int j = 0; j < MT; ++j) {
                     const float s_r0 = scv[2 * cp], s_r1 = scv[2 * cp + 1];
-                    accf[h][cp][j][0] = fmaf(__int2float_rn(P[h][cp][j][0]), s_r0, accf[h][cp][j][0]);
-                    accf[h][cp][j][1] = fmaf(__int2float_rn(P[h][cp][j][1]), s_r0, accf[h][cp][j][1]);
-                    accf[h][cp][j][2] = fmaf(__int2float_rn(P[h][cp][j][2]), s_r1, accf[h][cp][j][2]);
-                    accf[h][cp][j][3] = fmaf(__int2float_rn(P[h][cp][j][3]), s_r1, accf[h][cp][j][3]);
+                    accf[h][cp][j][0] = fmaf(i2f_small((uint32_t)P[h][cp][j][0]), s_r0, accf[h][cp][j][0]);
+                    accf[h][cp][j][1] = fmaf(i2f_small((uint32_t)P[h][cp][j][1]), s_r0, accf[h][cp][j][1]);
+                    accf[h][cp][j][2] = fmaf(i2f_small((uint32_t)P[h][cp][j][2]), s_r1, accf[h][cp][j][2]);
+                    accf[h][cp][j][3] = fmaf(i2f_small((uint32_t)P[h][cp][j][3]), s_r1, accf[h][cp][j][3]);
                     if (p.dbg && nval[h]) {
                         const int n_r0 = ncol[h] + 2 * cp, tk = 8 * j + 2 * t4;
 #pragma unroll

@@ -615,7 +615,8 @@ qg_status tc_w4a16(const qg::TcW4A16Args& a, qg_stream_t stream)
 // ---------------------------------------------------------------------------
 struct I8Plan {
     int NT, KB, nslabs, units, grid;
-    size_t partial_bytes;
+    size_t flags_bytes;    // [grid] u64 publication tokens, padded to 256 B
+    size_t partial_bytes;  // flags + [grid] published pieces of NT x 128 (4-byte elements)
 };
 
 I8Plan i8_plan(int M, int K, int N)
@@ -626,7 +627,8 @@ I8Plan i8_plan(int M, int K, int N)
     d.nslabs = (N + 127) / 128;
     d.units = d.KB * d.nslabs;
     d.grid = std::min(std::min(num_sms(), d.units), 160);
-    d.partial_bytes = (size_t)d.grid * 2 * 128 * d.NT * sizeof(int32_t);
+    d.flags_bytes = ((size_t)d.grid * 8 + 255) / 256 * 256;
+    d.partial_bytes = d.flags_bytes + (size_t)d.grid * 128 * d.NT * sizeof(int32_t);
     return d;
 }
 
@@ -646,9 +648,21 @@ qg_status launch_w8a8_decode(const int8_t* Xq, const float* t, int M, int K, con
     if ((st = make_tmap_2d(&tw, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Wq, N, K, 128, 128, CU_TENSOR_MAP_SWIZZLE_128B)) ||
         (st = make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Xq, K, M, 128, NT, CU_TENSOR_MAP_SWIZZLE_128B)))
         return st;
-    qg::I8DecodeParams p{t, sw, Y, acc_dbg, static_cast<int32_t*>(ws), M, K, N, d.KB, d.nslabs, d.units, d.grid};
-    if ((st = launch_pdl(kern, dim3(d.grid), dim3(C::THREADS), C::TOTAL, stream, p, tw, tx)) != QG_OK) return st;
-    return launch_pdl(qg::w8a8_decode_fixup_kernel, dim3(d.nslabs), dim3(256), 0, stream, p, NT);
+    qg::I8DecodeParams p{t,
+                         sw,
+                         Y,
+                         acc_dbg,
+                         reinterpret_cast<int32_t*>(static_cast<uint8_t*>(ws) + d.flags_bytes),
+                         static_cast<unsigned long long*>(ws),
+                         next_decode_token(),
+                         M,
+                         K,
+                         N,
+                         d.KB,
+                         d.nslabs,
+                         d.units,
+                         d.grid};
+    return launch_pdl(kern, dim3(d.grid), dim3(C::THREADS), C::TOTAL, stream, p, tw, tx);
 }
 
 // W4A8 stream-K (17 <= M < 128; M <= 64 per launch, larger M in chunks of 64 tokens).
@@ -667,7 +681,8 @@ I8Plan w4a8_plan(int M, int K, int N)
     d.nslabs = (N + 127) / 128;
     d.units = d.KB * d.nslabs;
     d.grid = std::min(std::min(num_sms(), d.units), 160);
-    d.partial_bytes = (size_t)d.grid * 2 * 128 * d.NT * sizeof(float);
+    d.flags_bytes = ((size_t)d.grid * 8 + 255) / 256 * 256;
+    d.partial_bytes = d.flags_bytes + (size_t)d.grid * 128 * d.NT * sizeof(float);
     return d;
 }
 
@@ -688,9 +703,21 @@ qg_status launch_w4a8_decode(const int8_t* Xq, const float* t, int M, int K, con
                            CU_TENSOR_MAP_SWIZZLE_NONE)) ||
         (st = make_tmap_2d(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, Xq, K, M, 128, NT, CU_TENSOR_MAP_SWIZZLE_128B)))
         return st;
-    qg::W4A8DecodeParams p{t, sg, Y, part_dbg, static_cast<float*>(ws), M, K, N, d.KB, d.nslabs, d.units, d.grid};
-    if ((st = launch_pdl(kern, dim3(d.grid), dim3(C::THREADS), C::TOTAL, stream, p, tw, tx)) != QG_OK) return st;
-    return launch_pdl(qg::w4a8_decode_fixup_kernel, dim3(d.nslabs), dim3(256), 0, stream, p, NT);
+    qg::W4A8DecodeParams p{t,
+                           sg,
+                           Y,
+                           part_dbg,
+                           reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + d.flags_bytes),
+                           static_cast<unsigned long long*>(ws),
+                           next_decode_token(),
+                           M,
+                           K,
+                           N,
+                           d.KB,
+                           d.nslabs,
+                           d.units,
+                           d.grid};
+    return launch_pdl(kern, dim3(d.grid), dim3(C::THREADS), C::TOTAL, stream, p, tw, tx);
 }
 
 // AWQ search workspace: every buffer one candidate needs, 256-byte aligned pieces
@@ -1045,7 +1072,7 @@ qg_status qg_gemm_w4a8(const int8_t* Xq, const float* t, int M, int K, const uin
     if (workspace && M >= kW4A8DecodeMinM) {
         if (ws_bytes < qg_workspace_size(QG_OP_GEMM_W4A8, M, K, N)) return QG_ERR_WORKSPACE;
         for (int m0 = 0; m0 < M; m0 += kW4A8DecodeMaxM) {
-            // chunks run in stream order; each reuses the workspace after the previous fixup
+            // chunks run in stream order; each reuses the workspace after the previous chunk's launch
             // (a ragged last chunk of 16 tokens or fewer runs on the 32-token tile)
             const int mc = std::min(kW4A8DecodeMaxM, M - m0);
             const int nt = w4a8_plan(mc, K, N).NT;
@@ -1490,23 +1517,6 @@ qg_status qg_quantize_w8_channel(const float* W, const float* s, int K, int N, i
         qg::w8_scale_kernel<<<(N + 255) / 256, 256, 0, st>>>(sw, N);
         QG_CUDA(cudaGetLastError());
         return QG_OK;
-    }
-    if (N % 32 == 0 && K <= 8192) {
-        // one pass over W: 32-column strips, K split over a cluster of up to 8 CTAs
-        if (K <= 4096) {
-            const int C = (K + 511) / 512;
-            return launch_cluster(qg::quantize_w8_strip32_kernel<8>, dim3(N / 32, C), dim3(512), 0, C, stream, W, s, K,
-                                  N, Wq, sw);
-        }
-        const int C = (K + 1023) / 1024;
-        return launch_cluster(qg::quantize_w8_strip32_kernel<16>, dim3(N / 32, C), dim3(512), 0, C, stream, W, s, K, N,
-                              Wq, sw);
-    }
-    if (N % 8 == 0 && K <= 8 * qg::kW8StripRows) {
-        // one pass over W: 8-column strips, K split over a cluster of up to 8 CTAs
-        const int C = (K + qg::kW8StripRows - 1) / qg::kW8StripRows;
-        return launch_cluster(qg::quantize_w8_strip_kernel, dim3(N / 8, C), dim3(qg::kW8StripThreads), 0, C, stream,
-                              W, s, K, N, Wq, sw);
     }
     qg::quantize_w8_channel_kernel<<<(N + 127) / 128, 128, 0, reinterpret_cast<cudaStream_t>(stream)>>>(W, s, K, N,
                                                                                                           Wq, sw);

@@ -422,107 +422,18 @@ __global__ void smooth_finalize_kernel(float* __restrict__ s_io /*in: ax*/, floa
 
 // ---------------------------------------------------------------------------
 // Per-output-channel symmetric INT8 ("AI Infra guide, ch.4" sec. 1.2-1.3) on
-// W~ = diag(s) W, one HBM pass: a strip of 8 columns (32-byte row segments) is
-// split along K over the CTAs of a thread-block cluster (up to 8), each CTA holding
-// its rows of the strip in registers (4 rows x 8 columns per thread, 2048 rows per
-// CTA).  The column absmax (exact in any order) is reduced within the CTA with warp
-// shuffles, then across the cluster through distributed shared memory; each CTA then
-// quantizes the values it holds.  For N % 8 == 0 and K <= 16384.
+// W~ = diag(s) W: sw[n] = max_k |W~[k][n]| / 127, Wq = clamp(round(W~ / sw), -127, 127).
 // ---------------------------------------------------------------------------
-// Wider strips for the same computation (N % 32 == 0): a strip of 32 columns, K split
-// over a cluster of C CTAs of 512 threads; thread (q, r) takes columns 4q .. 4q + 3
-// and rows r, r + 64, .. of its CTA's range (RPT of them), so a warp reads 4 rows x
-// 128 bytes per load and writes 4 rows x 32 bytes per store.  The column absmax meets
-// in shared memory, then across the cluster through distributed shared memory.
-template <int RPT>
-__global__ void __launch_bounds__(512) quantize_w8_strip32_kernel(const float* __restrict__ W,
-                                                                  const float* __restrict__ s, int K, int N,
-                                                                  int8_t* __restrict__ Wq, float* __restrict__ sw)
-{
-    __shared__ float wmax[16][32];
-    __shared__ __align__(16) float cmax[32];
-    __shared__ float csc[32];
-    const int n0 = 32 * blockIdx.x;
-    const uint32_t rank = cluster_ctarank();
-    const int C = (int)gridDim.y;  // the whole y extent is one cluster
-    const int kb = (int)((int64_t)K * rank / C), ke = (int)((int64_t)K * (rank + 1) / C);
-    const int cq = threadIdx.x & 7, rr = threadIdx.x >> 3;
-    float v[RPT][4];
-    float a[4] = {0.f, 0.f, 0.f, 0.f};
-    bool bad = false;
-#pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-        const int k = kb + rr + 64 * i;
-        if (k < ke) {
-            float4 w = __ldg(reinterpret_cast<const float4*>(W + (int64_t)k * N + n0 + 4 * cq));
-            if (s) {
-                const float sk = __ldg(s + k);
-                w = make_float4(__fmul_rn(w.x, sk), __fmul_rn(w.y, sk), __fmul_rn(w.z, sk), __fmul_rn(w.w, sk));
-            }
-            v[i][0] = w.x; v[i][1] = w.y; v[i][2] = w.z; v[i][3] = w.w;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                bad |= !isfinite(v[i][c]);
-                a[c] = fmaxf(a[c], fabsf(v[i][c]));
-            }
-        } else {
-#pragma unroll
-            for (int c = 0; c < 4; ++c) v[i][c] = 0.0f;
-        }
-    }
-    if (bad) set_status(5u);
-    // lanes with the same column quad: lane bits 3 and 4
-#pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        a[c] = fmaxf(a[c], __shfl_xor_sync(0xffffffffu, a[c], 8));
-        a[c] = fmaxf(a[c], __shfl_xor_sync(0xffffffffu, a[c], 16));
-    }
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane < 8)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) wmax[warp][4 * lane + c] = a[c];
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        float m = 0.0f;
-        for (int w = 0; w < 16; ++w) m = fmaxf(m, wmax[w][threadIdx.x]);
-        cmax[threadIdx.x] = m;
-    }
-    cluster_sync();
-    if (threadIdx.x < 32) {
-        float m = 0.0f;
-        const uint32_t la = smem_u32(&cmax[threadIdx.x]);
-        for (int r = 0; r < C; ++r) m = fmaxf(m, ld_dsmem_f32(dsmem_addr(la, (uint32_t)r)));
-        const float sc = __fdiv_rn(m, 127.0f);  // the column scale
-        csc[threadIdx.x] = sc;
-        if (rank == 0) sw[n0 + threadIdx.x] = sc;
-    }
-    cluster_sync();  // every CTA has read every cmax before any CTA moves on (and csc is set)
-    float sc[4];
-#pragma unroll
-    for (int c = 0; c < 4; ++c) sc[c] = csc[4 * cq + c];
-#pragma unroll
-    for (int i = 0; i < RPT; ++i) {
-        const int k = kb + rr + 64 * i;
-        if (k < ke) {
-            uint32_t word = 0;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                int q = 0;
-                if (sc[c] != 0.0f && isfinite(v[i][c])) q = min(max(__float2int_rn(__fdiv_rn(v[i][c], sc[c])), -127), 127);
-                word |= (uint32_t)(q & 0xFF) << (8 * c);
-            }
-            *reinterpret_cast<uint32_t*>(Wq + (int64_t)k * N + n0 + 4 * cq) = word;
-        }
-    }
-}
-
 // Per-output-channel INT8 in two streaming passes (N % 4 == 0): pass 1 takes the column
 // absmax of W~ = diag(s) W (|w| as integer bits, combined with atomicMax: the maximum of
 // non-negative floats, exact in any order; non-finite values are reported and left
 // out), pass 2 quantizes with sw = absmax / 127, and a last pass turns the absmax into
 // sw in place.  Every pass is a CTA of 256 threads over 128 columns x 256 rows with
-// 16-byte loads (a warp reads one 512-byte row segment) and 4-byte stores: W is read
-// twice, but at the copy rate, which beats one pass that must meet across K.
+// 16-byte loads (a warp reads one 512-byte row segment) and 4-byte stores.  W is read
+// twice: a one-read form (the rows of a column strip split over an 8-CTA cluster, held
+// in shared memory, the absmax met through distributed shared memory) measured slower,
+// held back by the cluster barrier per strip and by clusters of 8 filling 120 of 148 SMs,
+// and so did running the passes over L2-sized column chunks.
 __global__ void __launch_bounds__(256) w8_absmax_kernel(const float* __restrict__ W, const float* __restrict__ s,
                                                         int K, int N, unsigned int* __restrict__ amax_bits)
 {
@@ -601,92 +512,6 @@ __global__ void __launch_bounds__(256) w8_scale_kernel(float* __restrict__ sw, i
 {
     const int n = blockIdx.x * blockDim.x + threadIdx.x;
     if (n < N) sw[n] = __fdiv_rn(__uint_as_float(__float_as_uint(sw[n])), 127.0f);
-}
-
-constexpr int kW8StripThreads = 512;
-constexpr int kW8StripRowsPerThread = 4;
-constexpr int kW8StripRows = kW8StripThreads * kW8StripRowsPerThread;  // rows of K per CTA
-
-__global__ void __launch_bounds__(kW8StripThreads) quantize_w8_strip_kernel(const float* __restrict__ W,
-                                                                            const float* __restrict__ s, int K,
-                                                                            int N, int8_t* __restrict__ Wq,
-                                                                            float* __restrict__ sw)
-{
-    __shared__ float wmax[kW8StripThreads / 32][8];
-    __shared__ __align__(16) float cmax[8];
-    const int n0 = 8 * blockIdx.x;
-    const uint32_t rank = cluster_ctarank();
-    const int C = (int)gridDim.y;  // the whole y extent is one cluster
-    const int kb = (int)((int64_t)K * rank / C), ke = (int)((int64_t)K * (rank + 1) / C);
-    float v[kW8StripRowsPerThread][8];
-    float a[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) a[c] = 0.0f;
-    bool bad = false;
-#pragma unroll
-    for (int i = 0; i < kW8StripRowsPerThread; ++i) {
-        const int k = kb + (int)threadIdx.x + kW8StripThreads * i;
-        if (k < ke) {
-            const float4* src = reinterpret_cast<const float4*>(W + (int64_t)k * N + n0);
-            const float4 lo = __ldg(src), hi = __ldg(src + 1);
-            const float sk = s ? __ldg(s + k) : 1.0f;
-            const float raw[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                v[i][c] = s ? __fmul_rn(raw[c], sk) : raw[c];
-                bad |= !isfinite(v[i][c]);
-                a[c] = fmaxf(a[c], fabsf(v[i][c]));
-            }
-        } else {
-#pragma unroll
-            for (int c = 0; c < 8; ++c) v[i][c] = 0.0f;
-        }
-    }
-    if (bad) set_status(5u);
-    // CTA absmax per column
-#pragma unroll
-    for (int c = 0; c < 8; ++c)
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) a[c] = fmaxf(a[c], __shfl_xor_sync(0xffffffffu, a[c], o));
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    if (lane == 0)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) wmax[warp][c] = a[c];
-    __syncthreads();
-    if (threadIdx.x < 8) {
-        float m = 0.0f;
-        for (int w = 0; w < kW8StripThreads / 32; ++w) m = fmaxf(m, wmax[w][threadIdx.x]);
-        cmax[threadIdx.x] = m;
-    }
-    // cluster absmax per column through distributed shared memory
-    cluster_sync();
-    if (threadIdx.x < 8) {
-        float m = 0.0f;
-        const uint32_t la = smem_u32(&cmax[threadIdx.x]);
-        for (int r = 0; r < C; ++r) m = fmaxf(m, ld_dsmem_f32(dsmem_addr(la, (uint32_t)r)));
-        wmax[0][threadIdx.x] = __fdiv_rn(m, 127.0f);  // the column scale
-    }
-    cluster_sync();  // every CTA has read every cmax before any CTA moves on
-    float sc[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) sc[c] = wmax[0][c];
-    if (rank == 0 && threadIdx.x < 8 && n0 + (int)threadIdx.x < N) sw[n0 + threadIdx.x] = sc[threadIdx.x];
-#pragma unroll
-    for (int i = 0; i < kW8StripRowsPerThread; ++i) {
-        const int k = kb + (int)threadIdx.x + kW8StripThreads * i;
-        if (k < ke) {
-            uint32_t lo = 0, hi = 0;
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                int q = 0;
-                if (sc[c] != 0.0f && isfinite(v[i][c])) q = min(max(__float2int_rn(__fdiv_rn(v[i][c], sc[c])), -127), 127);
-                const uint32_t b = (uint32_t)(q & 0xFF) << (8 * (c & 3));
-                if (c < 4) lo |= b;
-                else hi |= b;
-            }
-            *reinterpret_cast<uint2*>(Wq + (int64_t)k * N + n0) = make_uint2(lo, hi);
-        }
-    }
 }
 
 // ---------------------------------------------------------------------------

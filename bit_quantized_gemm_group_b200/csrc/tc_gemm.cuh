@@ -139,9 +139,6 @@ QG_DEV_INLINE bool warp_wait(uint64_t* bar, uint32_t parity)
     return __shfl_sync(0xffffffffu, ok, 0) != 0;
 }
 
-// exact int32 -> fp32 for |v| < 2^22: add into the mantissa of 1.5 * 2^23, subtract it back
-QG_DEV_INLINE float i2f_small(uint32_t v) { return __uint_as_float(v + 0x4B400000u) - 12582912.0f; }
-
 template <int KIND>
 __global__ void __launch_bounds__(TcCfg<KIND>::THREADS, 1)
     tc_gemm_kernel(const TcParams p, const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_b)

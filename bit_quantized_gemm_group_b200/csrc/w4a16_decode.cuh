@@ -106,11 +106,12 @@ struct DecodeSmem {
     static constexpr int RED = RED_K > MP * TS * 4 ? RED_K : MP * TS * 4;  // the result tile aliases it
     static constexpr int SIDE = OUT ? 2 * MP * kDecBN * 4 : 0;  // side-path sums of a piece, 2 x [token][128] fp32
     static constexpr int TOTAL = ST * STAGE + RED + SIDE + 3 * ST * 8 + 16 + 1024;
-    // The producer is one warp after the consumers, or (PWG) a whole warpgroup of which
-    // the first warp works, so that the register file can be split with setmaxnreg: the
-    // producer warps keep 56 registers a thread (136 with the side path) and the consumers
-    // take the rest.
-    static constexpr int THREADS = 32 * NW + (PWG ? 128 : 32);
+    // The producer is a whole warpgroup after the consumers, whose first two warps issue
+    // (the weights, the activations) and, with the side path, whose last two sum it, so
+    // that the register file can be split with setmaxnreg: the producer warps keep 56
+    // registers a thread (136 with the side path) and the consumers take the rest.  (Two
+    // bare issuer warps without the split measured slower.)
+    static constexpr int THREADS = 32 * NW + 128;
     static constexpr int REG_LAUNCH = (65536 / THREADS) / 8 * 8 > 255 ? 248 : (65536 / THREADS) / 8 * 8;
     static constexpr int REG_PRODUCER = OUT ? 136 : 56;
     static constexpr int REG_CONSUMER_RAW = (REG_LAUNCH * THREADS - REG_PRODUCER * 128) / (32 * NW) / 8 * 8;
@@ -138,18 +139,6 @@ QG_DEV_INLINE void tma_load_4d(const CUtensorMap* m, uint64_t* bar, void* smem_d
         "%6}], [%2];" ::"r"(smem_u32(smem_dst)),
         "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(y), "r"(z), "r"(w)
         : "memory");
-}
-
-QG_DEV_INLINE unsigned long long ld_acquire_u64(const unsigned long long* p)
-{
-    unsigned long long v;
-    asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-    return v;
-}
-
-QG_DEV_INLINE void st_release_u64(unsigned long long* p, unsigned long long v)
-{
-    asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
 }
 
 // Walks a CTA's schedule: pieces (runs of groups within one slab) in order, each cut
@@ -282,7 +271,7 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG, SP, OUT>::THR
                                         for (int r = 0; r < kDecOutMax; ++r) {
                                             if (r < cnt) {
                                                 int k = (int)((i4[r] >> (8 * j)) & 0xFFu);
-                                                const float w = __fmul_rn((float)(int8_t)((q4[r] >> (8 * j)) & 0xFFu), s8v[j]);
+                                                const float w = __fmul_rn(i2f_small((uint32_t)(int32_t)(int8_t)((q4[r] >> (8 * j)) & 0xFFu)), s8v[j]);
                                                 if (k >= kDecBN) {  // not an offset inside the group: skipped, reported
                                                     bad = true;
                                                     continue;

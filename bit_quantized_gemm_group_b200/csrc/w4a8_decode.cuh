@@ -18,9 +18,11 @@
 //     group's P into a TMEM buffer of their own: an MMA holds its issuing thread for a
 //     while, and a unit here is half the bytes of a W8A8 unit.
 //   * Epilogue warps (thread = column) read each group's P, add float(P) s_g into fp32
-//     registers (and, on request, store P), and at a piece end finish Y or leave the fp32
-//     piece in the workspace for `w4a8_decode_fixup_kernel`, which adds the pieces of a
-//     split slab in CTA order.
+//     registers (and, on request, store P), and at a piece end finish Y, or publish the
+//     fp32 piece in the workspace under the launch's token (a split slab's later pieces,
+//     always their CTAs' first), or, holding the slab's first group (always the CTA's
+//     last piece), wait (bounded) for the other pieces' tokens, add them in CTA order and
+//     finish Y.  One launch per call.
 // Stage ring, A buffers and D buffers have even depth, so every mbarrier has one consumer
 // that waits on its phases in order.
 #pragma once
@@ -34,7 +36,9 @@ struct W4A8DecodeParams {
     const float* sg;   // fp32 [G][N]
     uint16_t* Y;       // bf16 [M][N]
     int32_t* dbg;      // NULL or int32 [M][G][N]: receives every P
-    float* partials;   // [grid][2][NT][128]
+    float* partials;   // [grid][NT][128]: the CTA's published piece
+    unsigned long long* flags;  // [grid] publication tokens
+    unsigned long long token;   // this launch's token (never 0)
     int M, K, N;
     int G, nslabs, units, grid;
 };
@@ -212,14 +216,15 @@ __global__ void __launch_bounds__(W4A8DecCfg<NT, NI>::THREADS, 1)
         float acc[TPW];
 #pragma unroll
         for (int t = 0; t < TPW; ++t) acc[t] = 0.f;
-        bool first_piece = true;
+        bool ok = true;  // after a wait gives up, the units are still walked (named barriers) without work
         for (int i = 0; i < n_it; ++i) {
             const int u = u0 + i, slab = u / G, g = u % G, n = slab * 128 + col;
             const int e = i % NI, j = i / NI, d = e * DP + j % DP;
             fetch_sg(i + LA - 1);
             cp_async_wait_group<LA - 1>();  // unit i's group has landed
             const float sv = sgr[(i % LA) * 32];
-            if (!mbar_wait(&dfull[d], (j / DP) & 1)) break;
+            if (ok && !mbar_wait(&dfull[d], (j / DP) & 1)) ok = false;
+            if (ok) {
             tc_fence_after();
             const uint32_t dcol = tmem + ((uint32_t)(32 * q) << 16) + d * NT + tb;
 #pragma unroll
@@ -229,7 +234,7 @@ __global__ void __launch_bounds__(W4A8DecCfg<NT, NI>::THREADS, 1)
                     tmem_ld_32x32b_x16(dcol + t0, P);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int t = 0; t < 16; ++t) acc[t0 + t] = fmaf(__int2float_rn((int32_t)P[t]), sv, acc[t0 + t]);
+                    for (int t = 0; t < 16; ++t) acc[t0 + t] = fmaf(i2f_small(P[t]), sv, acc[t0 + t]);  // |P| < 2^17
                 }
             }
             if (p.dbg) {  // the exact P, on request: one column at a time, off the fast path
@@ -243,25 +248,51 @@ __global__ void __launch_bounds__(W4A8DecCfg<NT, NI>::THREADS, 1)
             }
             tc_fence_before();
             mbar_arrive(&dempty[d]);
+            }
             if (i + 1 == n_it || g == G - 1) {
-                // piece end: a whole slab finishes Y, a partial one goes to this CTA's slot
+                // piece end: a whole slab finishes Y; a later piece of a split slab is
+                // published; the piece holding the slab's first group finishes the slab
                 const int gstart = slab == u0 / G ? u0 % G : 0;
-                if (gstart == 0 && g == G - 1) {
-                    if (n < p.N) {
+                const bool whole = gstart == 0 && g == G - 1;
+                const bool head = gstart == 0 && !whole;
+                if (head) {
+                    const int cl = i8_cta_of_unit(slab * G + G - 1, p.units, p.grid);
+                    bool ready = true;
+                    if (warp == 4 && ok) ready = watch_tokens(p.flags, (int)blockIdx.x + 1, cl, p.token, lane);
+                    if (!named_bar_and(1, 32 * C::EPI, ok && ready)) ok = false;
+                    if (ok) {
+                        // the other pieces in CTA order (the order of the sum is fixed)
+                        for (int c = (int)blockIdx.x + 1; c <= cl; ++c) {
+                            const float* other = p.partials + (size_t)c * NT * 128 + tb * 128 + col;
+#pragma unroll
+                            for (int t = 0; t < TPW; ++t)
+                                if (tb + t < M) acc[t] += __ldcg(other + t * 128);
+                        }
+                    }
+                }
+                if (whole || head) {
+                    if (ok && n < p.N) {
                         uint16_t* y = p.Y + (int64_t)tb * p.N + n;
 #pragma unroll
                         for (int t = 0; t < TPW; ++t)
                             if (tb + t < M) y[(int64_t)t * p.N] = f32_to_bf16_bits(__fmul_rn(ts[tb + t], acc[t]));
                     }
                 } else {
-                    float* mine = p.partials + ((size_t)blockIdx.x * 2 + (first_piece ? 0 : 1)) * NT * 128 + tb * 128 + col;
+                    float* mine = p.partials + (size_t)blockIdx.x * NT * 128 + tb * 128 + col;
+                    if (ok) {
 #pragma unroll
-                    for (int t = 0; t < TPW; ++t)
-                        if (tb + t < M) mine[t * 128] = acc[t];
+                        for (int t = 0; t < TPW; ++t)
+                            if (tb + t < M) __stcg(mine + t * 128, acc[t]);
+                    }
+                    // publish: every epilogue thread's stores, then one fence and the token
+                    named_bar_sync(1, 32 * C::EPI);
+                    if (ok && threadIdx.x == 128) {
+                        __threadfence();
+                        st_release_u64(p.flags + blockIdx.x, p.token);
+                    }
                 }
 #pragma unroll
                 for (int t = 0; t < TPW; ++t) acc[t] = 0.f;
-                first_piece = false;
             }
         }
         cp_async_wait_group<0>();  // no copy into shared memory outlives the loop
@@ -312,42 +343,6 @@ __global__ void __launch_bounds__(W4A8DecCfg<NT, NI>::THREADS, 1)
         __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, C::TMEM_COLS);
-    }
-}
-
-// Adds the fp32 pieces of every slab the decode grid split between CTAs, in CTA order,
-// and finishes Y; slabs held by one CTA were finished by the decode kernel.
-__global__ void __launch_bounds__(256) w4a8_decode_fixup_kernel(const W4A8DecodeParams p, int NT)
-{
-    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
-    const int slab = blockIdx.x;
-    const int G = p.G;
-    const int cf = i8_cta_of_unit(slab * G, p.units, p.grid);
-    const int cl = i8_cta_of_unit(slab * G + G - 1, p.units, p.grid);
-    if (cf == cl) return;
-    __shared__ int off[160];
-    for (int c = cf + threadIdx.x; c <= cl; c += blockDim.x) {
-        const int sl = i8_first_unit(c, p.units, p.grid) >= slab * G ? 0 : 1;  // first piece of CTA c?
-        off[c - cf] = (c * 2 + sl) * NT * 128;
-    }
-    __syncthreads();
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-    const int np = cl - cf + 1;
-    const int mrows = min(p.M, NT);
-    for (int e = threadIdx.x; e < mrows * 32; e += blockDim.x) {
-        const int t = e >> 5, c4 = 4 * (e & 31), n = slab * 128 + c4;
-        if (n >= p.N) continue;  // N % 16 == 0: the 4 columns are all in range or all out
-        const int o = t * 128 + c4;
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int i = 0; i < np; ++i) {  // in piece order
-            const float4 a = __ldcg(reinterpret_cast<const float4*>(p.partials + off[i] + o));
-            v.x += a.x; v.y += a.y; v.z += a.z; v.w += a.w;
-        }
-        const float tm = __ldg(p.t + t);
-        const uint16_t y0 = f32_to_bf16_bits(__fmul_rn(tm, v.x)), y1 = f32_to_bf16_bits(__fmul_rn(tm, v.y));
-        const uint16_t y2 = f32_to_bf16_bits(__fmul_rn(tm, v.z)), y3 = f32_to_bf16_bits(__fmul_rn(tm, v.w));
-        *reinterpret_cast<uint2*>(p.Y + (int64_t)t * p.N + n) =
-            make_uint2((uint32_t)y0 | ((uint32_t)y1 << 16), (uint32_t)y2 | ((uint32_t)y3 << 16));
     }
 }
 

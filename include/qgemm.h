@@ -187,10 +187,11 @@ qg_status qg_smooth_quant_act_i8(const uint16_t* X, int M, int K, const float* i
  * acc_dbg: NULL, or int32 [M][N] that also receives the exact accumulators.
  * Rules: K % 128 == 0, N % 16 == 0.
  * workspace: NULL, or (M < 128) a device buffer of at least
- *   qg_workspace_size(QG_OP_GEMM_W8A8, M, K, N) bytes (contents irrelevant; it holds
- *   the int32 partial sums of column slabs split between CTAs).  With it, M < 128 runs
- *   the stream-K tensor-core kernel; without it, the cluster split-K kernel.  Both give
- *   the same bits.  A workspace smaller than required -> QG_ERR_WORKSPACE before any
+ *   qg_workspace_size(QG_OP_GEMM_W8A8, M, K, N) bytes (contents irrelevant: it holds
+ *   per-launch 64-bit publication tokens and the int32 partial sums of column slabs
+ *   split between CTAs, which the CTA holding a slab's first block adds in the same
+ *   launch).  With it, M < 128 runs the stream-K tensor-core kernel (one launch); without
+ *   it, the cluster split-K kernel.  Both give the same bits.  A workspace smaller than required -> QG_ERR_WORKSPACE before any
  *   launch.  Calls that may run concurrently need workspaces of their own.
  * ------------------------------------------------------------------------ */
 qg_status qg_gemm_w8a8(const int8_t* Xq, const float* t, int M, int K, const int8_t* Wq,
@@ -208,10 +209,12 @@ qg_status qg_gemm_w8a8(const int8_t* Xq, const float* t, int M, int K, const int
  * part_dbg: NULL, or int32 [M][K/group][N] that also receives every P.
  * Rules: group == 128, K % 128 == 0, N % 16 == 0.
  * workspace: NULL, or (17 <= M < 128) a device buffer of at least
- *   qg_workspace_size(QG_OP_GEMM_W4A8, M, K, N) bytes (contents irrelevant; it holds
- *   the fp32 partial sums of column slabs split between CTAs; the size is 0, and any
- *   workspace is ignored, for M <= 16 and M >= 128).  With it, 17 <= M < 128 runs the
- *   stream-K tensor-core kernel on chunks of up to 64 tokens; without it (and always at
+ *   qg_workspace_size(QG_OP_GEMM_W4A8, M, K, N) bytes (contents irrelevant: it holds
+ *   per-launch publication tokens and the fp32 partial sums of column slabs split
+ *   between CTAs, added in CTA order by the CTA holding a slab's first group in the same
+ *   launch; the size is 0, and any workspace is ignored, for M <= 16 and M >= 128).
+ *   With it, 17 <= M < 128 runs the stream-K tensor-core kernel (one launch per chunk)
+ *   on chunks of up to 64 tokens; without it (and always at
  *   M <= 16), the cluster split-K kernel.  P is exact either way; Y may differ in the last bit
  *   (fp32 summation order).  A workspace smaller than required -> QG_ERR_WORKSPACE
  *   before any launch.  Calls that may run concurrently need workspaces of their own.

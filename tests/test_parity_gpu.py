@@ -62,6 +62,14 @@ def test_quantize_w4_asym_and_pack_bitexact(K, N, cfg):
         W[0:128, 0] = 0.0          # zero group
         W[128:256, 1] = 0.25       # constant group
         W[:, 2] = np.float32(0.5) * np.round(W[:, 2] * 64)  # many exact .5 ties of x/s
+        # group range [0, 15 c], c = 2^-8: s = c exactly, z = 0; x / s exactly on (column 3)
+        # and 2^-16 beside (column 4) the half-integers j + 1/2
+        c = np.float32(2.0 ** -8)
+        j = (np.arange(K) % 15).astype(np.float32)
+        W[:, 3] = (j + np.float32(0.5)) * c
+        W[:, 4] = (j + np.float32(0.5) + np.where(np.arange(K) % 2 == 0, 1, -1).astype(np.float32) * 2.0 ** -16) * c
+        W[0::128, 3] = W[0::128, 4] = 0.0
+        W[1::128, 3] = W[1::128, 4] = 15 * c
     codes, scales, zeros, packed = quant_w4_asym(W)
     c_o, s_o, z_o, st = oracle.quantize_w4_asym(W)
     assert st == oracle.OK
@@ -96,14 +104,23 @@ def test_smooth_scales_and_w8_channel_bitexact():
 
 @pytest.mark.parametrize("K,N,smooth", [(11008, 4096, True), (16384, 64, False), (2048, 24, True), (100, 136, True),
                                          (4096, 100, True), (20000, 8, False), (6000, 96, True), (700, 64, False),
-                                         (8192, 32, True), (4096, 11008, False)])
+                                         (8192, 32, True), (4096, 11008, False), (300, 30, True),
+                                         (25700, 16, False)])
 def test_quantize_w8_channel_shapes_bitexact(K, N, smooth):
-    """Every path of the INT8 channel quantizer: the 32-column strip kernel (N % 32 == 0,
-    K <= 8192: clusters of 1..8 CTAs along K with 8 or 16 rows a thread, ragged last CTA),
-    the 8-column strip kernel (N % 8 == 0, K <= 16384) and the general kernel (other
-    shapes); a zero column and smoothing on and off."""
+    """Both paths of the INT8 channel quantizer: the two-pass kernels over column chunks
+    of about 40 MB of W (N % 4 == 0: one chunk at most shapes, 5 at 4096 x 11008 and
+    at 11008 x 4096, ragged last chunks and last CTAs) and the general kernel (N % 4 != 0);
+    a zero column, and columns whose quotients w / sw sit exactly on and within 2^-16 of
+    half-integers (ties to even, and the product form's fallback to the quotient),
+    smoothing on and off."""
     W = synth.weights(K, N, 0.02, 0.01, 8.0, seed=K + N)
     W[:, 3] = 0.0
+    if N > 7:
+        c = np.float32(2.0 ** -10)  # sw = 127 c / 127 = c exactly
+        j = (np.arange(K) % 254 - 127).astype(np.float32)
+        W[:, 5] = (j + np.float32(0.5)) * c  # exact ties
+        W[:, 6] = (j + np.float32(0.5) + np.where(np.arange(K) % 2 == 0, 1, -1).astype(np.float32) * 2.0 ** -16) * c
+        W[0, 5] = W[0, 6] = 127 * c
     s_o = None
     if smooth:
         s_o = np.random.default_rng(K).uniform(0.5, 2.0, K).astype(np.float32)
@@ -224,8 +241,8 @@ def test_gemm_w4a16_decode_without_workspace(K, N):
 
 
 def test_gemm_w4a16_decode_repeatable():
-    """Stream-K fixup: calls in a row give identical bits (the split slabs' pieces are summed
-    in a fixed order by the fixup kernel)."""
+    """Stream-K finish: calls in a row give identical bits (the split slabs' pieces are summed
+    in a fixed order by the CTA that finishes each slab)."""
     _w4a16_case(4096, 12288, "w4a16_decode", [1, 4, 32], "bf16", repeat=3)
 
 
