@@ -288,19 +288,9 @@ QG_DEV_INLINE void tmem_dealloc(uint32_t taddr, uint32_t ncols)
 QG_DEV_INLINE void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 QG_DEV_INLINE void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// D[tmem] (+)= A[smem] * B[smem]^T for one instruction shape; kind::f16 (bf16/fp16 in, fp32 out)
-QG_DEV_INLINE void mma_f16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc, uint32_t accum)
-{
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accum)
-        : "memory");
-}
-
-// Same, with A read from tensor memory: lane i holds row i of A, and each 32-bit
-// column holds two consecutive k values (so one K = 16 step spans 8 columns).
+// D[tmem] (+)= A[tmem] * B[smem]^T for one instruction shape; kind::f16 (bf16/fp16 in,
+// fp32 out).  Lane i of A holds row i, and each 32-bit column holds two consecutive k
+// values (so one K = 16 step spans 8 columns).
 QG_DEV_INLINE void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc, uint32_t accum)
 {
     asm volatile(
@@ -384,19 +374,6 @@ QG_DEV_INLINE uint32_t tmem_ld_32x32b_x1(uint32_t taddr)
 
 QG_DEV_INLINE void tmem_ld_wait() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
-// 32 registers per thread -> 32 lanes x 32 consecutive 32-bit columns
-QG_DEV_INLINE void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32])
-{
-    asm volatile(
-        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
-        "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
-        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]),
-        "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
-        "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
-        : "memory");
-}
-
 // 16 registers per thread -> 32 lanes x 16 consecutive 32-bit columns
 QG_DEV_INLINE void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16])
 {
@@ -445,15 +422,6 @@ QG_DEV_INLINE uint32_t dsmem_addr(uint32_t local_saddr, uint32_t rank)
     uint32_t r;
     asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local_saddr), "r"(rank));
     return r;
-}
-
-QG_DEV_INLINE float4 ld_dsmem_f4(uint32_t addr)
-{
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(addr));
-    return v;
 }
 
 QG_DEV_INLINE float ld_dsmem_f32(uint32_t addr)
