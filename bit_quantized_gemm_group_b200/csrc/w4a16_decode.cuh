@@ -262,6 +262,31 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG, SP, OUT>::THR
                                         q4[r] = r < cnt ? *reinterpret_cast<const uint32_t*>(st + L::OC_OFF + (gi * cnt + r) * kDecBN + c0) : 0u;
                                     }
                                     const uint8_t* xgrp = st + L::X_OFF + gi * L::XG;
+                                    if (M == 1) {
+                                        // one token (row 0 of the tile, no swizzle offset): a
+                                        // loop of its own, so the code it runs stays compact
+#pragma unroll
+                                        for (int j = 0; j < 4; ++j) {
+                                            float g1 = SREG ? sacc[j][0] : 0.0f;
+#pragma unroll
+                                            for (int r = 0; r < kDecOutMax; ++r) {
+                                                if (r < cnt) {
+                                                    const int k = (int)((i4[r] >> (8 * j)) & 0xFFu);
+                                                    const float w = __fmul_rn(i2f_small((uint32_t)(int32_t)(int8_t)((q4[r] >> (8 * j)) & 0xFFu)), s8v[j]);
+                                                    if (k >= kDecBN) {  // not an offset inside the group: skipped, reported
+                                                        bad = true;
+                                                        continue;
+                                                    }
+                                                    const uint16_t xb = *reinterpret_cast<const uint16_t*>(
+                                                        xgrp + (k >> 6) * (MP * 128) + (k & 7) * 2 + (((k & 63) >> 3) << 4));
+                                                    const float xv = BF16 ? bf16_bits_to_f32(xb) : __half2float(__ushort_as_half(xb));
+                                                    g1 = fmaf(xv, w, g1);
+                                                }
+                                            }
+                                            if constexpr (SREG) sacc[j][0] = g1;
+                                            else mine[c0 + j] += g1;
+                                        }
+                                    } else {
 #pragma unroll
                                     for (int j = 0; j < 4; ++j) {
                                         float gacc[MP];
@@ -278,12 +303,6 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG, SP, OUT>::THR
                                                 }
                                                 const uint8_t* xk = xgrp + (k >> 6) * (MP * 128) + (k & 7) * 2;
                                                 const int ch = (k & 63) >> 3;
-                                                if (M == 1) {  // one token: row 0 of the tile, no swizzle offset
-                                                    const uint16_t xb = *reinterpret_cast<const uint16_t*>(xk + (ch << 4));
-                                                    const float xv = BF16 ? bf16_bits_to_f32(xb) : __half2float(__ushort_as_half(xb));
-                                                    gacc[0] = fmaf(xv, w, gacc[0]);
-                                                    continue;
-                                                }
 #pragma unroll
                                                 for (int mb = 0; mb < MP / 8; ++mb) {
                                                     if (8 * mb < M) {
@@ -308,6 +327,7 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG, SP, OUT>::THR
                                             for (int m = 0; m < MP; ++m)
                                                 if (m < M) mine[m * kDecBN + c0 + j] += gacc[m];
                                         }
+                                    }
                                     }
                                 }
                             }
