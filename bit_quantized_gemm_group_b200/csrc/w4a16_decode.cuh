@@ -248,7 +248,9 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG, SP, OUT>::THR
                         if (sok && !mbar_wait_backoff(&full[stage], phase)) sok = false;
                         if (sok) {
                             const uint8_t* st = ring + stage * L::STAGE;
-#pragma unroll
+                            // groups one at a time: the side code stays small beside the
+                            // consumers' loop in the instruction cache
+#pragma unroll 1
                             for (int gg = 0; gg < (GPS + 1) / 2; ++gg) {
                                 const int gi = 2 * gg + sw;
                                 if (gi < ng) {
