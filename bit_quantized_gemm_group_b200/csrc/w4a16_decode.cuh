@@ -289,8 +289,11 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG, SP, OUT>::THR
                                             else mine[c0 + j] += g1;
                                         }
                                     } else {
-#pragma unroll
+                                    // the four columns one at a time when the sums live in shared
+                                    // memory (more than 8 tokens): a quarter of the code
+#pragma unroll(SREG ? 4 : 1)
                                     for (int j = 0; j < 4; ++j) {
+                                        const float sj = (j & 2) ? ((j & 1) ? s4.w : s4.z) : ((j & 1) ? s4.y : s4.x);
                                         float gacc[MP];
 #pragma unroll
                                         for (int m = 0; m < MP; ++m) gacc[m] = SREG ? sacc[j][SREG ? m : 0] : 0.0f;
@@ -298,7 +301,7 @@ __global__ void __launch_bounds__(DecodeSmem<MT, NW, GPS, ST, PWG, SP, OUT>::THR
                                         for (int r = 0; r < kDecOutMax; ++r) {
                                             if (r < cnt) {
                                                 int k = (int)((i4[r] >> (8 * j)) & 0xFFu);
-                                                const float w = __fmul_rn(i2f_small((uint32_t)(int32_t)(int8_t)((q4[r] >> (8 * j)) & 0xFFu)), s8v[j]);
+                                                const float w = __fmul_rn(i2f_small((uint32_t)(int32_t)(int8_t)((q4[r] >> (8 * j)) & 0xFFu)), sj);
                                                 if (k >= kDecBN) {  // not an offset inside the group: skipped, reported
                                                     bad = true;
                                                     continue;
