@@ -170,6 +170,15 @@ def test_workspace_size_and_too_small_workspace():
     assert L.qg_workspace_size(2, 17, 4096, 11008) > 0     # W4A8 at 17..127 tokens: stream-K partials
     assert L.qg_workspace_size(2, 16, 4096, 11008) == 0    # W4A8 at 16 tokens and fewer: split-K, none
     assert L.qg_workspace_size(2, 128, 4096, 11008) == 0   # W4A8 tile kernel takes none
+    # the int8 stream-K kernels finish split slabs in the launch: one 64-bit publication
+    # token per CTA (padded to 256 B), then one published NT x 128 tile of 4-byte sums per
+    # CTA, NT the token tile (16 / 32 / 64 / 128); the plan has one CTA per SM (148 when
+    # no GPU answers the query, as here or on a B200)
+    tok = (148 * 8 + 255) // 256 * 256
+    for M, nt in ((1, 16), (16, 16), (17, 32), (32, 32), (64, 64), (100, 128)):
+        assert L.qg_workspace_size(1, M, 4096, 11008) == tok + 148 * nt * 128 * 4
+    for M, nt in ((17, 32), (64, 64)):
+        assert L.qg_workspace_size(2, M, 8192, 8192) == tok + 148 * nt * 128 * 4
     assert L.qg_workspace_size(0, 0, 4096, 4096) == 0
     # AWQ search: every buffer of one candidate, so at least codes + packed + outputs
     K, N, Mc = 4096, 12288, 512
