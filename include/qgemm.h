@@ -191,8 +191,9 @@ qg_status qg_smooth_quant_act_i8(const uint16_t* X, int M, int K, const float* i
  *   per-launch 64-bit publication tokens and the int32 partial sums of column slabs
  *   split between CTAs, which the CTA holding a slab's first block adds in the same
  *   launch).  With it, M < 128 runs the stream-K tensor-core kernel (one launch); without
- *   it, the cluster split-K kernel.  Both give the same bits.  A workspace smaller than required -> QG_ERR_WORKSPACE before any
- *   launch.  Calls that may run concurrently need workspaces of their own.
+ *   it, the cluster split-K kernel.  Both give the same bits.  A workspace smaller than
+ *   required -> QG_ERR_WORKSPACE before any launch.  Calls that may run concurrently need
+ *   workspaces of their own.
  * ------------------------------------------------------------------------ */
 qg_status qg_gemm_w8a8(const int8_t* Xq, const float* t, int M, int K, const int8_t* Wq,
                        const float* sw, int N, uint16_t* Y, int32_t* acc_dbg, void* workspace,
@@ -214,10 +215,10 @@ qg_status qg_gemm_w8a8(const int8_t* Xq, const float* t, int M, int K, const int
  *   between CTAs, added in CTA order by the CTA holding a slab's first group in the same
  *   launch; the size is 0, and any workspace is ignored, for M <= 16 and M >= 128).
  *   With it, 17 <= M < 128 runs the stream-K tensor-core kernel (one launch per chunk)
- *   on chunks of up to 64 tokens; without it (and always at
- *   M <= 16), the cluster split-K kernel.  P is exact either way; Y may differ in the last bit
- *   (fp32 summation order).  A workspace smaller than required -> QG_ERR_WORKSPACE
- *   before any launch.  Calls that may run concurrently need workspaces of their own.
+ *   on chunks of up to 64 tokens; without it (and always at M <= 16), the cluster
+ *   split-K kernel.  P is exact either way; Y may differ in the last bit (fp32 summation
+ *   order).  A workspace smaller than required -> QG_ERR_WORKSPACE before any launch.
+ *   Calls that may run concurrently need workspaces of their own.
  * ------------------------------------------------------------------------ */
 qg_status qg_gemm_w4a8(const int8_t* Xq, const float* t, int M, int K, const uint32_t* packed,
                        const float* sg, int N, int group, uint16_t* Y, int32_t* part_dbg,
