@@ -968,7 +968,8 @@ def main():
             "gpu_launches": sweep.launches_per_step() * args.steps,
             "clocks": ck,
             "tflops": sweep.flops_per_step() / (ms_step * 1e-3) / 1e12,
-            "per_call": [{k: (round(v, 3) if isinstance(v, float) else v) for k, v in c.items()} for c in calls],
+            "per_call": [dict({k: (round(v, 3) if isinstance(v, float) else v) for k, v in c.items()},
+                              roofline_frac=round(c["gbs"] / pk["hbm_gbs"], 3)) for c in calls],
             "configs": configs,
         }
         print(json.dumps(line), flush=True)
