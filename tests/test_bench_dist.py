@@ -60,3 +60,16 @@ def test_whole_job_aggregate_is_weak_scaling():
     assert one == pytest.approx(4.0e8 * 100 / 26.0e-3 / 1e9)
     assert two == pytest.approx(2 * one)  # same per-rank work and time: twice the bytes
     assert bench.max_over_ranks(3.5, 1) == 3.5  # one rank: no collective
+
+
+def test_rotations_cover_twice_the_l2(monkeypatch):
+    """The bench protocol: the input copies a timed graph rotates over together exceed
+    2x L2 (126 MB on a B200), for inputs from a few KB to more than L2 itself."""
+    sys.path.insert(0, ROOT)
+    import bench
+    L2 = 126 * 2**20
+    monkeypatch.setattr(bench, "l2_bytes", lambda: L2)
+    for by in (1, 4096, 8 * 2**20, 25 * 2**20 + 7, 2 * L2 - 1, 2 * L2, 5 * L2):
+        n = bench.rotations_for(by)
+        assert n >= 1 and (n * by >= 2 * L2 or n == 1 and by >= 2 * L2)
+        assert (n - 1) * by < 2 * L2  # no more copies than needed
