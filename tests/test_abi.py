@@ -127,6 +127,28 @@ def test_gemm_w4a16_rejects(args, want):
     ("qg_gemm_w4a16_24", (None, 1, 0, 256, 16, None, None, None, None, 128, None, None), 0),
     ("qg_gemm_w4a16_24", (A, 1, 1, 256, 16, A, None, A, A, 128, A, None), 1),
     ("qg_gemm_w4a16_24", (A, 1, 1, 256, 16, A, A, A, A, 128, B, None), 3),
+    # gptq_blocked(Xcal, Mc, K, W, N, group, damp, codes, scales, zeros, ws, ws_bytes, stream)
+    ("qg_gptq_blocked", (A, 16, 256, A, 64, 100, 0.01, A, A, A, A, 1 << 40, None), 2),    # group % 8
+    ("qg_gptq_blocked", (A, 16, 200, A, 64, 128, 0.01, A, A, A, A, 1 << 40, None), 2),    # K % group
+    ("qg_gptq_blocked", (A, 16, 32768, A, 64, 128, 0.01, A, A, A, A, 1 << 40, None), 2),  # K > 16384
+    ("qg_gptq_blocked", (A, 16, 256, A, 64, 128, 0.0, A, A, A, A, 1 << 40, None), 2),     # damp must be > 0
+    ("qg_gptq_blocked", (A, 16, 256, A, 64, 128, 0.01, A, A, A, None, 0, None), 1),       # workspace required
+    ("qg_gptq_blocked", (A, 16, 256, A, 64, 128, 0.01, A, A, A, A, 1000, None), 10),      # too small
+    ("qg_gptq_blocked", (A, 16, 256, A, 64, 128, 0.01, A, B, A, A, 1 << 40, None), 3),
+    # pack24_tc(vals, K, N, vals_tc, stream)
+    ("qg_pack24_tc", (None, 256, 16, A, None), 1),
+    ("qg_pack24_tc", (A, 200, 16, A, None), 2),                                # K % 128
+    ("qg_pack24_tc", (A, 256, 16, A, None), 2),                                # not in place
+    ("qg_pack24_tc", (A, 256, 16, B, None), 3),
+    # gemm_w4a16_24_tc(X, xdt, M, K, N, vals_tc, meta, scales, zeros, group, Y, ws, ws_bytes, stream)
+    ("qg_gemm_w4a16_24_tc", (A, 9, 1, 256, 32, A, A, A, A, 128, A, A, 1 << 30, None), 4),
+    ("qg_gemm_w4a16_24_tc", (A, 1, 1, 256, 16, A, A, A, A, 128, A, A, 1 << 30, None), 2),   # N % 32
+    ("qg_gemm_w4a16_24_tc", (A, 1, 1, 192, 32, A, A, A, A, 128, A, A, 1 << 30, None), 2),   # K % 128
+    ("qg_gemm_w4a16_24_tc", (A, 1, 1, 256, 32, A, A, A, A, 64, A, A, 1 << 30, None), 2),    # group 128 only
+    ("qg_gemm_w4a16_24_tc", (None, 1, 0, 256, 32, None, None, None, None, 128, None, None, 0, None), 0),
+    ("qg_gemm_w4a16_24_tc", (A, 1, 1, 256, 32, A, A, A, A, 128, A, None, 0, None), 1),      # workspace required
+    ("qg_gemm_w4a16_24_tc", (A, 1, 1, 256, 32, A, A, A, A, 128, B, A, 1 << 30, None), 3),
+    ("qg_gemm_w4a16_24_tc", (A, 1, 1, 256, 32, A, A, A, A, 128, A, A, 100, None), 10),      # too small
     ("qg_awq_act_mean", (A, 0, 16, A, None), 2),
     ("qg_awq_act_mean", (None, 4, 16, A, None), 1),
     ("qg_awq_act_mean", (A, 4, 16, B, None), 3),
